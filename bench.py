@@ -1,0 +1,401 @@
+#!/usr/bin/env python
+"""Benchmark of the fused NA2D forward (queries*heads per second).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+One step is one ``na2d_forward`` call per shape of the workload over one batch
+of synthetic input (default: the NAT-Tiny stage-1 shape, B=32 heads=2 56x56
+D=32 k=7 d=1, fp16).  Inputs are resident in HBM before timing; between steps
+the benchmark rotates through enough distinct input/output sets that their
+total exceeds 3x the L2 cache, so every step reads from HBM.  Steps are
+replayed from CUDA graphs and timed with CUDA events on the launching stream.
+
+For N > 1 (launched by torch.distributed.run) every rank processes its own
+batch (weak scaling, no collective on the data path); the time is the maximum
+over ranks.
+
+``--impl reference`` times the fp64 CPU oracle on the host cores instead, on a
+bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+from pathlib import Path
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+from neighborhood_attention_na2d_b200.inputs import HEADLINE, WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "NA2D forward queries·heads/sec (GB/s, % HBM roofline) at NAT/DiNAT shapes"
+UNIT = "queries*heads/s"
+FALLBACK_HBM_GBS = 6650.0
+PEAKS_FILE = ROOT / "MEASURED_PEAKS.json"
+PROFILES = ROOT / "profiles"
+KERNEL_SOURCES = ["neighborhood_attention_na2d_b200/csrc/na2d_tc.cu",
+                  "neighborhood_attention_na2d_b200/csrc/na2d_device.cuh"]
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def kernel_sha() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        h.update((ROOT / p).read_bytes())
+    return h.hexdigest()[:16]
+
+
+def hbm_peak() -> tuple[float, str]:
+    try:
+        d = json.loads(PEAKS_FILE.read_text())
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def recorded_traffic(workload: str) -> int | None:
+    """DRAM bytes per launch from the committed ncu summary of this workload,
+    only if it was taken on the current kernel source."""
+    f = PROFILES / f"na2d_fwd_tc_{workload}.md"
+    if not f.exists():
+        return None
+    text = f.read_text()
+    m = re.search(r"traffic_per_launch_bytes\s*=\s*(\d+)\s*;\s*kernel_sha\s*=\s*([0-9a-f]+)", text)
+    if not m or m.group(2) != kernel_sha():
+        return None
+    return int(m.group(1))
+
+
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting",
+               0x10: "sync_boost", 0x1: "gpu_idle"}
+
+    def __init__(self, index: int):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # noqa: BLE001
+            log(f"clock sampling unavailable: {e}")
+        self._stop = threading.Event()
+
+    def _run(self):
+        nv = self.nv
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = get_reasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:  # noqa: BLE001
+                pass
+            self._stop.wait(0.01)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world and world > 1:
+        log(f"--gpus {args.gpus} but WORLD_SIZE {world}: using WORLD_SIZE")
+    return world, rank, local
+
+
+def run_reference(args, world, rank):
+    """The oracle on host cores, per step a bounded sample of the workload."""
+    if rank != 0:
+        return
+    import oracle
+
+    wl = WORKLOADS[args.workload]
+    threads = oracle.default_threads()
+    # sample: the first nb batch elements of every shape -- enough (batch, head)
+    # slices to occupy every host core; the step count is cut below if needed
+    # so the run stays within minutes
+    nb = max(1, min(min(s.B for s in wl.shapes), math.ceil(threads / min(s.heads for s in wl.shapes))))
+    threads = min(threads, nb * min(s.heads for s in wl.shapes))
+    arrays = [[t[:nb].double().numpy() if t.dim() == 5 else t.double().numpy() for t in make_inputs(s)]
+              for s in wl.shapes]
+    def step():
+        for s, (qq, kk, vv, rr) in zip(wl.shapes, arrays):
+            oracle.forward(qq, kk, vv, rr, s.k, s.d, nthreads=threads)
+    t0 = time.perf_counter()
+    step()
+    one = time.perf_counter() - t0
+    budget = 150.0
+    steps, warmup = args.steps, args.warmup
+    if (steps + warmup) * one > budget:
+        steps = max(1, int(budget / one) - warmup)
+        warmup = min(warmup, 3)
+    for _ in range(warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        step()
+    dt = (time.perf_counter() - t0) / steps
+    units = sum(nb * s.heads * s.H * s.W for s in wl.shapes)
+    value = units / dt
+    sample = f"first {nb} batch element(s) of each shape ({units} query*heads per step), fp64, all-host-core oracle"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps,
+        "warmup": warmup, "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(wl, world),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    if steps != args.steps:
+        line["note"] = f"steps reduced from {args.steps} to fit the CPU time budget"
+    print(json.dumps(line), flush=True)
+
+
+def config_dict(wl, world):
+    s0 = wl.shapes[0]
+    cfg = {"workload": wl.name, "shapes": [s.describe() for s in wl.shapes],
+           "B": s0.B, "heads": s0.heads, "H": s0.H, "W": s0.W, "D": s0.D, "k": s0.k, "d": s0.d,
+           "global_batch": s0.B * world, "parallelism": f"replicas{world}" if world > 1 else "single"}
+    return cfg
+
+
+def cpu_baseline(wl):
+    """The oracle as it stands on all host cores, one pass over a bounded sample."""
+    import oracle
+    threads = oracle.default_threads()
+    total_units, total_t = 0, 0.0
+    parts = []
+    for s in wl.shapes:
+        q, k, v, rpb = make_inputs(s)
+        nb = s.B
+        # bound the sample to about 10 s of CPU work: ~5 us of fp64 work per key*query on one core
+        est = s.B * s.heads * s.H * s.W * s.k * s.k * 5e-8
+        if est > 10.0:
+            nb = max(1, int(s.B * 10.0 / est))
+        arr = [t[:nb].double().numpy() for t in (q, k, v)] + [rpb.double().numpy()]
+        t0 = time.perf_counter()
+        oracle.forward(*arr, s.k, s.d, nthreads=threads)
+        total_t += time.perf_counter() - t0
+        total_units += nb * s.heads * s.H * s.W
+        parts.append(f"{nb}/{s.B} batch of {s.describe()}")
+    used = min(threads, min(s.B * s.heads for s in wl.shapes))
+    return {"value": total_units / total_t, "unit": UNIT, "cores": used, "kind": "oracle",
+            "sample": "; ".join(parts) + "; one pass, fp64"}
+
+
+def run_ours(args, world, rank, local):
+    import torch
+    import neighborhood_attention_na2d_b200 as na
+    from neighborhood_attention_na2d_b200 import _native
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = dist
+    na.lib()
+    wl = WORKLOADS[args.workload]
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    elem = {"f32": 4, "f16": 2, "bf16": 2}
+
+    # ---- resident input sets, rotated so that every step misses L2
+    set_bytes = sum(4 * s.B * s.heads * s.H * s.W * s.D * elem[s.dtype] for s in wl.shapes)
+    R = max(2, math.ceil(3 * l2 / set_bytes))
+    sets = []
+    for r in range(R):
+        one = []
+        for s in wl.shapes:
+            q, k, v, rpb = make_inputs(s, s.seed + 1000 * r + 100000 * rank)
+            q, k, v, rpb = (t.to(dev) for t in (q, k, v, rpb))
+            one.append((s, q, k, v, rpb, torch.empty_like(q)))
+        sets.append(one)
+    torch.cuda.synchronize()
+    log(f"rank {rank}: {R} input sets x {set_bytes / 1e6:.1f} MB (L2 {l2 / 1e6:.0f} MB)")
+
+    def step(r):
+        for (s, q, k, v, rpb, out) in sets[r % R]:
+            na.na2d_forward(q, k, v, rpb, s.k, s.d, out=out)
+
+    # ---- warm-up (eager), then capture graphs of whole rotations
+    for i in range(max(args.warmup, 3)):
+        step(i)
+    torch.cuda.synchronize()
+    per_graph = R * max(1, 64 // R)
+    graph = torch.cuda.CUDAGraph()
+    cap_stream = torch.cuda.Stream(dev)
+    cap_stream.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(cap_stream):
+        with torch.cuda.graph(graph, stream=cap_stream):
+            for i in range(per_graph):
+                step(i)
+    torch.cuda.synchronize()
+    for _ in range(2):
+        graph.replay()
+    torch.cuda.synchronize()
+
+    K = args.steps
+    full, rest = divmod(K, per_graph)
+    stream = torch.cuda.current_stream(dev)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        start.record(stream)
+        for _ in range(full):
+            graph.replay()
+        for i in range(rest):
+            step(i)
+        end.record(stream)
+        end.synchronize()
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end)
+    if pg:
+        t = torch.tensor([ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms = float(t.item())
+        pg.barrier()
+    ms_per_step = ms / K
+    units_rank = sum(s.B * s.heads * s.H * s.W for s in wl.shapes)
+    value = world * units_rank / (ms_per_step / 1e3)
+
+    # ---- roofline of the dominant kernel (the fused forward; one launch per shape per step)
+    alg_bytes = sum(s.algorithmic_bytes() for s in wl.shapes)
+    achieved = alg_bytes / (ms_per_step / 1e3) / 1e9
+    peak, peak_kind = hbm_peak()
+    roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+            "traffic": recorded_traffic(wl.name), "peak_source": f"{peak_kind} hbm_gbs (copy)",
+            "algorithmic_bytes_per_step": alg_bytes}
+
+    # ---- end to end through the public API: pinned host -> device, forward, device -> host
+    e2e = run_e2e(args, wl, dev, rank, world, pg)
+
+    cfg = config_dict(wl, world)
+    cfg.update({"l2": f"rotating {R} input sets ({R * set_bytes / 1e6:.0f} MB) > 3x L2 ({l2 / 1e6:.0f} MB)",
+                "timing": f"CUDA graphs of {per_graph} steps, CUDA events on the launching stream"})
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": wl.shapes[0].dtype, "data": "synthetic (seeded N(0,1) q/k/v, N(0,0.02) rpb)", "config": cfg,
+        "roofline": roof, "e2e": e2e, "gpu_launches": K * len(wl.shapes), "clocks": clocks.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl)
+    del graph
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(args, wl, dev, rank, world, pg):
+    import torch
+    import neighborhood_attention_na2d_b200 as na
+
+    host = []
+    h2d = d2h = 0
+    for s in wl.shapes:
+        q, k, v, rpb = make_inputs(s, s.seed + 100000 * rank)
+        hq, hk, hv, hr = (t.pin_memory() for t in (q, k, v, rpb))
+        dq, dk, dv, dr = (torch.empty_like(t, device=dev) for t in (q, k, v, rpb))
+        hout = torch.empty_like(q).pin_memory()
+        host.append((s, hq, hk, hv, hr, dq, dk, dv, dr, hout))
+        h2d += sum(t.numel() * t.element_size() for t in (q, k, v, rpb))
+        d2h += hout.numel() * hout.element_size()
+
+    def step():
+        for (s, hq, hk, hv, hr, dq, dk, dv, dr, hout) in host:
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            dr.copy_(hr, non_blocking=True)
+            out = na.na2d_forward(dq, dk, dv, dr, s.k, s.d)
+            hout.copy_(out, non_blocking=True)
+
+    n = max(5, min(50, args.steps))
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    stream = torch.cuda.current_stream(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(n):
+        step()
+    b.record(stream)
+    b.synchronize()
+    ms = a.elapsed_time(b)
+    if pg:
+        t = torch.tensor([ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms = float(t.item())
+    units = world * sum(s.B * s.heads * s.H * s.W for s in wl.shapes)
+    return {"value": units / (ms / n / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "steps": n, "api": "neighborhood_attention_na2d_b200.na2d_forward (C ABI na2d_forward)"}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=HEADLINE)
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed oracle leg")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+    else:
+        run_ours(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,120 @@
+/*
+ * na2d.h -- C ABI of libna2d: 2D (dilated) neighborhood attention (NA / DiNA)
+ * forward for NVIDIA B200 (sm_100a).
+ *
+ * The operation (web pages on NAT / DiNAT):
+ *   - "Neighborhood Attention Transformer" (README mirror, figure caption under
+ *     the abstract): each query pixel attends to its nearest k x k
+ *     neighbourhood; at the image edges the window stays inside the image;
+ *     with the window as large as the image this is plain dot-product self
+ *     attention.
+ *   - "Dilated Neighborhood Attention Transformer" (HF docs, overview; gitcode
+ *     DiNAT article, section "DiNAT 的核心思想"): DiNA takes every d-th pixel,
+ *     keeping k*k keys per query; the layer is
+ *         scores = natten2dqkrpb(q, k, rpb, kernel_size, dilation)
+ *         probs  = softmax(scores, dim=-1)
+ *         out    = natten2dav(probs, v, kernel_size, dilation)
+ *     which this library exports as na2d_qk_rpb, na2d_softmax and na2d_av, and
+ *     fused (no k*k tensor in memory) as na2d_forward.
+ *
+ * Window rule (NATTEN clamp rule), per axis, for coordinate i on an axis of
+ * length L, r = k / 2:
+ *     g = i mod d, i' = i / d, Lg = ceil((L - g) / d),
+ *     s' = clamp(i' - r, 0, Lg - k), keys g + d * (s' + t), t = 0 .. k-1.
+ * Score of key (ty, tx):
+ *     q . key / sqrt(D) + rpb[h, s'_y + ty - i'_y + k - 1, s'_x + tx - i'_x + k - 1]
+ * The neighbour index in the k*k axis of the split path is n = ty * k + tx.
+ *
+ * Layouts (all row-major, contiguous, innermost last):
+ *     q, k, v, out : [B, heads, H, W, D] in the problem's dtype
+ *     rpb          : [heads, 2k-1, 2k-1] in the problem's dtype, or NULL for
+ *                    a zero bias
+ *     attn         : [B, heads, H, W, k*k] fp32 (split path only)
+ *
+ * Ownership and threading: every buffer is a DEVICE pointer owned by the
+ * caller.  The library allocates no memory and keeps no per-call state; calls
+ * are asynchronous on `stream` (a cudaStream_t; NULL means the legacy default
+ * stream) and never synchronise the host.  Calls from several host threads
+ * are safe.  Outputs must not overlap inputs.
+ *
+ * Errors: every argument check runs on the host before any launch; a failing
+ * check returns its status and launches nothing.  A failed launch returns
+ * NA2D_ERR_CUDA (the CUDA error is cleared with cudaGetLastError).  Nothing
+ * in the library aborts, traps or prints.
+ *
+ * Supported set: dtype f32 / f16 / bf16; D = 32; odd k in [1, 13]; d >= 1;
+ * H >= k*d and W >= k*d (every dilation group holds at least k positions);
+ * B, heads >= 0 (an empty problem returns NA2D_OK without a launch);
+ * B*heads*H*W*max(D, k*k) < 2^62; H*W*max(D, k*k) < 2^31; tensor pointers
+ * 16-byte aligned (rpb: element aligned).  Arithmetic: fp32 accumulation for
+ * every dtype; f16 / bf16 outputs are rounded to nearest even.
+ */
+#ifndef NA2D_H
+#define NA2D_H
+
+#if defined(__GNUC__)
+#define NA2D_API __attribute__((visibility("default")))
+#else
+#define NA2D_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    NA2D_OK = 0,
+    NA2D_ERR_NULL = 1,      /* a required pointer (problem, q, k, v, out, attn) is NULL */
+    NA2D_ERR_DTYPE = 2,     /* dtype is not one of na2d_dtype */
+    NA2D_ERR_SHAPE = 3,     /* negative B/heads, H or W < 1, H < k*d or W < k*d,
+                               D other than 32, or a size limit exceeded */
+    NA2D_ERR_KERNEL = 4,    /* k even, < 1 or > 13 */
+    NA2D_ERR_DILATION = 5,  /* d < 1 */
+    NA2D_ERR_ALIGN = 6,     /* q, k, v, out or attn not 16-byte aligned, rpb not element aligned */
+    NA2D_ERR_ALIAS = 7,     /* an output buffer overlaps an input buffer */
+    NA2D_ERR_CUDA = 8,      /* a CUDA runtime call or kernel launch failed */
+    NA2D_ERR_INTERNAL = 9   /* an internal consistency check failed */
+} na2d_status;
+
+typedef enum { NA2D_F32 = 0, NA2D_F16 = 1, NA2D_BF16 = 2 } na2d_dtype;
+
+/* One problem.  The softmax scale is fixed at 1/sqrt(D). */
+typedef struct {
+    int B;            /* batch */
+    int heads;        /* attention heads */
+    int H, W;         /* feature map height and width */
+    int D;            /* head dim (32) */
+    int k;            /* kernel size: odd, 1..13 */
+    int d;            /* dilation: >= 1 */
+    na2d_dtype dtype; /* element type of q, k, v, rpb and out */
+} na2d_problem;
+
+/* Scores (natten2dqkrpb): attn[b,h,i,j,n] = q.key_n / sqrt(D) + rpb bias, fp32.
+ * q, k: [B,heads,H,W,D]; rpb: [heads,2k-1,2k-1] or NULL; attn: [B,heads,H,W,k*k]. */
+NA2D_API na2d_status na2d_qk_rpb(const na2d_problem *p, const void *q, const void *k, const void *rpb,
+                        float *attn, void *stream);
+
+/* Softmax over the last (k*k) axis of attn, in place (dim=-1 softmax). */
+NA2D_API na2d_status na2d_softmax(const na2d_problem *p, float *attn, void *stream);
+
+/* Weighted sum (natten2dav): out[b,h,i,j,:] = sum_n attn[b,h,i,j,n] * v[key_n].
+ * attn: [B,heads,H,W,k*k] fp32; v, out: [B,heads,H,W,D] in the problem's dtype. */
+NA2D_API na2d_status na2d_av(const na2d_problem *p, const float *attn, const void *v, void *out,
+                    void *stream);
+
+/* Fused forward: out = softmax(q.key/sqrt(D) + rpb) . v over each query's k*k
+ * (dilated) window, in one kernel; no k*k tensor is written to memory. */
+NA2D_API na2d_status na2d_forward(const na2d_problem *p, const void *q, const void *k, const void *v,
+                         const void *rpb, void *out, void *stream);
+
+/* A static, human-readable name for a status. */
+NA2D_API const char *na2d_status_str(na2d_status s);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+NA2D_API int na2d_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NA2D_H */

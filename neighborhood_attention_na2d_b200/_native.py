@@ -1,0 +1,89 @@
+"""ctypes view of ``libna2d.so`` -- the C ABI declared in ``include/na2d.h``.
+
+Marshalling only: structures, prototypes and the status type.  Every step of
+the computation runs in the library's CUDA kernels; nothing here computes.
+"""
+from __future__ import annotations
+
+import ctypes
+from pathlib import Path
+
+LIB_PATH = Path(__file__).resolve().parent / "libna2d.so"
+
+NA2D_F32, NA2D_F16, NA2D_BF16 = 0, 1, 2
+
+STATUS_NAMES = {
+    0: "NA2D_OK", 1: "NA2D_ERR_NULL", 2: "NA2D_ERR_DTYPE", 3: "NA2D_ERR_SHAPE", 4: "NA2D_ERR_KERNEL",
+    5: "NA2D_ERR_DILATION", 6: "NA2D_ERR_ALIGN", 7: "NA2D_ERR_ALIAS", 8: "NA2D_ERR_CUDA", 9: "NA2D_ERR_INTERNAL",
+}
+
+# every symbol the header declares
+EXPORTS = ("na2d_qk_rpb", "na2d_softmax", "na2d_av", "na2d_forward", "na2d_status_str", "na2d_version")
+
+
+class Problem(ctypes.Structure):
+    """``na2d_problem``: one problem description (scale fixed at 1/sqrt(D))."""
+    _fields_ = [("B", ctypes.c_int), ("heads", ctypes.c_int), ("H", ctypes.c_int), ("W", ctypes.c_int),
+                ("D", ctypes.c_int), ("k", ctypes.c_int), ("d", ctypes.c_int), ("dtype", ctypes.c_int)]
+
+
+class Na2dError(RuntimeError):
+    """A non-OK ``na2d_status`` returned by the library."""
+
+    def __init__(self, status: int, what: str, message: str):
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)} ({message})")
+        self.status = status
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library.  Raises if it has not been built: there is no
+    fallback implementation."""
+    global _lib
+    if _lib is None:
+        if not LIB_PATH.exists():
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m neighborhood_attention_na2d_b200.build`")
+        L = ctypes.CDLL(str(LIB_PATH))
+        P, vp, fp = ctypes.POINTER(Problem), ctypes.c_void_p, ctypes.c_void_p
+        L.na2d_qk_rpb.argtypes = [P, vp, vp, vp, fp, vp]
+        L.na2d_softmax.argtypes = [P, fp, vp]
+        L.na2d_av.argtypes = [P, fp, vp, vp, vp]
+        L.na2d_forward.argtypes = [P, vp, vp, vp, vp, vp, vp]
+        for f in ("na2d_qk_rpb", "na2d_softmax", "na2d_av", "na2d_forward"):
+            getattr(L, f).restype = ctypes.c_int
+        L.na2d_status_str.argtypes = [ctypes.c_int]
+        L.na2d_status_str.restype = ctypes.c_char_p
+        L.na2d_version.argtypes = []
+        L.na2d_version.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def status_str(status: int) -> str:
+    return lib().na2d_status_str(status).decode()
+
+
+def check(status: int, what: str) -> None:
+    if status != 0:
+        raise Na2dError(status, what, status_str(status))
+
+
+# Raw-pointer calls (integers are device addresses; stream is a cudaStream_t
+# handle as an int, 0 for the legacy default stream).  They return the status.
+def forward_ptr(p: Problem, q: int, k: int, v: int, rpb: int | None, out: int, stream: int = 0) -> int:
+    return lib().na2d_forward(ctypes.byref(p), q, k, v, rpb, out, stream)
+
+
+def qk_rpb_ptr(p: Problem, q: int, k: int, rpb: int | None, attn: int, stream: int = 0) -> int:
+    return lib().na2d_qk_rpb(ctypes.byref(p), q, k, rpb, attn, stream)
+
+
+def softmax_ptr(p: Problem, attn: int, stream: int = 0) -> int:
+    return lib().na2d_softmax(ctypes.byref(p), attn, stream)
+
+
+def av_ptr(p: Problem, attn: int, v: int, out: int, stream: int = 0) -> int:
+    return lib().na2d_av(ctypes.byref(p), attn, v, out, stream)

@@ -1,0 +1,146 @@
+// na2d_abi.cu -- the extern "C" entry points declared in include/na2d.h:
+// host-side argument checks, then one launch on the caller's stream.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "../../include/na2d.h"
+#include "na2d_launch.h"
+
+namespace {
+
+using na2d::DType;
+using na2d::Problem;
+
+constexpr int64_t kMaxTotal = (int64_t)1 << 62;
+constexpr int64_t kMaxPlane = ((int64_t)1 << 31) - 1;
+
+size_t elem_size(na2d_dtype t) { return t == NA2D_F32 ? 4 : 2; }
+
+bool aligned16(const void *ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+bool overlap(const void *a, size_t na, const void *b, size_t nb) {
+    if (!a || !b || na == 0 || nb == 0) return false;
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+    return a0 < b0 + nb && b0 < a0 + na;
+}
+
+// Checks the problem description itself.  On success fills `out` and reports
+// whether the problem is empty (B or heads zero: nothing to launch).
+na2d_status check_problem(const na2d_problem *p, Problem *out, bool *empty) {
+    if (!p) return NA2D_ERR_NULL;
+    if (p->dtype != NA2D_F32 && p->dtype != NA2D_F16 && p->dtype != NA2D_BF16) return NA2D_ERR_DTYPE;
+    if (p->k < 1 || p->k > 13 || (p->k % 2) == 0) return NA2D_ERR_KERNEL;
+    if (p->d < 1) return NA2D_ERR_DILATION;
+    if (p->B < 0 || p->heads < 0 || p->H < 1 || p->W < 1) return NA2D_ERR_SHAPE;
+    if (p->D != 32) return NA2D_ERR_SHAPE;
+    // every dilation group must hold at least k positions: floor(L / d) >= k
+    if ((int64_t)p->k * p->d > p->H || (int64_t)p->k * p->d > p->W) return NA2D_ERR_SHAPE;
+    const int64_t inner = (int64_t)(p->D > p->k * p->k ? p->D : p->k * p->k);
+    const int64_t plane = (int64_t)p->H * p->W * inner;
+    if (plane > kMaxPlane) return NA2D_ERR_SHAPE;
+    const int64_t bh = (int64_t)p->B * p->heads;
+    if (bh > 0 && bh > kMaxTotal / plane) return NA2D_ERR_SHAPE;
+    *out = Problem{p->B, p->heads, p->H, p->W, p->D, p->k, p->d, static_cast<DType>(p->dtype)};
+    *empty = (bh == 0);
+    return NA2D_OK;
+}
+
+size_t tensor_bytes(const na2d_problem *p) {
+    return (size_t)p->B * p->heads * p->H * p->W * p->D * elem_size(p->dtype);
+}
+size_t attn_bytes(const na2d_problem *p) { return (size_t)p->B * p->heads * p->H * p->W * p->k * p->k * 4; }
+size_t rpb_bytes(const na2d_problem *p) {
+    return (size_t)p->heads * (2 * p->k - 1) * (2 * p->k - 1) * elem_size(p->dtype);
+}
+
+bool rpb_aligned(const na2d_problem *p, const void *rpb) {
+    return !rpb || (reinterpret_cast<uintptr_t>(rpb) % elem_size(p->dtype)) == 0;
+}
+
+na2d_status from_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return NA2D_OK;
+    cudaGetLastError();   // clear a sticky launch error for the caller's next call
+    return NA2D_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+na2d_status na2d_forward(const na2d_problem *p, const void *q, const void *k, const void *v, const void *rpb,
+                         void *out, void *stream) {
+    Problem pr;
+    bool empty = false;
+    na2d_status s = check_problem(p, &pr, &empty);
+    if (s != NA2D_OK) return s;
+    if (empty) return NA2D_OK;
+    if (!q || !k || !v || !out) return NA2D_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !rpb_aligned(p, rpb))
+        return NA2D_ERR_ALIGN;
+    const size_t n = tensor_bytes(p);
+    if (overlap(out, n, q, n) || overlap(out, n, k, n) || overlap(out, n, v, n) || overlap(out, n, rpb, rpb_bytes(p)))
+        return NA2D_ERR_ALIAS;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (na2d::tc_supported(pr)) return from_cuda(na2d::launch_forward_tc(pr, q, k, v, rpb, out, st));
+    return from_cuda(na2d::launch_forward_simt(pr, q, k, v, rpb, out, st));
+}
+
+na2d_status na2d_qk_rpb(const na2d_problem *p, const void *q, const void *k, const void *rpb, float *attn,
+                        void *stream) {
+    Problem pr;
+    bool empty = false;
+    na2d_status s = check_problem(p, &pr, &empty);
+    if (s != NA2D_OK) return s;
+    if (empty) return NA2D_OK;
+    if (!q || !k || !attn) return NA2D_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(attn) || !rpb_aligned(p, rpb)) return NA2D_ERR_ALIGN;
+    const size_t n = tensor_bytes(p), na = attn_bytes(p);
+    if (overlap(attn, na, q, n) || overlap(attn, na, k, n) || overlap(attn, na, rpb, rpb_bytes(p)))
+        return NA2D_ERR_ALIAS;
+    return from_cuda(na2d::launch_qk_rpb(pr, q, k, rpb, attn, static_cast<cudaStream_t>(stream)));
+}
+
+na2d_status na2d_softmax(const na2d_problem *p, float *attn, void *stream) {
+    Problem pr;
+    bool empty = false;
+    na2d_status s = check_problem(p, &pr, &empty);
+    if (s != NA2D_OK) return s;
+    if (empty) return NA2D_OK;
+    if (!attn) return NA2D_ERR_NULL;
+    if (!aligned16(attn)) return NA2D_ERR_ALIGN;
+    return from_cuda(na2d::launch_softmax(pr, attn, static_cast<cudaStream_t>(stream)));
+}
+
+na2d_status na2d_av(const na2d_problem *p, const float *attn, const void *v, void *out, void *stream) {
+    Problem pr;
+    bool empty = false;
+    na2d_status s = check_problem(p, &pr, &empty);
+    if (s != NA2D_OK) return s;
+    if (empty) return NA2D_OK;
+    if (!attn || !v || !out) return NA2D_ERR_NULL;
+    if (!aligned16(attn) || !aligned16(v) || !aligned16(out)) return NA2D_ERR_ALIGN;
+    const size_t n = tensor_bytes(p);
+    if (overlap(out, n, v, n) || overlap(out, n, attn, attn_bytes(p))) return NA2D_ERR_ALIAS;
+    return from_cuda(na2d::launch_av(pr, attn, v, out, static_cast<cudaStream_t>(stream)));
+}
+
+const char *na2d_status_str(na2d_status s) {
+    switch (s) {
+    case NA2D_OK: return "ok";
+    case NA2D_ERR_NULL: return "null pointer";
+    case NA2D_ERR_DTYPE: return "unsupported dtype";
+    case NA2D_ERR_SHAPE: return "unsupported shape";
+    case NA2D_ERR_KERNEL: return "unsupported kernel size";
+    case NA2D_ERR_DILATION: return "unsupported dilation";
+    case NA2D_ERR_ALIGN: return "misaligned pointer";
+    case NA2D_ERR_ALIAS: return "output overlaps an input";
+    case NA2D_ERR_CUDA: return "CUDA error";
+    case NA2D_ERR_INTERNAL: return "internal error";
+    }
+    return "unknown status";
+}
+
+int na2d_version(void) { return 100; }
+
+}  // extern "C"

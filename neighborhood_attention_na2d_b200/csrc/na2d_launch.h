@@ -1,0 +1,34 @@
+// na2d_launch.h -- host-side launchers behind the C ABI (internal).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace na2d {
+
+enum class DType { F32 = 0, F16 = 1, BF16 = 2 };
+
+struct Problem {
+    int B, heads, H, W, D, k, d;
+    DType dtype;
+    int64_t bh() const { return (int64_t)B * heads; }
+};
+
+// Fused forward on the tensor cores (f16 / bf16, D = 32, k in 3..13).
+cudaError_t launch_forward_tc(const Problem &p, const void *q, const void *k, const void *v,
+                              const void *rpb, void *out, cudaStream_t stream);
+
+// Fused forward on the CUDA cores (any dtype, D = 32, any odd k <= 13).
+cudaError_t launch_forward_simt(const Problem &p, const void *q, const void *k, const void *v,
+                                const void *rpb, void *out, cudaStream_t stream);
+
+// Split path.
+cudaError_t launch_qk_rpb(const Problem &p, const void *q, const void *k, const void *rpb, float *attn,
+                          cudaStream_t stream);
+cudaError_t launch_softmax(const Problem &p, float *attn, cudaStream_t stream);
+cudaError_t launch_av(const Problem &p, const float *attn, const void *v, void *out, cudaStream_t stream);
+
+// True when launch_forward_tc handles this problem.
+bool tc_supported(const Problem &p);
+
+}  // namespace na2d

@@ -1,0 +1,130 @@
+"""The C-ABI library on the host (no GPU needed): it loads, exports exactly what
+include/na2d.h declares, and rejects bad arguments before any CUDA call.
+
+The argument checks pass fake, never-dereferenced addresses.  They run in a
+child process with CUDA_VISIBLE_DEVICES set empty, so even a case that wrongly
+passed the checks could not launch a kernel on a real device.
+"""
+import json
+import os
+import re
+import subprocess
+import sys
+from pathlib import Path
+
+import pytest
+
+from neighborhood_attention_na2d_b200 import _native
+from neighborhood_attention_na2d_b200.build import build
+
+ROOT = Path(__file__).resolve().parent.parent
+HEADER = ROOT / "include" / "na2d.h"
+FAKE = 0x10000          # 16-byte aligned, never dereferenced
+FAKE2 = 0x200000
+
+BAD_PROBLEMS = [
+    (dict(k=6), 4), (dict(k=0), 4), (dict(k=15), 4), (dict(k=-3), 4),
+    (dict(d=0), 5), (dict(d=-1), 5),
+    (dict(H=13, d=2), 3), (dict(W=13, d=2), 3), (dict(H=6), 3), (dict(W=6), 3),
+    (dict(H=0), 3), (dict(B=-1), 3), (dict(heads=-2), 3),
+    (dict(D=64), 3), (dict(D=16), 3),
+    (dict(dtype=7), 2),
+    (dict(H=1 << 20, W=1 << 20, k=1), 3),  # plane too large
+]
+
+
+def prob(**kw):
+    base = dict(B=2, heads=2, H=14, W=14, D=32, k=7, d=1, dtype=_native.NA2D_F16)
+    base.update(kw)
+    return _native.Problem(**base)
+
+
+def _host_checks() -> dict:
+    """Runs in the child process: every call must fail (or be empty) on the host."""
+    r = {}
+    for i, (kw, _) in enumerate(BAD_PROBLEMS):
+        r[f"bad{i}"] = _native.forward_ptr(prob(**kw), FAKE, FAKE, FAKE, None, FAKE2)
+    p = prob()
+    L = _native.lib()
+    r["null_problem"] = L.na2d_forward(None, FAKE, FAKE, FAKE, None, FAKE2, None)
+    r["null_q"] = _native.forward_ptr(p, 0, FAKE, FAKE, None, FAKE2)
+    r["null_out"] = _native.forward_ptr(p, FAKE, FAKE, FAKE, None, 0)
+    r["null_qk_k"] = _native.qk_rpb_ptr(p, FAKE, 0, None, FAKE2)
+    r["null_softmax"] = _native.softmax_ptr(p, 0)
+    r["null_av_v"] = _native.av_ptr(p, FAKE, 0, FAKE2)
+    r["align_q"] = _native.forward_ptr(p, FAKE + 8, FAKE, FAKE, None, FAKE2)
+    r["align_rpb"] = _native.forward_ptr(p, FAKE, FAKE, FAKE, FAKE + 1, FAKE2)
+    r["align_attn"] = _native.qk_rpb_ptr(p, FAKE, FAKE, None, FAKE2 + 4)
+    r["align_softmax"] = _native.softmax_ptr(p, FAKE + 4)
+    r["align_av"] = _native.av_ptr(p, FAKE + 4, FAKE, FAKE2)
+    nbytes = 2 * 2 * 14 * 14 * 32 * 2
+    r["alias_out_q"] = _native.forward_ptr(p, FAKE, FAKE2, FAKE2, None, FAKE)
+    r["alias_partial"] = _native.forward_ptr(p, FAKE, FAKE, FAKE, None, FAKE + nbytes - 16)
+    r["alias_av"] = _native.av_ptr(p, FAKE, FAKE2, FAKE2)
+    r["empty_B"] = _native.forward_ptr(prob(B=0), 0, 0, 0, None, 0)
+    r["empty_heads"] = _native.forward_ptr(prob(heads=0), 0, 0, 0, None, 0)
+    r["empty_qk"] = _native.qk_rpb_ptr(prob(B=0), 0, 0, None, 0)
+    r["empty_softmax"] = _native.softmax_ptr(prob(B=0), 0)
+    r["empty_av"] = _native.av_ptr(prob(B=0), 0, 0, 0)
+    return r
+
+
+@pytest.fixture(scope="module")
+def host_results():
+    build()
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    code = ("import json, sys; sys.path[:0] = [%r, %r]; import test_abi_host as t; "
+            "print(json.dumps(t._host_checks()))") % (str(ROOT), str(Path(__file__).parent))
+    out = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stderr
+    return json.loads(out.stdout.strip().splitlines()[-1])
+
+
+def header_functions():
+    text = HEADER.read_text()
+    return sorted(set(re.findall(r"NA2D_API\s+[\w\s\*]+?\b(na2d_\w+)\s*\(", text)))
+
+
+def test_exports_match_header():
+    build()
+    lib = _native.lib()
+    declared = header_functions()
+    assert declared == sorted(_native.EXPORTS)
+    out = subprocess.run(["nm", "-D", "--defined-only", str(_native.LIB_PATH)], capture_output=True, text=True,
+                         check=True).stdout
+    exported = sorted({ln.split()[-1] for ln in out.splitlines() if ln.split() and ln.split()[-1].startswith("na2d")})
+    assert exported == declared          # nothing internal leaks, nothing is missing
+    for name in declared:
+        assert hasattr(lib, name)
+
+
+def test_version_and_status_strings():
+    build()
+    assert _native.lib().na2d_version() == 100
+    names = [_native.status_str(s) for s in range(10)]
+    assert names[0] == "ok" and len(set(names)) == 10
+    assert _native.status_str(99) == "unknown status"
+
+
+@pytest.mark.parametrize("i", range(len(BAD_PROBLEMS)))
+def test_forward_rejects_bad_problems(host_results, i):
+    assert host_results[f"bad{i}"] == BAD_PROBLEMS[i][1], BAD_PROBLEMS[i][0]
+
+
+@pytest.mark.parametrize("case,status", [
+    ("null_problem", 1), ("null_q", 1), ("null_out", 1), ("null_qk_k", 1), ("null_softmax", 1), ("null_av_v", 1),
+    ("align_q", 6), ("align_rpb", 6), ("align_attn", 6), ("align_softmax", 6), ("align_av", 6),
+    ("alias_out_q", 7), ("alias_partial", 7), ("alias_av", 7),
+    ("empty_B", 0), ("empty_heads", 0), ("empty_qk", 0), ("empty_softmax", 0), ("empty_av", 0),
+])
+def test_host_checks(host_results, case, status):
+    assert host_results[case] == status
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    import neighborhood_attention_na2d_b200 as na
+    build()
+    x = torch.zeros(1, 1, 7, 7, 32, dtype=torch.float16)
+    with pytest.raises(na.Na2dError):
+        na.na2d_forward(x, x, x, None, 7, 1, out=torch.empty_like(x))

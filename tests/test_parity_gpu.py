@@ -1,0 +1,190 @@
+"""GPU parity: the CUDA library, called through its C ABI, against the fp64
+oracle on the same seeded inputs.
+
+Tolerances (max abs error, fp32 accumulation everywhere): 1e-5 for fp32,
+5e-3 for fp16 and 2e-2 for bf16 -- the bounds the problem statement sets for
+this operation.  Inputs are drawn in fp32 and rounded to the dtype first; the
+oracle sees exactly those rounded values, upcast to fp64.
+"""
+import math
+import random
+
+import numpy as np
+import pytest
+import torch
+
+import neighborhood_attention_na2d_b200 as na
+import oracle
+from neighborhood_attention_na2d_b200.build import build
+from neighborhood_attention_na2d_b200.inputs import WORKLOADS, Shape, all_shapes, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-5, "f16": 5e-3, "bf16": 2e-2}
+PAD = 256   # guard-band elements around every output (keeps 16-byte alignment)
+SENTINEL = -12345.0
+
+
+@pytest.fixture(scope="module", autouse=True)
+def gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    build()
+    torch.cuda.init()
+
+
+def f64(t):
+    return None if t is None else t.double().numpy()
+
+
+def guarded_out(like: torch.Tensor):
+    """An output tensor inside a larger buffer whose margins hold a sentinel."""
+    n = like.numel()
+    buf = torch.full((n + 2 * PAD,), SENTINEL, dtype=like.dtype, device="cuda")
+    return buf, buf[PAD:PAD + n].view(like.shape)
+
+
+def check_guards(buf):
+    edge = torch.cat([buf[:PAD], buf[-PAD:]]).float()
+    assert bool((edge == float(torch.tensor(SENTINEL, dtype=buf.dtype).float())).all()), "write outside the output"
+
+
+def run_forward(shape: Shape, with_rpb=True, seed=None):
+    q, k, v, rpb = make_inputs(shape, seed)
+    if not with_rpb:
+        rpb = None
+    buf, out = guarded_out(q)
+    na.na2d_forward(q.cuda(), k.cuda(), v.cuda(), None if rpb is None else rpb.cuda(), shape.k, shape.d, out=out)
+    torch.cuda.synchronize()
+    check_guards(buf)
+    return (q, k, v, rpb), out.double().cpu().numpy()
+
+
+def max_err(a, b):
+    return float(np.abs(a - b).max()) if a.size else 0.0
+
+
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("name,shape", all_shapes(), ids=[f"{n}:{s.describe()}" for n, s in all_shapes()])
+def test_workload_parity(name, shape):
+    """Every workload shape, every output element, against the oracle."""
+    (q, k, v, rpb), got = run_forward(shape)
+    want = oracle.forward(f64(q), f64(k), f64(v), f64(rpb), shape.k, shape.d)
+    err = max_err(got, want)
+    assert err <= TOL[shape.dtype], f"{shape.describe()}: max abs err {err}"
+
+
+def _ragged_cases():
+    rnd = random.Random(2024)
+    cases = []
+    for n in range(48):
+        k = rnd.choice([1, 3, 5, 7, 7, 9, 11, 13])
+        d = rnd.choice([1, 1, 2, 3, 4, 5, 8])
+        while k * d > 40:
+            d = max(1, d // 2)
+        H = rnd.randint(k * d, k * d + 2 * d + 11)
+        W = rnd.randint(k * d, k * d + 2 * d + 11)
+        dtype = rnd.choice(["f16", "bf16", "bf16", "f32"])
+        cases.append((Shape(rnd.choice([1, 2]), rnd.choice([1, 3]), H, W, 32, k, d, dtype, 5000 + n),
+                      rnd.random() < 0.8))
+    return cases
+
+
+@pytest.mark.parametrize("shape,with_rpb", _ragged_cases(), ids=lambda x: x.describe() if isinstance(x, Shape) else str(x))
+def test_ragged_shapes(shape, with_rpb):
+    """Seeded sweep of ragged sizes (H, W not multiples of any tile), every
+    supported k, dilations 1..8, all three dtypes, with and without bias."""
+    (q, k, v, rpb), got = run_forward(shape, with_rpb)
+    want = oracle.forward(f64(q), f64(k), f64(v), f64(rpb), shape.k, shape.d)
+    err = max_err(got, want)
+    assert err <= TOL[shape.dtype], f"{shape.describe()} rpb={with_rpb}: max abs err {err}"
+
+
+@pytest.mark.parametrize("k,d,L", [(3, 1, 3), (7, 1, 7), (13, 1, 13), (7, 2, 14), (13, 2, 26), (5, 8, 40), (13, 9, 117)])
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_window_covers_group(k, d, L, dtype):
+    """Edge case: every dilation group exactly k long, so every query attends to
+    its whole group (dense attention per sub-grid); includes the largest k and
+    a large dilation."""
+    shape = Shape(2, 2, L, L, 32, k, d, dtype, 77)
+    (q, kk, v, rpb), got = run_forward(shape)
+    want = oracle.forward(f64(q), f64(kk), f64(v), f64(rpb), k, d)
+    assert max_err(got, want) <= TOL[dtype]
+
+
+def test_full_attention_matches_dense_torch():
+    """k = H = W, d = 1, no bias: the GPU result is plain softmax attention,
+    compared with a dense fp64 torch computation (not the oracle)."""
+    for k, dtype in [(7, "f16"), (13, "bf16"), (7, "f32")]:
+        shape = Shape(2, 3, k, k, 32, k, 1, dtype, 91)
+        (q, kk, v, _), got = run_forward(shape, with_rpb=False)
+        Q, K, V = (t.double().reshape(2, 3, k * k, 32) for t in (q, kk, v))
+        P = torch.softmax(Q @ K.transpose(-1, -2) / math.sqrt(32), dim=-1)
+        want = (P @ V).reshape(2, 3, k, k, 32).numpy()
+        assert max_err(got, want) <= TOL[dtype]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
+@pytest.mark.parametrize("k,d,H,W", [(7, 1, 14, 17), (3, 3, 11, 13), (13, 1, 15, 13), (5, 2, 13, 10)])
+def test_split_path(dtype, k, d, H, W):
+    """na2d_qk_rpb -> na2d_softmax -> na2d_av, stage by stage against the oracle."""
+    shape = Shape(2, 2, H, W, 32, k, d, dtype, 123)
+    q, kk, v, rpb = make_inputs(shape)
+    qd, kd, vd, rd = (t.cuda() for t in (q, kk, v, rpb))
+    attn = na.na2d_qk_rpb(qd, kd, rd, k, d)
+    torch.cuda.synchronize()
+    ref_scores = oracle.qk_rpb(f64(q), f64(kk), f64(rpb), k, d)
+    assert max_err(attn.double().cpu().numpy(), ref_scores) <= 1e-4
+    gpu_scores = attn.double().cpu().numpy()
+    na.na2d_softmax(attn, k, d)
+    torch.cuda.synchronize()
+    probs = attn.double().cpu().numpy()
+    assert max_err(probs, oracle.softmax(gpu_scores, k, d)) <= 1e-6
+    out = na.na2d_av(attn, vd, k, d)
+    torch.cuda.synchronize()
+    assert max_err(out.double().cpu().numpy(), oracle.av(probs, f64(v), k, d)) <= TOL[dtype]
+    # the whole chain against the fused definition
+    assert max_err(out.double().cpu().numpy(), oracle.forward(f64(q), f64(kk), f64(v), f64(rpb), k, d)) <= TOL[dtype]
+
+
+def test_empty_batch():
+    x = torch.empty(0, 2, 14, 14, 32, dtype=torch.float16, device="cuda")
+    out = na.na2d_forward(x, x, x, None, 7, 1)
+    assert out.shape == x.shape
+
+
+def test_side_stream_and_determinism():
+    shape = WORKLOADS["dinat_s1_bf16"].shapes[0]
+    q, k, v, rpb = (t.cuda() for t in make_inputs(shape))
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        a = na.na2d_forward(q, k, v, rpb, shape.k, shape.d)
+        b = na.na2d_forward(q, k, v, rpb, shape.k, shape.d)
+    s.synchronize()
+    assert torch.equal(a, b)
+
+
+def test_misaligned_tensor_is_rejected():
+    q = torch.zeros(2 * 14 * 14 * 32 + 4, dtype=torch.float16, device="cuda")[4:].view(1, 2, 14, 14, 32)
+    with pytest.raises(na.Na2dError) as e:
+        na.na2d_forward(q, q, q, None, 7, 1, out=torch.empty(1, 2, 14, 14, 32, dtype=torch.float16, device="cuda"))
+    assert e.value.status == 6
+
+
+@pytest.mark.parametrize("name", ["nat_tiny_s1_fp16", "dinat_s1_bf16"])
+def test_bench_buffers_sampled(name):
+    """The benchmark's rotating input sets (seeds shape.seed + 1000 r), as the
+    benchmark calls them, checked at sampled queries including all four corners."""
+    shape = WORKLOADS[name].shapes[0]
+    rnd = random.Random(9)
+    for r in (1, 3):
+        q, k, v, rpb = make_inputs(shape, shape.seed + 1000 * r)
+        out = na.na2d_forward(q.cuda(), k.cuda(), v.cuda(), rpb.cuda(), shape.k, shape.d).double().cpu().numpy()
+        pts = [(0, 0, 0, 0), (shape.B - 1, shape.heads - 1, shape.H - 1, shape.W - 1),
+               (0, 1, 0, shape.W - 1), (1, 0, shape.H - 1, 0)]
+        pts += [(rnd.randrange(shape.B), rnd.randrange(shape.heads), rnd.randrange(shape.H), rnd.randrange(shape.W))
+                for _ in range(60)]
+        q64, k64, v64, r64 = f64(q), f64(k), f64(v), f64(rpb)
+        for (b, h, i, j) in pts:
+            want = oracle.forward_query(q64, k64, v64, r64, shape.k, shape.d, b, h, i, j)
+            assert float(np.abs(out[b, h, i, j] - want).max()) <= TOL[shape.dtype]
