@@ -107,6 +107,15 @@ NA2D_API na2d_status na2d_av(const na2d_problem *p, const float *attn, const voi
 NA2D_API na2d_status na2d_forward(const na2d_problem *p, const void *q, const void *k, const void *v,
                          const void *rpb, void *out, void *stream);
 
+/* Diagnostic.  Kernels that wait on shared-memory barriers for their own
+ * tensor copies give up after about a second of device time (a wait that long
+ * means the copy will never arrive), skip their remaining work and count the
+ * event.  This call writes that count for the current device into *count and
+ * clears it.  Unlike the calls above it synchronises `stream`.  A non-zero
+ * count means some outputs of the kernels since the last call were not
+ * written; it has never been observed and indicates a library bug. */
+NA2D_API na2d_status na2d_device_faults(unsigned int *count, void *stream);
+
 /* A static, human-readable name for a status. */
 NA2D_API const char *na2d_status_str(na2d_status s);
 

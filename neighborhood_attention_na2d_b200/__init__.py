@@ -16,10 +16,10 @@ from the library raises ``Na2dError``; there is no CPU fallback.
 """
 from __future__ import annotations
 
-from ._native import Na2dError, Problem, check, lib, status_str  # noqa: F401
+from ._native import Na2dError, Problem, check, device_faults, lib, status_str  # noqa: F401
 
-__all__ = ["na2d_qk_rpb", "na2d_softmax", "na2d_av", "na2d_forward", "na2d_status_str", "Na2dError",
-           "make_problem"]
+__all__ = ["na2d_qk_rpb", "na2d_softmax", "na2d_av", "na2d_forward", "na2d_status_str", "na2d_device_faults",
+           "Na2dError", "make_problem"]
 
 
 def _torch():
@@ -56,6 +56,15 @@ def _stream(t) -> int:
 
 def na2d_status_str(status: int) -> str:
     return status_str(status)
+
+
+def na2d_device_faults(device=None) -> int:
+    """Count of device-side bounded waits that timed out since the last call
+    (synchronises the current stream); zero unless the library has a bug."""
+    torch = _torch()
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        return device_faults(torch.cuda.current_stream(dev).cuda_stream)
 
 
 def na2d_forward(q, k, v, rpb, kernel_size: int, dilation: int = 1, out=None):

@@ -18,7 +18,8 @@ STATUS_NAMES = {
 }
 
 # every symbol the header declares
-EXPORTS = ("na2d_qk_rpb", "na2d_softmax", "na2d_av", "na2d_forward", "na2d_status_str", "na2d_version")
+EXPORTS = ("na2d_qk_rpb", "na2d_softmax", "na2d_av", "na2d_forward", "na2d_device_faults", "na2d_status_str",
+           "na2d_version")
 
 
 class Problem(ctypes.Structure):
@@ -54,6 +55,8 @@ def lib() -> ctypes.CDLL:
         L.na2d_forward.argtypes = [P, vp, vp, vp, vp, vp, vp]
         for f in ("na2d_qk_rpb", "na2d_softmax", "na2d_av", "na2d_forward"):
             getattr(L, f).restype = ctypes.c_int
+        L.na2d_device_faults.argtypes = [ctypes.POINTER(ctypes.c_uint), vp]
+        L.na2d_device_faults.restype = ctypes.c_int
         L.na2d_status_str.argtypes = [ctypes.c_int]
         L.na2d_status_str.restype = ctypes.c_char_p
         L.na2d_version.argtypes = []
@@ -87,3 +90,10 @@ def softmax_ptr(p: Problem, attn: int, stream: int = 0) -> int:
 
 def av_ptr(p: Problem, attn: int, v: int, out: int, stream: int = 0) -> int:
     return lib().na2d_av(ctypes.byref(p), attn, v, out, stream)
+
+
+def device_faults(stream: int = 0) -> int:
+    """Reads and clears the device's count of timed-out bounded waits."""
+    c = ctypes.c_uint(0)
+    check(lib().na2d_device_faults(ctypes.byref(c), stream), "na2d_device_faults")
+    return c.value

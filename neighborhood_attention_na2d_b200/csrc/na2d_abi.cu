@@ -125,6 +125,11 @@ na2d_status na2d_av(const na2d_problem *p, const float *attn, const void *v, voi
     return from_cuda(na2d::launch_av(pr, attn, v, out, static_cast<cudaStream_t>(stream)));
 }
 
+na2d_status na2d_device_faults(unsigned int *count, void *stream) {
+    if (!count) return NA2D_ERR_NULL;
+    return from_cuda(na2d::read_device_faults(count, static_cast<cudaStream_t>(stream)));
+}
+
 const char *na2d_status_str(na2d_status s) {
     switch (s) {
     case NA2D_OK: return "ok";

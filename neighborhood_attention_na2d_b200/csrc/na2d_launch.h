@@ -28,6 +28,10 @@ cudaError_t launch_qk_rpb(const Problem &p, const void *q, const void *k, const 
 cudaError_t launch_softmax(const Problem &p, float *attn, cudaStream_t stream);
 cudaError_t launch_av(const Problem &p, const float *attn, const void *v, void *out, cudaStream_t stream);
 
+// Reads and clears the count of device-side bounded waits that ran out;
+// synchronises the stream.
+cudaError_t read_device_faults(unsigned int *count, cudaStream_t stream);
+
 // True when launch_forward_tc handles this problem.
 bool tc_supported(const Problem &p);
 

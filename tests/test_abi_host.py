@@ -66,6 +66,7 @@ def _host_checks() -> dict:
     r["empty_qk"] = _native.qk_rpb_ptr(prob(B=0), 0, 0, None, 0)
     r["empty_softmax"] = _native.softmax_ptr(prob(B=0), 0)
     r["empty_av"] = _native.av_ptr(prob(B=0), 0, 0, 0)
+    r["faults_null"] = L.na2d_device_faults(None, None)
     return r
 
 
@@ -115,7 +116,7 @@ def test_forward_rejects_bad_problems(host_results, i):
     ("null_problem", 1), ("null_q", 1), ("null_out", 1), ("null_qk_k", 1), ("null_softmax", 1), ("null_av_v", 1),
     ("align_q", 6), ("align_rpb", 6), ("align_attn", 6), ("align_softmax", 6), ("align_av", 6),
     ("alias_out_q", 7), ("alias_partial", 7), ("alias_av", 7),
-    ("empty_B", 0), ("empty_heads", 0), ("empty_qk", 0), ("empty_softmax", 0), ("empty_av", 0),
+    ("empty_B", 0), ("empty_heads", 0), ("empty_qk", 0), ("empty_softmax", 0), ("empty_av", 0), ("faults_null", 1),
 ])
 def test_host_checks(host_results, case, status):
     assert host_results[case] == status

@@ -147,6 +147,12 @@ def test_split_path(dtype, k, d, H, W):
     assert max_err(out.double().cpu().numpy(), oracle.forward(f64(q), f64(kk), f64(v), f64(rpb), k, d)) <= TOL[dtype]
 
 
+def test_no_device_wait_timed_out():
+    """Runs after the parity tests above (same module): no kernel gave up on a
+    bounded wait."""
+    assert na.na2d_device_faults() == 0
+
+
 def test_empty_batch():
     x = torch.empty(0, 2, 14, 14, 32, dtype=torch.float16, device="cuda")
     out = na.na2d_forward(x, x, x, None, 7, 1)
