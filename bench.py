@@ -34,6 +34,8 @@ from pathlib import Path
 ROOT = Path(__file__).resolve().parent
 sys.path.insert(0, str(ROOT))
 
+from dataclasses import replace  # noqa: E402
+
 from neighborhood_attention_na2d_b200.inputs import HEADLINE, WORKLOADS, make_inputs  # noqa: E402
 
 METRIC = "NA2D forward queries·heads/sec (GB/s, % HBM roofline) at NAT/DiNAT shapes"
@@ -131,6 +133,15 @@ class ClockSampler:
                 "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
+def workload(args):
+    """The selected workload, with B overridden by --batch if given."""
+    wl = WORKLOADS[args.workload]
+    if args.batch:
+        wl = replace(wl, name=f"{wl.name}_B{args.batch}",
+                     shapes=tuple(replace(s, B=args.batch) for s in wl.shapes))
+    return wl
+
+
 # ---------------------------------------------------------------------------
 def dist_setup(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -147,7 +158,7 @@ def run_reference(args, world, rank):
         return
     import oracle
 
-    wl = WORKLOADS[args.workload]
+    wl = workload(args)
     threads = oracle.default_threads()
     # sample: the first nb batch elements of every shape -- enough (batch, head)
     # slices to occupy every host core; the step count is cut below if needed
@@ -237,7 +248,7 @@ def run_ours(args, world, rank, local):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
         pg = dist
     na.lib()
-    wl = WORKLOADS[args.workload]
+    wl = workload(args)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     elem = {"f32": 4, "f16": 2, "bf16": 2}
 
@@ -387,6 +398,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=HEADLINE)
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed oracle leg")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override B of every shape (a larger or smaller case of the same kernels)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
