@@ -44,6 +44,7 @@ FALLBACK_HBM_GBS = 6650.0
 PEAKS_FILE = ROOT / "MEASURED_PEAKS.json"
 PROFILES = ROOT / "profiles"
 KERNEL_SOURCES = ["neighborhood_attention_na2d_b200/csrc/na2d_tc.cu",
+                  "neighborhood_attention_na2d_b200/csrc/na2d_stream.cu",
                   "neighborhood_attention_na2d_b200/csrc/na2d_device.cuh"]
 
 

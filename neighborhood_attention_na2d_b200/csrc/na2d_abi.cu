@@ -82,7 +82,12 @@ na2d_status na2d_forward(const na2d_problem *p, const void *q, const void *k, co
     if (overlap(out, n, q, n) || overlap(out, n, k, n) || overlap(out, n, v, n) || overlap(out, n, rpb, rpb_bytes(p)))
         return NA2D_ERR_ALIAS;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (na2d::tc_supported(pr)) return from_cuda(na2d::launch_forward_tc(pr, q, k, v, rpb, out, st));
+    if (na2d::tc_supported(pr)) {
+        bool launched = false;
+        const cudaError_t e = na2d::launch_forward_stream(pr, q, k, v, rpb, out, st, &launched);
+        if (e != cudaSuccess || launched) return from_cuda(e);
+        return from_cuda(na2d::launch_forward_tc(pr, q, k, v, rpb, out, st));
+    }
     return from_cuda(na2d::launch_forward_simt(pr, q, k, v, rpb, out, st));
 }
 
@@ -127,7 +132,12 @@ na2d_status na2d_av(const na2d_problem *p, const float *attn, const void *v, voi
 
 na2d_status na2d_device_faults(unsigned int *count, void *stream) {
     if (!count) return NA2D_ERR_NULL;
-    return from_cuda(na2d::read_device_faults(count, static_cast<cudaStream_t>(stream)));
+    unsigned int a = 0, b = 0;
+    cudaError_t e = na2d::read_device_faults(&a, static_cast<cudaStream_t>(stream));
+    if (e == cudaSuccess) e = na2d::read_stream_faults(&b, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return from_cuda(e);
+    *count = a + b;
+    return NA2D_OK;
 }
 
 const char *na2d_status_str(na2d_status s) {

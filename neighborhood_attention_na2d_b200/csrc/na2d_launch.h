@@ -35,4 +35,14 @@ cudaError_t read_device_faults(unsigned int *count, cudaStream_t stream);
 // True when launch_forward_tc handles this problem.
 bool tc_supported(const Problem &p);
 
+// Streaming tensor-core forward for k = 7 (f16 / bf16, D = 32): d = 1 maps with
+// 14 <= W <= 64 and H >= 8, or H = W = 7d (every dilation group 7 x 7).  Sets
+// *launched when it took the problem; otherwise the caller uses
+// launch_forward_tc.
+bool stream_supported(const Problem &p);
+cudaError_t launch_forward_stream(const Problem &p, const void *q, const void *k, const void *v,
+                                  const void *rpb, void *out, cudaStream_t stream, bool *launched);
+// As read_device_faults, for the streaming kernel's counter.
+cudaError_t read_stream_faults(unsigned int *count, cudaStream_t stream);
+
 }  // namespace na2d

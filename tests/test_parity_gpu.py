@@ -100,6 +100,34 @@ def test_ragged_shapes(shape, with_rpb):
     assert err <= TOL[shape.dtype], f"{shape.describe()} rpb={with_rpb}: max abs err {err}"
 
 
+def _stream_cases():
+    """Shapes of the k = 7 streaming schedules: d = 1 row streaming (W from 14
+    to 64, odd and short H, several images per CTA, CTA ranges that cross
+    images) and dense 7 x 7 groups (H = W = 7d, odd group counts)."""
+    cases = []
+    n = 0
+    for (B, heads, H, W) in [(1, 1, 8, 14), (2, 3, 9, 15), (1, 2, 13, 21), (3, 1, 14, 28), (1, 2, 29, 40),
+                             (2, 1, 17, 49), (2, 2, 56, 56), (1, 3, 11, 57), (1, 1, 30, 63), (2, 3, 8, 64),
+                             (4, 3, 56, 56), (9, 5, 14, 14)]:
+        for dtype in ("f16", "bf16"):
+            cases.append((Shape(B, heads, H, W, 32, 7, 1, dtype, 7000 + n), n % 3 != 2))
+            n += 1
+    for (B, heads, d) in [(1, 1, 1), (3, 3, 1), (1, 2, 2), (2, 1, 3), (1, 3, 5), (1, 1, 8), (3, 1, 8)]:
+        for dtype in ("f16", "bf16"):
+            cases.append((Shape(B, heads, 7 * d, 7 * d, 32, 7, d, dtype, 7000 + n), n % 3 != 2))
+            n += 1
+    return cases
+
+
+@pytest.mark.parametrize("shape,with_rpb", _stream_cases(), ids=lambda x: x.describe() if isinstance(x, Shape) else str(x))
+def test_stream_shapes(shape, with_rpb):
+    """The streaming k = 7 kernel's schedules, every output element."""
+    (q, k, v, rpb), got = run_forward(shape, with_rpb)
+    want = oracle.forward(f64(q), f64(k), f64(v), f64(rpb), shape.k, shape.d)
+    err = max_err(got, want)
+    assert err <= TOL[shape.dtype], f"{shape.describe()} rpb={with_rpb}: max abs err {err}"
+
+
 @pytest.mark.parametrize("k,d,L", [(3, 1, 3), (7, 1, 7), (13, 1, 13), (7, 2, 14), (13, 2, 26), (5, 8, 40), (13, 9, 117)])
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
 def test_window_covers_group(k, d, L, dtype):
