@@ -17,29 +17,33 @@
 //    whose dilated window spans the map): a group is a dense 49 x 49
 //    attention.  A step is NWC / 4 consecutive groups, staged whole.
 //
-// Roles: warp NWC is a producer that issues 16-byte cp.async copies for up to
-// NS steps ahead and signals each step's stage through an mbarrier
-// (cp.async.mbarrier.arrive.noinc); warps 0 .. NWC-1 consume.  A consumer
-// releases a stage by arriving on its "empty" barrier; the producer refills a
-// stage only after every consumer released it.  All waits are bounded.
+// Loading: every warp issues its share of the 16-byte cp.async copies of the
+// step NS - 1 ahead (many warps keep enough requests in flight to stream at
+// HBM speed; a single issuing thread does not), and every thread arrives on
+// the stage's "full" mbarrier once its copies have landed
+// (cp.async.mbarrier.arrive.noinc).  A warp refills a stage only after all
+// warps released it on its "empty" mbarrier, which keeps the warps within
+// one step of each other.  All waits are bounded.
 //
 // Per warp, one 16-query tile per step: 2 query rows x 8 query columns.  Its
 // keys form n-tiles of 4 key rows x 2 key columns (14 n-tiles = 8 x 14 keys for
 // SLIDE, 8 n-tiles = 8 x 8 padded keys for DENSE), so the C-fragment pair a
 // thread holds is two horizontally adjacent keys.  The relative-position bias
-// (pre-multiplied by sqrt(D), masked keys at -1e30) lives in registers and is
-// the C input of the first QK^T MMA, so the bias costs no instruction; it is
-// rebuilt only when the head or the tile's window geometry changes.  The
-// softmax takes the row max with quad shuffles, then exponentiates in packed
-// f16x2 / bf16x2 (the P operand's own type) and feeds P straight back as the
-// A fragments of P.V; row sums come from an MMA against ones.
+// (pre-multiplied by sqrt(D), masked keys at -1e30) is the C input of the first
+// QK^T MMA, so adding it costs no instruction.  Each lane's bias values are
+// kept in tensor memory (TMEM, one lane quarter and 64 columns per warp),
+// rewritten only when the head or the tile's window geometry changes and read
+// back with tcgen05.ld per chunk of key columns; keeping them there instead of
+// in 56 registers leaves room for 16 warps per SM.  The softmax runs over two
+// chunks of key columns with a running max, exponentiates in fp32 and packs P
+// straight into the A fragments of P.V; row sums come from an MMA against ones.
 //
 // Shared-memory layouts (64 bytes per pixel, four 16-byte chunks):
-//  * K / V rows: chunk ^ (row & 3), where row is the ring (or group) row; any
-//    8 keys of an n-tile (4 consecutive rows x 2 adjacent columns) then fall
-//    in 8 distinct bank groups.
-//  * Q rows: chunk ^ ((slot >> 1) & 3) over the linear slot index; any 8
-//    consecutive query columns fall in 8 distinct bank groups.
+//  * SLIDE rows (Q, K, V): row r of a buffer starts at r * (W + 1) * 64 +
+//    16 * (r & 3); any 4 consecutive rows x 2 adjacent pixels of one chunk
+//    index fall in 8 distinct bank groups.
+//  * DENSE group blocks (8 x 8 pixels): K / V chunk c of row t stored at
+//    c ^ (t & 3); Q chunk c of slot s at c ^ ((s >> 1) & 3).
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -111,6 +115,38 @@ __device__ __forceinline__ void sb_arrive(uint32_t bar) {
 // have landed (the arrival is counted in the barrier's initial count).
 __device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(bar) : "memory");
+}
+
+// ---- tensor memory (TMEM) helpers -------------------------------------------
+constexpr int kTmemCols = 256;   // 4 column slots of 64, one per warp of a lane quarter
+
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(dst_smem),
+                 "n"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(taddr), "n"(kTmemCols) : "memory");
+}
+__device__ __forceinline__ void tmem_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
+__device__ __forceinline__ void tmem_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
+// 8 consecutive columns of this thread's lane
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const float (&v)[8]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};\n" ::"r"(taddr),
+        "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
+// 4 consecutive columns (one n-tile's C-init) of this thread's lane; complete
+// after tmem_ld_wait()
+__device__ __forceinline__ void tmem_ld4(uint32_t taddr, float (&v)[4]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];\n"
+                 : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3])
+                 : "r"(taddr)
+                 : "memory");
 }
 
 // ---- swizzled offsets --------------------------------------------------------
@@ -194,6 +230,7 @@ __device__ __forceinline__ int pair_halo(int pair, int H) { return min(win_start
 // kept; the rest is recomputed from them.
 struct SlideWalk {
     int bh, k;        // image and step index within it
+    int h;            // head of image bh
     int ring_lo;      // ring row of lo()
     __device__ __forceinline__ int p0(const StreamParams &p) const { return k * p.SP; }
     __device__ __forceinline__ int plast(const StreamParams &p) const { return min(k * p.SP + p.SP, p.NP) - 1; }
@@ -202,6 +239,7 @@ struct SlideWalk {
     __device__ __forceinline__ void init(const StreamParams &p, int s) {
         bh = s / p.SPI;
         k = s - bh * p.SPI;
+        h = bh % p.heads;
         ring_lo = 0;
     }
     __device__ __forceinline__ static int wrap(int x, int NR) { return x >= NR ? x - NR : x; }
@@ -215,6 +253,7 @@ struct SlideWalk {
         if (++k == p.SPI) {
             k = 0;
             ++bh;
+            if (++h == p.heads) h = 0;
             ring_lo = wrap(hi_ring + 1, p.NR);
             return lo(p);
         }
@@ -245,6 +284,8 @@ __device__ __forceinline__ uint32_t row_base(int r, uint32_t pitch) { return (ui
 //   columns 2J, 2J+1); a P.V k-step takes the pair (0, J) + (1, J).
 //   The key columns are processed in chunks [J0, J1) with an online softmax
 //   (running max, rescaled sums), which bounds the live score registers.
+//   tb: this warp's TMEM bias address for this lane; n-tile (R, J) holds its
+//       four C-init values in columns (2J + R) * 4 .. + 3.
 //   qa0, qa1: this lane's ldmatrix addresses of the Q fragments (k-steps 0, 1).
 //   kb0, kb1: this lane's K address of n-tile (R, 0); n-tile (R, J) is + J*128.
 //   dv: V address minus K address (same layout).
@@ -256,10 +297,17 @@ struct TileAcc {
     float m0, m1;    // running row max of rows r and r + 8 (raw accumulator units)
 };
 
-template <typename T, int NJ, int J0, int J1, bool SKEW, bool FIRST>
+template <typename T, int J0, int J1, bool SKEW, bool FIRST>
 __device__ __forceinline__ void tile_chunk(TileAcc &acc, const uint32_t (&qf)[2][4], uint32_t kb0, uint32_t kb1,
-                                           uint32_t vsel, const float (&bias)[2][NJ][4], float c_log2) {
+                                           uint32_t vsel, uint32_t tb, float c_log2) {
     constexpr int NC = J1 - J0;
+    // ---- bias C-init of the chunk's n-tiles from TMEM
+    float bias[2][NC][4];
+#pragma unroll
+    for (int j = 0; j < NC; ++j)
+#pragma unroll
+        for (int R = 0; R < 2; ++R) tmem_ld4(tb + (uint32_t)((2 * (J0 + j) + R) * 4), bias[R][j]);
+    tmem_ld_wait();
     // ---- S = Q K^T + bias*sqrt(D) over the chunk's 2 * NC n-tiles
     float s[2][NC][4];
 #pragma unroll
@@ -268,7 +316,7 @@ __device__ __forceinline__ void tile_chunk(TileAcc &acc, const uint32_t (&qf)[2]
         for (int R = 0; R < 2; ++R) {
             uint32_t kf[4];
             ldsm_x4(kf, (R ? kb1 : kb0) + (J0 + j) * 128);
-            MmaC<T>::run(s[R][j], qf[0], kf[0], kf[1], bias[R][J0 + j]);
+            MmaC<T>::run(s[R][j], qf[0], kf[0], kf[1], bias[R][j]);
             Mma<T>::run(s[R][j], qf[1], kf[2], kf[3]);
         }
     }
@@ -333,8 +381,8 @@ __device__ __forceinline__ void tile_chunk(TileAcc &acc, const uint32_t (&qf)[2]
 
 template <typename T, int NJ, bool SKEW>
 __device__ __forceinline__ void tile_compute(uint32_t qa0, uint32_t qa1, uint32_t kb0, uint32_t kb1, uint32_t dv,
-                                             const float (&bias)[2][NJ][4], float c_log2, int lane,
-                                             unsigned char *out0, unsigned char *out1) {
+                                             uint32_t tb, float c_log2, int lane, unsigned char *out0,
+                                             unsigned char *out1) {
     uint32_t qf[2][4];
     ldsm_x4(qf[0], qa0);
     ldsm_x4(qf[1], qa1);
@@ -343,10 +391,10 @@ __device__ __forceinline__ void tile_compute(uint32_t qa0, uint32_t qa1, uint32_
     const uint32_t vsel = (((lane >> 3) & 1) ? kb1 : kb0) + dv;
     TileAcc acc;
     if constexpr (NJ == 7) {
-        tile_chunk<T, NJ, 0, 2, SKEW, true>(acc, qf, kb0, kb1, vsel, bias, c_log2);
-        tile_chunk<T, NJ, 2, 7, SKEW, false>(acc, qf, kb0, kb1, vsel, bias, c_log2);
+        tile_chunk<T, 0, 4, SKEW, true>(acc, qf, kb0, kb1, vsel, tb, c_log2);
+        tile_chunk<T, 4, 7, SKEW, false>(acc, qf, kb0, kb1, vsel, tb, c_log2);
     } else {
-        tile_chunk<T, NJ, 0, NJ, SKEW, true>(acc, qf, kb0, kb1, vsel, bias, c_log2);
+        tile_chunk<T, 0, NJ, SKEW, true>(acc, qf, kb0, kb1, vsel, tb, c_log2);
     }
     // ---- normalise and store: row r holds channels 8*cn + 2*(lane&3) (+1)
     float i0, i1;
@@ -367,9 +415,27 @@ __device__ __forceinline__ void tile_compute(uint32_t qa0, uint32_t qa1, uint32_
     }
 }
 
+// Writes one lane's bias C-init values (n-tile (R, J) at columns
+// (2J + R) * 4 ..) into TMEM, 8 columns at a time.
+template <int NJ>
+__device__ __forceinline__ void tmem_store_bias(uint32_t tb, const float (&bias)[2][NJ][4]) {
+#pragma unroll
+    for (int J = 0; J < NJ; ++J) {
+        const float v[8] = {bias[0][J][0], bias[0][J][1], bias[0][J][2], bias[0][J][3],
+                            bias[1][J][0], bias[1][J][1], bias[1][J][2], bias[1][J][3]};
+        tmem_st8(tb + (uint32_t)(8 * J), v);
+    }
+    tmem_st_wait();
+}
+
 // ---------------------------------------------------------------------------
 // Kernel.
 // ---------------------------------------------------------------------------
+// Warps 0 .. NWC-1 consume; warp NWC produces (SLIDE: one thread issues one
+// bulk copy per image row; DENSE: the warp issues 16-byte cp.async).  Each
+// consumer warp owns a fixed tile position of every step (SLIDE: pair
+// warp / MX of the step, column tile warp % MX; DENSE: group warp / 4 of the
+// step, query-row pair warp % 4), so per-warp geometry is set up once.
 template <typename T, bool DENSE, int NWC>
 __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __grid_constant__ StreamParams p) {
     extern __shared__ __align__(1024) unsigned char smem[];
@@ -377,18 +443,24 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
     const int s_begin = (int)((int64_t)p.nsteps * blockIdx.x / gridDim.x);
     const int s_end = (int)((int64_t)p.nsteps * (blockIdx.x + 1) / gridDim.x);
     if (s_begin >= s_end) return;
+    const int nst = s_end - s_begin;
+    constexpr int GPS = NWC / 4;   // DENSE groups per step
 
     const uint32_t sbase = smem_u32(smem);
     const uint32_t bar_full = sbase + p.off_bar, bar_empty = bar_full + 8 * NS;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + p.off_bar + 16 * NS);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + p.off_bar + 16 * NS + 4);
     float *tab = reinterpret_cast<float *>(smem + p.off_tab);
+    const uint32_t pitch = (uint32_t)(p.W + 1) * kPixB;   // SLIDE row pitch in bytes
 
-    // ---- prologue: zero the staging buffers (pads and unused rows must hold
-    // finite values), build the bias table, init the barriers.
+    // ---- prologue: (DENSE) zero the staging blocks, whose pad pixels must
+    // hold finite values; build the bias table; init the barriers; allocate TMEM.
     {
-        uint4 *z = reinterpret_cast<uint4 *>(smem);
-        const int n16 = (int)(p.off_tab / 16);
-        for (int i = threadIdx.x; i < n16; i += blockDim.x) z[i] = make_uint4(0, 0, 0, 0);
+        if constexpr (DENSE) {
+            uint4 *z = reinterpret_cast<uint4 *>(smem);
+            const int n16 = (int)(p.off_tab / 16);
+            for (int i = threadIdx.x; i < n16; i += blockDim.x) z[i] = make_uint4(0, 0, 0, 0);
+        }
         const T *rpb = reinterpret_cast<const T *>(p.rpb);
         for (int i = threadIdx.x; i < p.heads * kTabHead; i += blockDim.x) {
             const int h = i / kTabHead, a = (i / kTabPitch) % 13, b = i % kTabPitch;
@@ -406,50 +478,51 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
             *abort_flag = 0;
             asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
         }
+        if (warp == 0) tmem_alloc(smem_u32(tmem_slot));
+        tmem_fence_before();
         __syncthreads();
+        tmem_fence_after();
     }
-    const uint32_t pitch = (uint32_t)(p.W + 1) * kPixB;   // SLIDE row pitch in bytes
-    constexpr int GPS = NWC / 4;                           // DENSE groups per step
 
     if (warp == NWC) {
         // =================== producer ===================
         if constexpr (!DENSE) {
             // one thread issues one bulk copy per image row: the step's new
             // K and V rows into the ring, its query rows into the stage
-            if (lane != 0) return;
-            const uint32_t rowbytes = (uint32_t)p.W * kPixB;
-            SlideWalk w;
-            w.init(p, s_begin);
-            int issued = 0;
-            for (int s = s_begin, i = 0; s < s_end; ++s, ++i) {
-                const int stage = i % NS;
-                const int first = i ? w.next(p) : w.lo(p);
-                if (i >= NS && !sb_wait(bar_empty + 8 * stage, (uint32_t)(((i / NS) - 1) & 1))) {
-                    atomicAdd(&g_stream_timeouts, 1u);
-                    *abort_flag = 1;
-                    break;
+            if (lane == 0) {
+                const uint32_t rowbytes = (uint32_t)p.W * kPixB;
+                SlideWalk w;
+                w.init(p, s_begin);
+                int issued = 0;
+                for (int i = 0; i < nst; ++i) {
+                    const int stage = i % NS;
+                    const int first = i ? w.next(p) : w.lo(p);
+                    if (i >= NS && !sb_wait(bar_empty + 8 * stage, (uint32_t)(((i / NS) - 1) & 1))) {
+                        atomicAdd(&g_stream_timeouts, 1u);
+                        *abort_flag = 1;
+                        break;
+                    }
+                    if (*abort_flag) break;
+                    const int hi = w.hi(p);
+                    const int y0 = 2 * w.p0(p), y1 = min(2 * (w.plast(p) + 1), p.H);
+                    const uint32_t bar = bar_full + 8 * stage;
+                    sb_expect_tx(bar, (uint32_t)(2 * (hi - first + 1) + (y1 - y0)) * rowbytes);
+                    for (int row = first; row <= hi; ++row) {
+                        const uint32_t o = row_base(w.ring(p, row), pitch);
+                        const size_t src = ((size_t)w.bh * p.H + row) * rowbytes;
+                        bulk_g2s(sbase + p.off_k + o, p.k + src, rowbytes, bar);
+                        bulk_g2s(sbase + p.off_v + o, p.v + src, rowbytes, bar);
+                    }
+                    for (int y = y0; y < y1; ++y)
+                        bulk_g2s(sbase + row_base(stage * 2 * p.SP + (y - y0), pitch),
+                                 p.q + ((size_t)w.bh * p.H + y) * rowbytes, rowbytes, bar);
+                    ++issued;
                 }
-                if (*abort_flag) break;
-                const int hi = w.hi(p);
-                const int y0 = 2 * w.p0(p), y1 = min(2 * (w.plast(p) + 1), p.H);
-                const uint32_t bar = bar_full + 8 * stage;
-                sb_expect_tx(bar, (uint32_t)(2 * (hi - first + 1) + (y1 - y0)) * rowbytes);
-                for (int row = first; row <= hi; ++row) {
-                    const uint32_t o = row_base(w.ring(p, row), pitch);
-                    const size_t src = ((size_t)w.bh * p.H + row) * rowbytes;
-                    bulk_g2s(sbase + p.off_k + o, p.k + src, rowbytes, bar);
-                    bulk_g2s(sbase + p.off_v + o, p.v + src, rowbytes, bar);
-                }
-                for (int y = y0; y < y1; ++y)
-                    bulk_g2s(sbase + row_base(stage * 2 * p.SP + (y - y0), pitch),
-                             p.q + ((size_t)w.bh * p.H + y) * rowbytes, rowbytes, bar);
-                ++issued;
+                // copies still in flight must land before the CTA's shared
+                // memory is released (all of them, unless a wait ran out)
+                for (int j = max(0, issued - NS); j < issued; ++j)
+                    sb_wait(bar_full + 8 * (j % NS), (uint32_t)((j / NS) & 1));
             }
-            // copies still in flight must land before the CTA's shared memory
-            // is released (all of them, unless a wait ran out); bounded waits
-            for (int j = max(0, issued - NS); j < issued; ++j)
-                sb_wait(bar_full + 8 * (j % NS), (uint32_t)((j / NS) & 1));
-            return;
         } else {
             // GPS = 3 group-units per step, 16-byte cp.async per lane.  Lanes
             // 0-23 work: lane l copies chunk l & 3 of group (l >> 2) % 3 for
@@ -471,8 +544,8 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
                 dst_kv[t] = (uint32_t)(g * kDenseBlk) + kv_off(ty, 8, jx, ch);
             }
             const int dd = p.d * p.d;
-            for (int s = s_begin, i = 0; s < s_end; ++s, ++i) {
-                const int stage = i % NS;
+            for (int i = 0; i < nst; ++i) {
+                const int s = s_begin + i, stage = i % NS;
                 if (i >= NS && !sb_wait(bar_empty + 8 * stage, (uint32_t)(((i / NS) - 1) & 1))) {
                     if (lane == 0) {
                         atomicAdd(&g_stream_timeouts, 1u);
@@ -499,136 +572,171 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
                 cp_async_arrive(bar_full + 8 * stage);
             }
             cp_async_wait<0>();
-            return;
         }
-    }
-
-    // =================== consumers ===================
-    const int r = lane >> 2, c = lane & 3;
-    const int li = (lane & 7) >> 1, lj = lane & 1;   // this lane's key (row, col) in an n-tile
-    const int lch = lane >> 3;                       // this lane's channel chunk for K loads
-    constexpr int NJ = DENSE ? 4 : 7;
-    float bias[2][NJ][4];
-    int bias_key = -1;
-    SlideWalk w;
-    if constexpr (!DENSE) w.init(p, s_begin);
-    for (int s = s_begin, i = 0; s < s_end; ++s, ++i) {
-        const int stage = i % NS;
-        if constexpr (!DENSE)
-            if (i) w.next(p);
-        if (!sb_wait(bar_full + 8 * stage, (uint32_t)((i / NS) & 1))) {
-            if (lane == 0) {
-                atomicAdd(&g_stream_timeouts, 1u);
-                *abort_flag = 1;
-            }
-            break;
-        }
-        if (*abort_flag) break;
+    } else {
+        // =================== consumers ===================
+        const int r = lane >> 2, c = lane & 3;
+        const int li = (lane & 7) >> 1, lj = lane & 1;   // this lane's key (row, col) in an n-tile
+        const int lch = lane >> 3;                       // this lane's channel chunk for K loads
+        constexpr int NJ = DENSE ? 4 : 7;
+        // this warp's TMEM bias columns: lane quarter warp % 4, column slot warp / 4
+        const uint32_t tb = *tmem_slot + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(64 * (warp >> 2));
+        int bias_key = -1;
         if constexpr (!DENSE) {
-            const int pair = w.p0(p) + warp / p.MX;
-            if (warp < p.SP * p.MX && pair <= w.plast(p)) {
-                const int H = p.H, W = p.W;
-                const int qy0 = 2 * pair, qy1 = min(qy0 + 1, H - 1);
-                const int x0 = 8 * (warp % p.MX);
-                const int hy = pair_halo(pair, H);
-                const int hx = min(win_start(x0, W), W - 14);
-                const int h = w.bh % p.heads;
-                const int sy0 = win_start(qy0, H), sy1 = win_start(qy1, H);
-                // bias registers: rebuilt when the head or the row geometry changes
-                // (the column geometry is fixed per warp)
-                const int key = ((h * 8 + (qy0 - hy)) * 2 + (qy1 - qy0)) * 4 + (sy0 - hy) * 2 + (sy1 - hy);
-                if (key != bias_key) {
-                    bias_key = key;
-                    const int qx = min(x0 + r, W - 1), sx = win_start(qx, W);
-                    const float *th = tab + h * kTabHead;
-#pragma unroll
-                    for (int m = 0; m < 2; ++m) {
-                        const int qy = m ? qy1 : qy0, sy = m ? sy1 : sy0;
-#pragma unroll
-                        for (int R = 0; R < 2; ++R) {
-                            const int ky = hy + 4 * R + c;
-                            const bool yv = (unsigned)(ky - sy) < (unsigned)KW;
-                            const float *row = th + clampi(ky - qy + 6, 0, 12) * kTabPitch;
-#pragma unroll
-                            for (int J = 0; J < NJ; ++J)
-#pragma unroll
-                                for (int e = 0; e < 2; ++e) {
-                                    const int kx = hx + 2 * J + e;
-                                    const bool v = yv && (unsigned)(kx - sx) < (unsigned)KW;
-                                    const float b = row[clampi(kx - qx + 6, 0, 12)];
-                                    bias[R][J][2 * m + e] = v ? b : kMaskC;
-                                }
-                        }
+            const int H = p.H, W = p.W;
+            // fixed per warp: column tile, halo columns, this lane's query column
+            const int pw = warp / p.MX, x0 = 8 * (warp - pw * p.MX);
+            const bool active = warp < p.SP * p.MX;
+            const int hx = min(win_start(x0, W), W - 14);
+            const int qx = min(x0 + r, W - 1), sx = win_start(qx, W);
+            const bool colok = x0 + r < W;
+            const uint32_t kcol = (uint32_t)(hx + lj) * kPixB + 16u * lch;
+            const uint32_t qcol = (uint32_t)min(x0 + (lane & 7), W - 1) * kPixB + 16u * (lane >> 4);
+            const uint32_t dv = (p.off_v - p.off_k) + 16u * (uint32_t)((lane >> 4) - lch);
+            const int qsel = (lane >> 3) & 1;
+            SlideWalk w;
+            w.init(p, s_begin);
+            for (int i = 0; i < nst; ++i) {
+                const int stage = i % NS;
+                if (i) w.next(p);
+                if (!sb_wait(bar_full + 8 * stage, (uint32_t)((i / NS) & 1))) {
+                    if (lane == 0) {
+                        atomicAdd(&g_stream_timeouts, 1u);
+                        *abort_flag = 1;
                     }
+                    break;
                 }
-                // Q fragment addresses: lanes 0-7 / 16-23 row qy0, 8-15 / 24-31
-                // row qy1; lanes 16-31 take the odd 16-byte chunk
-                const int qr = stage * 2 * p.SP + (((lane >> 3) & 1) ? qy1 : qy0) - 2 * w.p0(p);
-                const uint32_t qa0 = sbase + row_base(qr, pitch) + (uint32_t)min(x0 + (lane & 7), W - 1) * kPixB +
-                                     16u * (lane >> 4);
-                // K addresses of n-tiles (0, 0) and (1, 0); V (x4.trans) lanes
-                // address the same keys with chunk lane >> 4
-                const uint32_t kcol = (uint32_t)(hx + lj) * kPixB + 16u * lch;
-                const uint32_t kb0 = sbase + p.off_k + row_base(w.ring(p, hy + li), pitch) + kcol;
-                const uint32_t kb1 = sbase + p.off_k + row_base(w.ring(p, hy + 4 + li), pitch) + kcol;
-                const uint32_t dv = (p.off_v - p.off_k) + 16u * (uint32_t)((lane >> 4) - lch);
-                unsigned char *o0 = nullptr, *o1 = nullptr;
-                if (x0 + r < W) {
-                    const size_t base = (size_t)w.bh * H;
-                    o0 = p.out + ((base + qy0) * W + x0 + r) * kPixB;
-                    if (qy0 + 1 < H) o1 = p.out + ((base + qy0 + 1) * W + x0 + r) * kPixB;
+                if (*abort_flag) break;
+                const int pair = w.p0(p) + pw;
+                if (active && pair <= w.plast(p)) {
+                    const int qy0 = 2 * pair, qy1 = min(qy0 + 1, H - 1);
+                    const int hy = pair_halo(pair, H);
+                    const int sy0 = win_start(qy0, H), sy1 = win_start(qy1, H);
+                    // bias: rewritten when the head or the row geometry changes
+                    const int key = ((w.h * 8 + (qy0 - hy)) * 2 + (qy1 - qy0)) * 4 + (sy0 - hy) * 2 + (sy1 - hy);
+                    if (key != bias_key) {
+                        bias_key = key;
+                        const float *th = tab + w.h * kTabHead;
+                        float bias[2][NJ][4];
+#pragma unroll
+                        for (int m = 0; m < 2; ++m) {
+                            const int qy = m ? qy1 : qy0, sy = m ? sy1 : sy0;
+#pragma unroll
+                            for (int R = 0; R < 2; ++R) {
+                                const int ky = hy + 4 * R + c;
+                                const bool yv = (unsigned)(ky - sy) < (unsigned)KW;
+                                const float *row = th + clampi(ky - qy + 6, 0, 12) * kTabPitch;
+#pragma unroll
+                                for (int J = 0; J < NJ; ++J)
+#pragma unroll
+                                    for (int e = 0; e < 2; ++e) {
+                                        const int kx = hx + 2 * J + e;
+                                        const bool v = yv && (unsigned)(kx - sx) < (unsigned)KW;
+                                        const float b = row[clampi(kx - qx + 6, 0, 12)];
+                                        bias[R][J][2 * m + e] = v ? b : kMaskC;
+                                    }
+                            }
+                        }
+                        tmem_store_bias<NJ>(tb, bias);
+                    }
+                    // Q fragment addresses: lanes 0-7 / 16-23 row qy0, 8-15 /
+                    // 24-31 row qy1; lanes 16-31 take the odd 16-byte chunk
+                    const int qr = stage * 2 * p.SP + (qsel ? qy1 : qy0) - 2 * w.p0(p);
+                    const uint32_t qa0 = sbase + row_base(qr, pitch) + qcol;
+                    // K addresses of n-tiles (0, 0) and (1, 0); V (x4.trans)
+                    // lanes address the same keys with chunk lane >> 4
+                    const uint32_t kb0 = sbase + p.off_k + row_base(w.ring(p, hy + li), pitch) + kcol;
+                    const uint32_t kb1 = sbase + p.off_k + row_base(w.ring(p, hy + 4 + li), pitch) + kcol;
+                    unsigned char *o0 = nullptr, *o1 = nullptr;
+                    if (colok) {
+                        o0 = p.out + (((size_t)w.bh * H + qy0) * W + x0 + r) * kPixB;
+                        if (qy0 + 1 < H) o1 = o0 + (size_t)W * kPixB;
+                    }
+                    tile_compute<T, NJ, true>(qa0, qa0 + 32u, kb0, kb1, dv, tb, p.c_log2, lane, o0, o1);
                 }
-                tile_compute<T, NJ, true>(qa0, qa0 + 32u, kb0, kb1, dv, bias, p.c_log2, lane, o0, o1);
+                __syncwarp();
+                if (lane == 0) sb_arrive(bar_empty + 8 * stage);
             }
         } else {
             const int g = warp >> 2, pp = warp & 3;
-            const int gu = GPS * s + g;
-            if (gu < p.GU) {
-                const int dd = p.d * p.d;
-                const int bh = gu / dd, rem = gu - bh * dd, gy = rem / p.d, gx = rem - gy * p.d;
-                const int h = bh % p.heads;
-                if (h != bias_key) {
-                    bias_key = h;
-                    const int qx = min(r, 6);
-                    const float *th = tab + h * kTabHead;
-#pragma unroll
-                    for (int m = 0; m < 2; ++m) {
-                        const int qy = min(2 * pp + m, 6);
-#pragma unroll
-                        for (int R = 0; R < 2; ++R) {
-                            const int ky = 4 * R + c;
-                            const float *row = th + clampi(ky - qy + 6, 0, 12) * kTabPitch;
-#pragma unroll
-                            for (int J = 0; J < NJ; ++J)
-#pragma unroll
-                                for (int e = 0; e < 2; ++e) {
-                                    const int kx = 2 * J + e;
-                                    const float b = row[clampi(kx - qx + 6, 0, 12)];
-                                    bias[R][J][2 * m + e] = (ky < KW && kx < KW) ? b : kMaskC;
-                                }
+            const int qx = min(r, 6);
+            const int qslot = (2 * pp + ((lane >> 3) & 1)) * 8 + (lane & 7);
+            const uint32_t qoff0 = q_off(qslot, (lane >> 4)), qoff1 = q_off(qslot, 2 + (lane >> 4));
+            const uint32_t koff0 = kv_off(li, 8, lj, lch), koff1 = kv_off(4 + li, 8, lj, lch);
+            const uint32_t dv = (p.off_v - p.off_k) + (uint32_t)((((lane >> 4) ^ li) - (lch ^ li)) * 16);
+            const int qy = 2 * pp;
+            const int dd = p.d * p.d;
+            // this warp's group of the first step, then advanced by GPS groups per step
+            int gu = GPS * s_begin + g;
+            int bh = gu / dd, rem = gu - bh * dd, gy = rem / p.d, gx = rem - gy * p.d;
+            int h = bh % p.heads;
+            for (int i = 0; i < nst; ++i) {
+                const int stage = i % NS;
+                if (i) {
+                    gu += GPS;
+                    gx += GPS;
+                    while (gx >= p.d) {
+                        gx -= p.d;
+                        if (++gy == p.d) {
+                            gy = 0;
+                            ++bh;
+                            if (++h == p.heads) h = 0;
                         }
                     }
                 }
-                const uint32_t blk = (uint32_t)((stage * GPS + g) * kDenseBlk);
-                const int qslot = (2 * pp + ((lane >> 3) & 1)) * 8 + (lane & 7);
-                const uint32_t qa0 = sbase + blk + q_off(qslot, (lane >> 4));
-                const uint32_t qa1 = sbase + blk + q_off(qslot, 2 + (lane >> 4));
-                const uint32_t kb0 = sbase + p.off_k + blk + kv_off(li, 8, lj, lch);
-                const uint32_t kb1 = sbase + p.off_k + blk + kv_off(4 + li, 8, lj, lch);
-                const uint32_t dv = (p.off_v - p.off_k) + (uint32_t)((((lane >> 4) ^ li) - (lch ^ li)) * 16);
-                unsigned char *o0 = nullptr, *o1 = nullptr;
-                const int qy = 2 * pp;
-                if (r < 7) {
-                    const size_t base = (size_t)bh * p.H;
-                    const size_t col = (size_t)gx + (size_t)p.d * r;
-                    o0 = p.out + ((base + gy + (size_t)p.d * qy) * p.W + col) * kPixB;
-                    if (qy + 1 < 7) o1 = p.out + ((base + gy + (size_t)p.d * (qy + 1)) * p.W + col) * kPixB;
+                if (!sb_wait(bar_full + 8 * stage, (uint32_t)((i / NS) & 1))) {
+                    if (lane == 0) {
+                        atomicAdd(&g_stream_timeouts, 1u);
+                        *abort_flag = 1;
+                    }
+                    break;
                 }
-                tile_compute<T, NJ, false>(qa0, qa1, kb0, kb1, dv, bias, p.c_log2, lane, o0, o1);
+                if (*abort_flag) break;
+                if (gu < p.GU) {
+                    if (h != bias_key) {
+                        bias_key = h;
+                        const float *th = tab + h * kTabHead;
+                        float bias[2][NJ][4];
+#pragma unroll
+                        for (int m = 0; m < 2; ++m) {
+                            const int qyy = min(2 * pp + m, 6);
+#pragma unroll
+                            for (int R = 0; R < 2; ++R) {
+                                const int ky = 4 * R + c;
+                                const float *row = th + clampi(ky - qyy + 6, 0, 12) * kTabPitch;
+#pragma unroll
+                                for (int J = 0; J < NJ; ++J)
+#pragma unroll
+                                    for (int e = 0; e < 2; ++e) {
+                                        const int kx = 2 * J + e;
+                                        const float b = row[clampi(kx - qx + 6, 0, 12)];
+                                        bias[R][J][2 * m + e] = (ky < KW && kx < KW) ? b : kMaskC;
+                                    }
+                            }
+                        }
+                        tmem_store_bias<NJ>(tb, bias);
+                    }
+                    const uint32_t blk = sbase + (uint32_t)((stage * GPS + g) * kDenseBlk);
+                    unsigned char *o0 = nullptr, *o1 = nullptr;
+                    if (r < 7) {
+                        o0 = p.out + ((((size_t)bh * p.H + gy + (size_t)p.d * qy) * p.W) + gx + (size_t)p.d * r) * kPixB;
+                        if (qy + 1 < 7) o1 = o0 + (size_t)p.d * p.W * kPixB;
+                    }
+                    tile_compute<T, NJ, false>(blk + qoff0, blk + qoff1, blk + p.off_k + koff0, blk + p.off_k + koff1,
+                                               dv, tb, p.c_log2, lane, o0, o1);
+                }
+                __syncwarp();
+                if (lane == 0) sb_arrive(bar_empty + 8 * stage);
             }
         }
-        __syncwarp();
-        if (lane == 0) sb_arrive(bar_empty + 8 * stage);
+    }
+    // ---- epilogue: TMEM released by the warp that took it, after every warp
+    // is done with it
+    tmem_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tmem_fence_after();
+        tmem_dealloc(*tmem_slot);
     }
 }
 
@@ -699,6 +807,24 @@ uint32_t plan_slide(StreamParams &sp, const Problem &pr, int SP) {
     return sp.off_bar + 16 * NS + 16;
 }
 
+template <typename T, int NWC>
+cudaError_t launch_slide(StreamParams &sp, const Problem &pr, cudaStream_t st, bool *launched) {
+    const void *kern = reinterpret_cast<const void *>(&fwd_stream_kernel<T, false, NWC>);
+    int sms = 0, cap = 0;
+    cudaError_t e = stream_device(&sms, &cap, kern);
+    if (e != cudaSuccess) return e;
+    const int MX = (pr.W + 7) / 8;
+    for (int SP = std::max(1, NWC / MX); SP >= 1; --SP) {
+        const uint32_t smem = plan_slide(sp, pr, SP);
+        if ((int)smem > cap) continue;
+        const int64_t nsteps = pr.bh() * sp.SPI;
+        if (nsteps >= INT32_MAX || nsteps <= 0) return cudaSuccess;
+        sp.nsteps = (int)nsteps;
+        return launch_stream_t<T, false, NWC>(sp, smem, sms, st, launched);
+    }
+    return cudaSuccess;
+}
+
 template <typename T>
 cudaError_t launch_stream_impl(const Problem &pr, const void *q, const void *k, const void *v, const void *rpb,
                                void *out, cudaStream_t st, bool *launched) {
@@ -714,8 +840,8 @@ cudaError_t launch_stream_impl(const Problem &pr, const void *q, const void *k, 
     const int64_t bh = pr.bh();
     const bool dense = (pr.H == KW * pr.d && pr.W == KW * pr.d);
     if (dense) {
-        // 12 consumer warps: three 7 x 7 groups per step, one warp per query-row
-        // pair of a group (13 warps in all keep 128 registers per thread)
+        // 12 consumer warps (three 7 x 7 groups per step, one warp per
+        // query-row pair of a group) and a producer warp
         constexpr int NWC = 12, GPS = NWC / 4;
         const void *kern = reinterpret_cast<const void *>(&fwd_stream_kernel<T, true, NWC>);
         int sms = 0, cap = 0;
@@ -735,23 +861,9 @@ cudaError_t launch_stream_impl(const Problem &pr, const void *q, const void *k, 
         if ((int)smem > cap) return cudaSuccess;
         return launch_stream_t<T, true, NWC>(sp, smem, sms, st, launched);
     }
-    // SLIDE: up to 15 consumer warps (SP query-row pairs of MX tiles each;
-    // 16 warps in all keep 128 registers per thread), fewer pairs per step if
-    // the rings do not fit
-    const int MX = (pr.W + 7) / 8;
-    const void *kern = reinterpret_cast<const void *>(&fwd_stream_kernel<T, false, 15>);
-    int sms = 0, cap = 0;
-    cudaError_t e = stream_device(&sms, &cap, kern);
-    if (e != cudaSuccess) return e;
-    for (int SP = std::max(1, 15 / MX); SP >= 1; --SP) {
-        const uint32_t smem = plan_slide(sp, pr, SP);
-        if ((int)smem > cap) continue;
-        const int64_t nsteps = bh * sp.SPI;
-        if (nsteps >= INT32_MAX || nsteps <= 0) return cudaSuccess;
-        sp.nsteps = (int)nsteps;
-        return launch_stream_t<T, false, 15>(sp, smem, sms, st, launched);
-    }
-    return cudaSuccess;
+    // SLIDE: 14 consumer warps (SP query-row pairs of MX column tiles each)
+    // and a producer warp; 15 warps keep 128 registers per thread
+    return launch_slide<T, 14>(sp, pr, st, launched);
 }
 
 }  // namespace
