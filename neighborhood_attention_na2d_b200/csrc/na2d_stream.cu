@@ -450,7 +450,8 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
     const uint32_t bar_full = sbase + p.off_bar, bar_empty = bar_full + 8 * NS;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + p.off_bar + 16 * NS);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + p.off_bar + 16 * NS + 4);
-    float *tab = reinterpret_cast<float *>(smem + p.off_tab);
+    // bias table, with 64 bytes of padding on either side for unclamped column reads
+    float *tab = reinterpret_cast<float *>(smem + p.off_tab + 64);
     const uint32_t pitch = (uint32_t)(p.W + 1) * kPixB;   // SLIDE row pitch in bytes
 
     // ---- prologue: (DENSE) zero the staging blocks, whose pad pixels must
@@ -590,6 +591,12 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
             const int hx = min(win_start(x0, W), W - 14);
             const int qx = min(x0 + r, W - 1), sx = win_start(qx, W);
             const bool colok = x0 + r < W;
+            // this lane's key columns hx + 2J + e: bias-table column b0 + 2J + e,
+            // inside the query's window for the bits set in xmask
+            const int b0 = hx - qx + 6;
+            uint32_t xmask = 0;
+#pragma unroll
+            for (int t = 0; t < 2 * NJ; ++t) xmask |= ((unsigned)(hx + t - sx) < (unsigned)KW ? 1u : 0u) << t;
             const uint32_t kcol = (uint32_t)(hx + lj) * kPixB + 16u * lch;
             const uint32_t qcol = (uint32_t)min(x0 + (lane & 7), W - 1) * kPixB + 16u * (lane >> 4);
             const uint32_t dv = (p.off_v - p.off_k) + 16u * (uint32_t)((lane >> 4) - lch);
@@ -624,16 +631,17 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
 #pragma unroll
                             for (int R = 0; R < 2; ++R) {
                                 const int ky = hy + 4 * R + c;
-                                const bool yv = (unsigned)(ky - sy) < (unsigned)KW;
-                                const float *row = th + clampi(ky - qy + 6, 0, 12) * kTabPitch;
+                                // a key row outside the window masks the whole row
+                                const uint32_t rmask = (unsigned)(ky - sy) < (unsigned)KW ? xmask : 0u;
+                                // table row; columns b0 - 1 .. b0 + 13 stay inside the
+                                // padded table, so the loads need no clamp
+                                const float *row = th + clampi(ky - qy + 6, 0, 12) * kTabPitch + b0;
 #pragma unroll
                                 for (int J = 0; J < NJ; ++J)
 #pragma unroll
                                     for (int e = 0; e < 2; ++e) {
-                                        const int kx = hx + 2 * J + e;
-                                        const bool v = yv && (unsigned)(kx - sx) < (unsigned)KW;
-                                        const float b = row[clampi(kx - qx + 6, 0, 12)];
-                                        bias[R][J][2 * m + e] = v ? b : kMaskC;
+                                        const float b = row[2 * J + e];
+                                        bias[R][J][2 * m + e] = (rmask >> (2 * J + e)) & 1u ? b : kMaskC;
                                     }
                             }
                         }
@@ -803,7 +811,7 @@ uint32_t plan_slide(StreamParams &sp, const Problem &pr, int SP) {
     sp.off_k = align_up(qbytes, 128);
     sp.off_v = sp.off_k + align_up(ring, 128);
     sp.off_tab = sp.off_v + align_up(ring, 128);
-    sp.off_bar = align_up(sp.off_tab + (uint32_t)(pr.heads * kTabHead * 4), 16);
+    sp.off_bar = align_up(sp.off_tab + 128 + (uint32_t)(pr.heads * kTabHead * 4), 16);
     return sp.off_bar + 16 * NS + 16;
 }
 
@@ -856,7 +864,7 @@ cudaError_t launch_stream_impl(const Problem &pr, const void *q, const void *k, 
         sp.off_k = NS * stage_bytes;
         sp.off_v = 2 * NS * stage_bytes;
         sp.off_tab = 3 * NS * stage_bytes;
-        sp.off_bar = align_up(sp.off_tab + (uint32_t)(pr.heads * kTabHead * 4), 16);
+        sp.off_bar = align_up(sp.off_tab + 128 + (uint32_t)(pr.heads * kTabHead * 4), 16);
         const uint32_t smem = sp.off_bar + 16 * NS + 16;
         if ((int)smem > cap) return cudaSuccess;
         return launch_stream_t<T, true, NWC>(sp, smem, sms, st, launched);
