@@ -70,7 +70,7 @@ def hbm_peak() -> tuple[float, str]:
 def recorded_traffic(workload: str) -> int | None:
     """DRAM bytes per launch from the committed ncu summary of this workload,
     only if it was taken on the current kernel source."""
-    f = PROFILES / f"na2d_fwd_tc_{workload}.md"
+    f = PROFILES / f"fwd_stream_kernel_{workload}.md"
     if not f.exists():
         return None
     text = f.read_text()
