@@ -84,7 +84,9 @@ na2d_status na2d_forward(const na2d_problem *p, const void *q, const void *k, co
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (na2d::tc_supported(pr)) {
         bool launched = false;
-        const cudaError_t e = na2d::launch_forward_stream(pr, q, k, v, rpb, out, st, &launched);
+        cudaError_t e = na2d::launch_forward_umma(pr, q, k, v, rpb, out, st, &launched);
+        if (e != cudaSuccess || launched) return from_cuda(e);
+        e = na2d::launch_forward_stream(pr, q, k, v, rpb, out, st, &launched);
         if (e != cudaSuccess || launched) return from_cuda(e);
         return from_cuda(na2d::launch_forward_tc(pr, q, k, v, rpb, out, st));
     }
@@ -132,11 +134,12 @@ na2d_status na2d_av(const na2d_problem *p, const float *attn, const void *v, voi
 
 na2d_status na2d_device_faults(unsigned int *count, void *stream) {
     if (!count) return NA2D_ERR_NULL;
-    unsigned int a = 0, b = 0;
+    unsigned int a = 0, b = 0, c = 0;
     cudaError_t e = na2d::read_device_faults(&a, static_cast<cudaStream_t>(stream));
     if (e == cudaSuccess) e = na2d::read_stream_faults(&b, static_cast<cudaStream_t>(stream));
+    if (e == cudaSuccess) e = na2d::read_umma_faults(&c, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return from_cuda(e);
-    *count = a + b;
+    *count = a + b + c;
     return NA2D_OK;
 }
 

@@ -1,6 +1,7 @@
 // na2d_launch.h -- host-side launchers behind the C ABI (internal).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cstdint>
 
@@ -34,6 +35,22 @@ cudaError_t read_device_faults(unsigned int *count, cudaStream_t stream);
 
 // True when launch_forward_tc handles this problem.
 bool tc_supported(const Problem &p);
+
+// 5-D TMA view (D, gx, j', gy, bh * H / d + i') of a [B*heads, H, W, 32]
+// tensor with H and W multiples of d (pixel (gy + d*i', gx + d*j') of plane
+// bh), 64-byte swizzled boxes of 32 x 1 x box_cols x 1 x box_rows elements.
+// False when the driver entry point is missing or the encoding is refused.
+bool encode_group_map(CUtensorMap *map, const void *base, DType dt, int64_t bh, int H, int W, int d, int box_cols,
+                      int box_rows);
+
+// Forward on the 5th-generation tensor cores (tcgen05) for maps whose
+// dilation groups are all exactly 7 x 7 (H = W = 7d, k = 7, D = 32, f16 /
+// bf16).  Sets *launched when it took the problem.
+bool umma_supported(const Problem &p);
+cudaError_t launch_forward_umma(const Problem &p, const void *q, const void *k, const void *v,
+                                const void *rpb, void *out, cudaStream_t stream, bool *launched);
+// As read_device_faults, for the tcgen05 kernel's counter.
+cudaError_t read_umma_faults(unsigned int *count, cudaStream_t stream);
 
 // Streaming tensor-core forward for k = 7 (f16 / bf16, D = 32): d = 1 maps with
 // 14 <= W <= 64 and H >= 8, or H = W = 7d (every dilation group 7 x 7).  Sets

@@ -1008,6 +1008,11 @@ cudaError_t read_device_faults(unsigned int *count, cudaStream_t st) {
     return e;
 }
 
+bool encode_group_map(CUtensorMap *map, const void *base, DType dt, int64_t bh, int H, int W, int d, int box_cols,
+                      int box_rows) {
+    return encode_map(map, base, dt, bh, H, W, d, box_cols, box_rows);
+}
+
 bool tc_supported(const Problem &p) {
     return (p.dtype == DType::F16 || p.dtype == DType::BF16) && p.D == 32 && p.k >= 3 && p.k <= 13 && (p.k & 1);
 }

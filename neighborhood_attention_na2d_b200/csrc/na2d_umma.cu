@@ -1,0 +1,579 @@
+// na2d_umma.cu -- NA2D forward on the 5th-generation tensor cores (tcgen05)
+// for maps whose dilation groups are all exactly 7 x 7: H = W = 7d, k = 7,
+// D = 32, f16 / bf16.
+//
+// What it computes is the same as na2d_tc.cu ("Dilated Neighborhood Attention
+// Transformer", gitcode DiNAT article, section "DiNAT 的核心思想":
+// natten2dqkrpb -> softmax -> natten2dav, fused, NATTEN clamp rule).  When a
+// dilation group is exactly k = 7 long on both axes, every query of the group
+// has the whole group as its window (clamped start 0), so a group is a dense
+// 49 x 49 attention with a relative-position bias.
+//
+// Work unit: two groups, A and B, as one M = 128 tile.  Each group's Q, K
+// and V arrive by TMA as an 8 x 8 block of pixels (7 x 7 plus a zero-filled
+// column and a spare row), 64 bytes per pixel, 64-byte swizzled: slot
+// s = 8 * row + col is tile row s (A) or 64 + s (B).
+//   1. S = Q K^T: two tcgen05.mma (K = 16 each, A and B K-major in shared
+//      memory), S = [128 x 128] fp32 in tensor memory (TMEM).  Only the
+//      diagonal 64 x 64 blocks (a query and a key of the same group) are used.
+//   2. softmax: one thread per tile row (its TMEM lane) loads its 56 scores,
+//      adds the bias (pre-multiplied by sqrt(D), kept in registers per head),
+//      exponentiates in fp32 and writes P as 16-bit pairs over its own S
+//      columns: 32 columns for its group's 64 keys and 32 columns of zeros for
+//      the other group's keys.
+//   3. O = P V: eight tcgen05.mma with A = P in TMEM and B = V (MN-major in
+//      shared memory), O = [128 x 32] fp32 in TMEM.
+//   4. epilogue: the same thread loads its O row, divides by its row sum and
+//      stores 64 bytes.
+// Warps 0-3 and 4-7 are two softmax warpgroups taking alternate units, each
+// with its own S / P and O columns (TMEM columns 0-127 / 128-255 and
+// 256-287 / 288-319), so one warpgroup's softmax overlaps the other's MMAs
+// and epilogue.  Warp 8, lane 0 issues the TMA copies into a ring of NSTG
+// stages; warp 9, lane 0 issues the MMAs and signals completion with
+// tcgen05.commit on mbarriers; warp 9 owns the TMEM allocation.  Every wait is
+// bounded: one that runs out counts the event, raises the block's abort flag,
+// and the block winds down (its MMAs and copies in flight are waited for
+// before TMEM and shared memory are released).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <map>
+#include <mutex>
+#include <set>
+#include <type_traits>
+
+#include "na2d_device.cuh"
+#include "na2d_launch.h"
+
+namespace na2d {
+namespace {
+
+constexpr int KW = 7;
+constexpr int NSTG = 6;                  // shared-memory stages (units in flight)
+constexpr uint32_t kBlk = 4096;          // one group's 8 x 8 block of one tensor
+constexpr uint32_t kTile = 2 * kBlk;     // one tensor of a unit (128 rows of 64 bytes)
+constexpr uint32_t kStage = 3 * kTile;   // Q, K, V tiles of a unit
+constexpr int kTabPitch = 16;            // floats per bias-table row (13 used)
+constexpr int kTabHead = 13 * kTabPitch;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kThreads = 320;            // 8 softmax warps, producer warp, MMA warp
+constexpr int kWarpTma = 8, kWarpMma = 9;
+
+__device__ unsigned int g_umma_timeouts;
+
+struct UmmaParams {
+    CUtensorMap tq, tk, tv;   // 5-D group views, 32 x 1 x 8 x 1 x 8 boxes
+    unsigned char *out;
+    const void *rpb;
+    int H, W, heads, d;
+    int GU;                   // groups: B * heads * d * d
+    int NU;                   // units: ceil(GU / 2)
+    float c_log2;             // log2(e) / sqrt(D)
+    float sqrt_d;
+    uint32_t off_tab, off_bar;   // byte offsets from the 1024-aligned base
+};
+
+// ---- mbarriers ---------------------------------------------------------------
+__device__ __forceinline__ void mb_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ bool mb_try(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(20000)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait: gives up after about 2^31 SM clocks (about a second).
+__device__ __forceinline__ bool mb_wait(uint32_t bar, uint32_t parity) {
+    if (mb_try(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mb_try(bar, parity))
+        if (clock64() - t0 > (1LL << 31)) return false;
+    return true;
+}
+__device__ __forceinline__ void mb_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mb_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+// ---- TMA ---------------------------------------------------------------------
+__device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap *map, uint32_t bar, int c1, int c2,
+                                            int c3, int c4) {
+    asm volatile(
+        "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, "
+        "%5, %6}], [%7];\n" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "r"(bar)
+        : "memory");
+}
+
+// ---- TMEM --------------------------------------------------------------------
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(dst_smem),
+                 "n"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(taddr), "n"(kTmemCols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
+
+// Loads N consecutive 32-bit columns of this thread's lane (complete after
+// tmem_ld_wait).
+__device__ __forceinline__ void tmem_ld8(uint32_t ta, float *v) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n"
+                 : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7])
+                 : "r"(ta)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t ta, float *v) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+        : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7]),
+          "=f"(v[8]), "=f"(v[9]), "=f"(v[10]), "=f"(v[11]), "=f"(v[12]), "=f"(v[13]), "=f"(v[14]), "=f"(v[15])
+        : "r"(ta)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t ta, float *v) {
+    tmem_ld16(ta, v);
+    tmem_ld16(ta + 16, v + 16);
+}
+// Stores 16 consecutive 32-bit columns of this thread's lane.
+__device__ __forceinline__ void tmem_st16(uint32_t ta, const uint32_t *v) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n" ::"r"(
+            ta),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+        "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+        : "memory");
+}
+
+// ---- MMA -----------------------------------------------------------------------
+// Shared-memory matrix descriptor, 64-byte swizzle (the layout the TMA copies
+// write: 16-byte chunk c of the 64-byte row at byte address a stored at chunk
+// c ^ ((a >> 7) & 3)); byte offsets in 16-byte units; version 1.
+__device__ __forceinline__ uint64_t sw64_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (4ull << 61);
+}
+// Instruction descriptor of kind::f16: fp32 accumulator, A and B of type T,
+// A K-major, B K-major (b_mn = 0) or MN-major (1), M = 128.
+template <typename T> __host__ __device__ constexpr uint32_t idesc_f16(int N, int b_mn) {
+    return (1u << 4) | ((std::is_same<T, __nv_bfloat16>::value ? 1u : 0u) << 7) |
+           ((std::is_same<T, __nv_bfloat16>::value ? 1u : 0u) << 10) | ((uint32_t)b_mn << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+// D[tmem] (+)= A[smem] * B[smem]
+__device__ __forceinline__ void umma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
+            d),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+// D[tmem] (+)= A[tmem] * B[smem]
+__device__ __forceinline__ void umma_ts(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(
+            d),
+        "r"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+// Arrives once on the mbarrier when every earlier tcgen05.mma of this thread
+// has completed.
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)
+                 : "memory");
+}
+
+template <typename T> struct Pack2;
+template <> struct Pack2<__half> {
+    __device__ __forceinline__ static uint32_t run(float lo, float hi) {
+        uint32_t e;
+        asm("cvt.rn.f16x2.f32 %0, %1, %2;\n" : "=r"(e) : "f"(hi), "f"(lo));
+        return e;
+    }
+};
+template <> struct Pack2<__nv_bfloat16> {
+    __device__ __forceinline__ static uint32_t run(float lo, float hi) {
+        uint32_t e;
+        asm("cvt.rn.bf16x2.f32 %0, %1, %2;\n" : "=r"(e) : "f"(hi), "f"(lo));
+        return e;
+    }
+};
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;\n" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// ---------------------------------------------------------------------------
+// Kernel.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(kThreads, 1) fwd_umma_kernel(const __grid_constant__ UmmaParams p) {
+    extern __shared__ unsigned char smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t sbase = (raw + 1023u) & ~1023u;   // swizzled tiles need 1024-byte alignment
+    unsigned char *smem = smem_raw + (sbase - raw);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int u_begin = (int)((int64_t)p.NU * blockIdx.x / gridDim.x);
+    const int u_end = (int)((int64_t)p.NU * (blockIdx.x + 1) / gridDim.x);
+    if (u_begin >= u_end) return;
+    const int nst = u_end - u_begin;
+    const int dd = p.d * p.d;
+
+    float *tab = reinterpret_cast<float *>(smem + p.off_tab);
+    const uint32_t bar_full = sbase + p.off_bar;        // [NSTG] stage landed (TMA bytes)
+    const uint32_t bar_empty = bar_full + 8 * NSTG;     // [NSTG] stage consumed (commit)
+    const uint32_t bar_s = bar_empty + 8 * NSTG;        // [2] S ready (commit)
+    const uint32_t bar_p = bar_s + 16;                  // [2] P written (4 warps)
+    const uint32_t bar_o = bar_p + 16;                  // [2] O ready (commit)
+    const uint32_t bar_drain = bar_o + 16;              // all MMAs done (commit)
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + p.off_bar + 16 * NSTG + 56);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + p.off_bar + 16 * NSTG + 60);
+
+    // ---- prologue: zero the stages (pad pixels and a missing second group
+    // must hold finite values), bias table, barriers, TMEM.
+    {
+        uint4 *z = reinterpret_cast<uint4 *>(smem);
+        for (int i = threadIdx.x; i < (int)(NSTG * kStage / 16); i += kThreads) z[i] = make_uint4(0, 0, 0, 0);
+        const T *rpb = reinterpret_cast<const T *>(p.rpb);
+        for (int i = threadIdx.x; i < p.heads * kTabHead; i += kThreads) {
+            const int h = i / kTabHead, a = (i / kTabPitch) % 13, b = i % kTabPitch;
+            float v = 0.f;
+            if (rpb && b < 13) v = Elem<T>::to_f(rpb[(h * 13 + a) * 13 + b]) * p.sqrt_d;
+            tab[i] = v;
+        }
+        if (threadIdx.x == 0) {
+            for (int i = 0; i < NSTG; ++i) {
+                mb_init(bar_full + 8 * i, 1);
+                mb_init(bar_empty + 8 * i, 1);
+            }
+            for (int i = 0; i < 2; ++i) {
+                mb_init(bar_s + 8 * i, 1);
+                mb_init(bar_p + 8 * i, 4);
+                mb_init(bar_o + 8 * i, 1);
+            }
+            mb_init(bar_drain, 1);
+            *abort_flag = 0;
+            asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+        }
+        // the zeros (generic proxy) are ordered before the TMA writes and MMA
+        // reads (async proxy) of the same bytes
+        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+        if (warp == kWarpMma) tmem_alloc(smem_u32(tmem_slot));
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    }
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == kWarpTma) {
+        // =================== TMA producer ===================
+        if (lane == 0) {
+            int issued = 0;
+            for (int j = 0; j < nst; ++j) {
+                const int s = j % NSTG;
+                if (j >= NSTG && !mb_wait(bar_empty + 8 * s, (uint32_t)(((j / NSTG) - 1) & 1))) {
+                    atomicAdd(&g_umma_timeouts, 1u);
+                    *abort_flag = 1;
+                    break;
+                }
+                if (*abort_flag) break;
+                const int g0 = 2 * (u_begin + j);
+                const int ng = g0 + 1 < p.GU ? 2 : 1;
+                const uint32_t fb = bar_full + 8 * s;
+                const uint32_t st = sbase + (uint32_t)s * kStage;
+                mb_expect_tx(fb, (uint32_t)(3 * ng) * kBlk);
+                for (int e = 0; e < ng; ++e) {
+                    const int g = g0 + e;
+                    const int bh = g / dd, rem = g - bh * dd, gy = rem / p.d, gx = rem - gy * p.d;
+                    const int row = bh * KW;   // merged (plane, group row) coordinate of group row 0
+                    tma_load_5d(st + (uint32_t)e * kBlk, &p.tq, fb, gx, 0, gy, row);
+                    tma_load_5d(st + kTile + (uint32_t)e * kBlk, &p.tk, fb, gx, 0, gy, row);
+                    tma_load_5d(st + 2 * kTile + (uint32_t)e * kBlk, &p.tv, fb, gx, 0, gy, row);
+                }
+                ++issued;
+            }
+            // copies still in flight land before shared memory is released
+            for (int j = max(0, issued - NSTG); j < issued; ++j)
+                mb_wait(bar_full + 8 * (j % NSTG), (uint32_t)((j / NSTG) & 1));
+        }
+    } else if (warp == kWarpMma) {
+        // =================== MMA issuer ===================
+        if (lane == 0) {
+            constexpr uint32_t idesc_qk = idesc_f16<T>(128, 0);
+            constexpr uint32_t idesc_pv = idesc_f16<T>(32, 1);
+            for (int j = 0; j <= nst; ++j) {
+                if (j < nst) {
+                    // S_j = Q K^T into S buffer j & 1 (free: its previous
+                    // unit's P was consumed by a P.V issued earlier)
+                    const int s = j % NSTG;
+                    if (!mb_wait(bar_full + 8 * s, (uint32_t)((j / NSTG) & 1))) {
+                        atomicAdd(&g_umma_timeouts, 1u);
+                        *abort_flag = 1;
+                        break;
+                    }
+                    if (*abort_flag) break;
+                    tc_fence_after();
+                    const uint32_t st = sbase + (uint32_t)s * kStage;
+                    // K-major, 64-byte rows: 8-row groups 512 bytes apart; the
+                    // second K = 16 step starts 32 bytes into the rows
+                    const uint64_t da = sw64_desc(st, 16, 512), db = sw64_desc(st + kTile, 16, 512);
+                    const uint32_t dS = tmem + (uint32_t)(j & 1) * 128;
+                    umma_ss(dS, da, db, idesc_qk, 0);
+                    umma_ss(dS, da + 2, db + 2, idesc_qk, 1);
+                    umma_commit(bar_s + 8 * (j & 1));
+                }
+                if (j >= 1) {
+                    // O_{j-1} = P V
+                    const int jp = j - 1, b = jp & 1, s = jp % NSTG;
+                    if (!mb_wait(bar_p + 8 * b, (uint32_t)((jp >> 1) & 1))) {
+                        atomicAdd(&g_umma_timeouts, 1u);
+                        *abort_flag = 1;
+                        break;
+                    }
+                    if (*abort_flag) break;
+                    tc_fence_after();
+                    const uint32_t vt = sbase + (uint32_t)s * kStage + 2 * kTile;
+                    const uint32_t dO = tmem + 256u + (uint32_t)b * 32;
+                    const uint32_t aP = tmem + (uint32_t)b * 128;
+                    // V MN-major: 64-byte rows of 32 channels, 8-key groups
+                    // 512 bytes apart; k-step t takes keys 16t .. 16t + 15
+#pragma unroll
+                    for (int t = 0; t < 8; ++t)
+                        umma_ts(dO, aP + 8u * t, sw64_desc(vt + 1024u * t, 16, 512), idesc_pv, t > 0 ? 1u : 0u);
+                    umma_commit(bar_o + 8 * b);
+                    umma_commit(bar_empty + 8 * s);
+                }
+            }
+            // every MMA issued has completed before TMEM is released
+            umma_commit(bar_drain);
+            mb_wait(bar_drain, 0);
+        }
+    } else {
+        // =================== softmax warpgroups ===================
+        const int w = warp >> 2;                      // warpgroup = TMEM buffer set
+        const int q4 = warp & 3;                      // lane quarter of this warp
+        const int m = q4 * 32 + lane;                 // tile row = TMEM lane
+        const int e = m >> 6;                         // group A (0) or B (1); uniform per warp
+        const int slot = m & 63, qy = slot >> 3, qx = slot & 7;
+        const bool qok = qy < KW && qx < KW;
+        const int qyc = min(qy, KW - 1), qxc = min(qx, KW - 1);
+        const uint32_t tl = tmem + ((uint32_t)(32 * q4) << 16);
+        const uint32_t tS = tl + (uint32_t)w * 128 + (uint32_t)e * 64;
+        const uint32_t tP = tl + (uint32_t)w * 128;
+        const uint32_t tO = tl + 256u + (uint32_t)w * 32;
+        const float c = p.c_log2;
+        float bias[KW * KW];
+        int cur_h = -1;
+        for (int j = w, k = 0; j < nst; j += 2, ++k) {
+            const int g = 2 * (u_begin + j) + e;
+            const bool gok = g < p.GU;
+            const int bh = gok ? g / dd : 0;
+            const int h = bh % p.heads;
+            if (h != cur_h) {
+                cur_h = h;
+                // bias of key (ky, kx): table row ky - qy + 6, column kx - qx + 6
+                const float *tb = tab + h * kTabHead + (6 - qyc) * kTabPitch + (6 - qxc);
+#pragma unroll
+                for (int ky = 0; ky < KW; ++ky)
+#pragma unroll
+                    for (int kx = 0; kx < KW; ++kx) bias[ky * KW + kx] = tb[ky * kTabPitch + kx];
+            }
+            bool ok = mb_wait(bar_s + 8 * w, (uint32_t)(k & 1));
+            if (!__all_sync(0xffffffffu, ok) || __any_sync(0xffffffffu, *abort_flag != 0)) {
+                if (lane == 0) {
+                    atomicAdd(&g_umma_timeouts, 1u);
+                    *abort_flag = 1;
+                }
+                break;
+            }
+            tc_fence_after();
+            // scores of keys 8 * ky + kx, ky, kx < 8 (kx = 7 and ky = 7 are pads)
+            float s[56];
+            tmem_ld32(tS, s);
+            tmem_ld16(tS + 32, s + 32);
+            tmem_ld8(tS + 48, s + 48);
+            tmem_ld_wait();
+            float mx = -3.0e38f;
+#pragma unroll
+            for (int ky = 0; ky < KW; ++ky) {
+#pragma unroll
+                for (int kx = 0; kx < KW; ++kx) s[ky * 8 + kx] += bias[ky * KW + kx];
+                mx = max3(mx, max3(s[ky * 8 + 0], s[ky * 8 + 1], s[ky * 8 + 2]),
+                          max3(s[ky * 8 + 3], s[ky * 8 + 4], fmaxf(s[ky * 8 + 5], s[ky * 8 + 6])));
+            }
+            const float nm = -mx * c;
+            float l = 0.f;
+            uint32_t pk[32];
+#pragma unroll
+            for (int i = 0; i < 28; ++i) {
+                const float p0 = ex2(fmaf(s[2 * i], c, nm));
+                const float p1 = ((2 * i + 1) & 7) < KW ? ex2(fmaf(s[2 * i + 1], c, nm)) : 0.f;
+                l += p0 + p1;
+                pk[i] = Pack2<T>::run(p0, p1);
+            }
+#pragma unroll
+            for (int i = 28; i < 32; ++i) pk[i] = 0u;
+            uint32_t zero[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) zero[i] = 0u;
+            // own group's keys: P columns 32e .. 32e + 31; the other group's: zeros
+            tmem_st16(tP + (uint32_t)e * 32, pk);
+            tmem_st16(tP + (uint32_t)e * 32 + 16, pk + 16);
+            tmem_st16(tP + (uint32_t)(e ^ 1) * 32, zero);
+            tmem_st16(tP + (uint32_t)(e ^ 1) * 32 + 16, zero);
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mb_arrive(bar_p + 8 * w);
+            // ---- epilogue
+            ok = mb_wait(bar_o + 8 * w, (uint32_t)(k & 1));
+            if (!__all_sync(0xffffffffu, ok)) {
+                if (lane == 0) {
+                    atomicAdd(&g_umma_timeouts, 1u);
+                    *abort_flag = 1;
+                }
+                break;
+            }
+            tc_fence_after();
+            float o[32];
+            tmem_ld32(tO, o);
+            tmem_ld_wait();
+            if (gok && qok) {
+                float inv;
+                asm("rcp.approx.ftz.f32 %0, %1;\n" : "=f"(inv) : "f"(l));
+                const int rem = g - bh * dd, gy = rem / p.d, gx = rem - gy * p.d;
+                uint4 *dst = reinterpret_cast<uint4 *>(
+                    p.out + ((((size_t)bh * p.H + gy + (size_t)p.d * qy) * p.W) + gx + (size_t)p.d * qx) * 64);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    dst[i] = make_uint4(Pack2<T>::run(o[8 * i + 0] * inv, o[8 * i + 1] * inv),
+                                        Pack2<T>::run(o[8 * i + 2] * inv, o[8 * i + 3] * inv),
+                                        Pack2<T>::run(o[8 * i + 4] * inv, o[8 * i + 5] * inv),
+                                        Pack2<T>::run(o[8 * i + 6] * inv, o[8 * i + 7] * inv));
+            }
+        }
+    }
+    // ---- teardown: TMEM released by the warp that took it, after every
+    // thread is done with it
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kWarpMma) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Host side.
+// ---------------------------------------------------------------------------
+struct UmmaCache {
+    std::mutex mu;
+    std::map<int, std::pair<int, int>> dev;   // device -> (SMs, opt-in smem per block)
+    std::set<std::pair<int, const void *>> attr;
+};
+UmmaCache &ucache() {
+    static UmmaCache c;
+    return c;
+}
+
+cudaError_t umma_device(int *sms, int *smem_cap, const void *kern) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    UmmaCache &c = ucache();
+    std::lock_guard<std::mutex> lock(c.mu);
+    auto it = c.dev.find(dev);
+    if (it == c.dev.end()) {
+        int n = 0, m = 0;
+        if ((e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+        if ((e = cudaDeviceGetAttribute(&m, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) return e;
+        it = c.dev.emplace(dev, std::make_pair(n, m)).first;
+    }
+    *sms = it->second.first;
+    *smem_cap = it->second.second;
+    if (!c.attr.count({dev, kern})) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, *smem_cap);
+        if (e != cudaSuccess) return e;
+        c.attr.insert({dev, kern});
+    }
+    return cudaSuccess;
+}
+
+uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
+
+template <typename T>
+cudaError_t launch_umma_t(const Problem &pr, const void *q, const void *k, const void *v, const void *rpb, void *out,
+                          cudaStream_t st, bool *launched) {
+    const void *kern = reinterpret_cast<const void *>(&fwd_umma_kernel<T>);
+    int sms = 0, cap = 0;
+    cudaError_t e = umma_device(&sms, &cap, kern);
+    if (e != cudaSuccess) return e;
+    UmmaParams up{};
+    const int64_t bh = pr.bh();
+    const int64_t gu = bh * pr.d * pr.d;
+    if (gu <= 0 || gu >= INT32_MAX || bh * KW >= INT32_MAX) return cudaSuccess;
+    if (!encode_group_map(&up.tq, q, pr.dtype, bh, pr.H, pr.W, pr.d, 8, 8) ||
+        !encode_group_map(&up.tk, k, pr.dtype, bh, pr.H, pr.W, pr.d, 8, 8) ||
+        !encode_group_map(&up.tv, v, pr.dtype, bh, pr.H, pr.W, pr.d, 8, 8))
+        return cudaSuccess;
+    up.out = static_cast<unsigned char *>(out);
+    up.rpb = rpb;
+    up.H = pr.H; up.W = pr.W; up.heads = pr.heads; up.d = pr.d;
+    up.GU = (int)gu;
+    up.NU = (int)((gu + 1) / 2);
+    up.c_log2 = kLog2e / std::sqrt((float)pr.D);
+    up.sqrt_d = std::sqrt((float)pr.D);
+    up.off_tab = NSTG * kStage;
+    up.off_bar = align_up(up.off_tab + (uint32_t)(pr.heads * kTabHead * 4), 16);
+    // + 1024 bytes for aligning the base; at least 116 KB so that two blocks
+    // never share an SM (each takes all 512 TMEM columns)
+    const uint32_t smem = std::max<uint32_t>(up.off_bar + 16 * NSTG + 64 + 1024, 116u * 1024u);
+    if ((int)smem > cap) return cudaSuccess;
+    const int grid = std::min(up.NU, sms);
+    fwd_umma_kernel<T><<<grid, kThreads, smem, st>>>(up);
+    *launched = true;
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool umma_supported(const Problem &p) {
+    if (p.dtype != DType::F16 && p.dtype != DType::BF16) return false;
+    return p.k == KW && p.D == 32 && p.heads <= 64 && p.H == KW * p.d && p.W == KW * p.d;
+}
+
+cudaError_t launch_forward_umma(const Problem &p, const void *q, const void *k, const void *v, const void *rpb,
+                                void *out, cudaStream_t st, bool *launched) {
+    *launched = false;
+    if (!umma_supported(p)) return cudaSuccess;
+    if (p.dtype == DType::F16) return launch_umma_t<__half>(p, q, k, v, rpb, out, st, launched);
+    return launch_umma_t<__nv_bfloat16>(p, q, k, v, rpb, out, st, launched);
+}
+
+cudaError_t read_umma_faults(unsigned int *count, cudaStream_t st) {
+    unsigned int zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbolAsync(count, g_umma_timeouts, sizeof(unsigned int), 0,
+                                              cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess)
+        e = cudaMemcpyToSymbolAsync(g_umma_timeouts, &zero, sizeof(unsigned int), 0, cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    return e;
+}
+
+}  // namespace na2d
