@@ -38,10 +38,11 @@ bool tc_supported(const Problem &p);
 
 // 5-D TMA view (D, gx, j', gy, bh * H / d + i') of a [B*heads, H, W, 32]
 // tensor with H and W multiples of d (pixel (gy + d*i', gx + d*j') of plane
-// bh), 64-byte swizzled boxes of 32 x 1 x box_cols x 1 x box_rows elements.
-// False when the driver entry point is missing or the encoding is refused.
+// bh), 64-byte swizzled boxes of 32 x box_gx x box_cols x 1 x box_rows
+// elements (box_gx adjacent groups side by side).  False when the driver
+// entry point is missing or the encoding is refused.
 bool encode_group_map(CUtensorMap *map, const void *base, DType dt, int64_t bh, int H, int W, int d, int box_cols,
-                      int box_rows);
+                      int box_rows, int box_gx);
 
 // Forward on the 5th-generation tensor cores (tcgen05) for maps whose
 // dilation groups are all exactly 7 x 7 (H = W = 7d, k = 7, D = 32, f16 /

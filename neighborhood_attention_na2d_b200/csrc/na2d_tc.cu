@@ -881,12 +881,12 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 // H and W multiples of d: pixel (gy + d*i', gx + d*j') of plane bh.  Strides
 // are non-decreasing, each the product of the previous extent and stride.
 bool encode_map(CUtensorMap *m, const void *base, DType dt, int64_t bh, int H, int W, int d, int box_cols,
-                int box_rows) {
+                int box_rows, int box_gx = 1) {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
     const cuuint64_t dims[5] = {32, (cuuint64_t)d, (cuuint64_t)(W / d), (cuuint64_t)d, (cuuint64_t)bh * (H / d)};
     const cuuint64_t strides[4] = {64, 64ull * d, 64ull * W, 64ull * W * d};
-    const cuuint32_t box[5] = {32, 1, (cuuint32_t)box_cols, 1, (cuuint32_t)box_rows};
+    const cuuint32_t box[5] = {32, (cuuint32_t)box_gx, (cuuint32_t)box_cols, 1, (cuuint32_t)box_rows};
     const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
     const CUresult r = enc(m, dt == DType::F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5,
                            const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -1009,8 +1009,8 @@ cudaError_t read_device_faults(unsigned int *count, cudaStream_t st) {
 }
 
 bool encode_group_map(CUtensorMap *map, const void *base, DType dt, int64_t bh, int H, int W, int d, int box_cols,
-                      int box_rows) {
-    return encode_map(map, base, dt, bh, H, W, d, box_cols, box_rows);
+                      int box_rows, int box_gx) {
+    return encode_map(map, base, dt, bh, H, W, d, box_cols, box_rows, box_gx);
 }
 
 bool tc_supported(const Problem &p) {

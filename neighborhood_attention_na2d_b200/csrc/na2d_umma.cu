@@ -10,9 +10,10 @@
 // 49 x 49 attention with a relative-position bias.
 //
 // Work unit: two groups, A and B, as one M = 128 tile.  Each group's Q, K
-// and V arrive by TMA as an 8 x 8 block of pixels (7 x 7 plus a zero-filled
-// column and a spare row), 64 bytes per pixel, 64-byte swizzled: slot
-// s = 8 * row + col is tile row s (A) or 64 + s (B).
+// and V arrive by TMA as a 7 x 8 box of pixels (the group's 7 x 7 and a
+// zero-filled column), 64 bytes per pixel, 64-byte swizzled: slot
+// s = 8 * row + col is tile row s (A) or 64 + s (B); slot row 7 is a spare
+// that holds zeros.
 //   1. S = Q K^T: two tcgen05.mma (K = 16 each, A and B K-major in shared
 //      memory), S = [128 x 128] fp32 in tensor memory (TMEM).  Only the
 //      diagonal 64 x 64 blocks (a query and a key of the same group) are used.
@@ -26,14 +27,18 @@
 //   4. epilogue: the same thread loads its O row, divides by its row sum and
 //      stores 64 bytes.
 // Warps 0-3 and 4-7 are two softmax warpgroups taking alternate units, each
-// with its own S / P and O columns (TMEM columns 0-127 / 128-255 and
-// 256-287 / 288-319), so one warpgroup's softmax overlaps the other's MMAs
-// and epilogue.  Warp 8, lane 0 issues the TMA copies into a ring of NSTG
-// stages; warp 9, lane 0 issues the MMAs and signals completion with
-// tcgen05.commit on mbarriers; warp 9 owns the TMEM allocation.  Every wait is
-// bounded: one that runs out counts the event, raises the block's abort flag,
-// and the block winds down (its MMAs and copies in flight are waited for
-// before TMEM and shared memory are released).
+// with its own S / P columns (TMEM columns 0-127 / 128-255); O rotates over
+// four 32-column buffers (256-383).  A warpgroup runs the softmax of its
+// unit j and then the epilogue of its unit j - 2, so it never waits for a
+// P.V that was just issued, and one warpgroup's softmax overlaps the other's
+// MMAs and epilogue.  Warp 8, lane 0 issues the TMA copies into a ring of
+// NSTG stages; warp 9, lane 0 issues the MMAs (each unit's P.V before the
+// Q K^T two units ahead, so a P.V never waits for a copy) and signals
+// completion with tcgen05.commit on mbarriers; warp 9 owns the TMEM
+// allocation.  Every wait is bounded: one that runs out counts the event,
+// raises the block's abort flag, and the block winds down (its MMAs and
+// copies in flight are waited for before TMEM and shared memory are
+// released).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -53,6 +58,7 @@ namespace {
 constexpr int KW = 7;
 constexpr int NSTG = 6;                  // shared-memory stages (units in flight)
 constexpr uint32_t kBlk = 4096;          // one group's 8 x 8 block of one tensor
+constexpr uint32_t kRowsBytes = 56 * 64; // the 7 x 8 slots a copy writes (slot row 7 is spare)
 constexpr uint32_t kTile = 2 * kBlk;     // one tensor of a unit (128 rows of 64 bytes)
 constexpr uint32_t kStage = 3 * kTile;   // Q, K, V tiles of a unit
 constexpr int kTabPitch = 16;            // floats per bias-table row (13 used)
@@ -239,24 +245,38 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_umma_kernel(const __grid_cons
     const uint32_t bar_empty = bar_full + 8 * NSTG;     // [NSTG] stage consumed (commit)
     const uint32_t bar_s = bar_empty + 8 * NSTG;        // [2] S ready (commit)
     const uint32_t bar_p = bar_s + 16;                  // [2] P written (4 warps)
-    const uint32_t bar_o = bar_p + 16;                  // [2] O ready (commit)
-    const uint32_t bar_drain = bar_o + 16;              // all MMAs done (commit)
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + p.off_bar + 16 * NSTG + 56);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + p.off_bar + 16 * NSTG + 60);
+    const uint32_t bar_o = bar_p + 16;                  // [4] O ready (commit)
+    const uint32_t bar_drain = bar_o + 32;              // all MMAs done (commit)
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + p.off_bar + 16 * NSTG + 72);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + p.off_bar + 16 * NSTG + 76);
 
-    // ---- prologue: zero the stages (pad pixels and a missing second group
-    // must hold finite values), bias table, barriers, TMEM.
-    {
-        uint4 *z = reinterpret_cast<uint4 *>(smem);
-        for (int i = threadIdx.x; i < (int)(NSTG * kStage / 16); i += kThreads) z[i] = make_uint4(0, 0, 0, 0);
-        const T *rpb = reinterpret_cast<const T *>(p.rpb);
-        for (int i = threadIdx.x; i < p.heads * kTabHead; i += kThreads) {
-            const int h = i / kTabHead, a = (i / kTabPitch) % 13, b = i % kTabPitch;
-            float v = 0.f;
-            if (rpb && b < 13) v = Elem<T>::to_f(rpb[(h * 13 + a) * 13 + b]) * p.sqrt_d;
-            tab[i] = v;
+    // One unit's copies into stage j % NSTG: Q, K, V of groups 2u and 2u + 1;
+    // a unit without a second group loads the first one twice (finite
+    // values; its outputs are not stored).
+    auto issue_unit = [&](int j) {
+        const uint32_t fb = bar_full + 8 * (j % NSTG);
+        const uint32_t st = sbase + (uint32_t)(j % NSTG) * kStage;
+        mb_expect_tx(fb, 6u * kRowsBytes);
+        const int g0 = 2 * (u_begin + j);
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int g = min(g0 + e, p.GU - 1);
+            const int bh = g / dd, rem = g - bh * dd, gy = rem / p.d, gx = rem - gy * p.d;
+            const int row = bh * KW;   // merged (plane, group row) coordinate of group row 0
+            tma_load_5d(st + (uint32_t)e * kBlk, &p.tq, fb, gx, 0, gy, row);
+            tma_load_5d(st + kTile + (uint32_t)e * kBlk, &p.tk, fb, gx, 0, gy, row);
+            tma_load_5d(st + 2 * kTile + (uint32_t)e * kBlk, &p.tv, fb, gx, 0, gy, row);
         }
-        if (threadIdx.x == 0) {
+    };
+    const int n_first = min(NSTG, nst);   // units whose copies start in the prologue
+
+    // ---- prologue.  The producer thread initialises the barriers and starts
+    // the first NSTG units' copies at once; meanwhile the other threads zero
+    // the spare slot row 7 of every block, which the 7-row copies never write
+    // (V's must be finite: P is 0 there, and 0 * NaN would not be), build the
+    // bias table and allocate TMEM.
+    {
+        if (warp == kWarpTma && lane == 0) {
             for (int i = 0; i < NSTG; ++i) {
                 mb_init(bar_full + 8 * i, 1);
                 mb_init(bar_empty + 8 * i, 1);
@@ -264,14 +284,27 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_umma_kernel(const __grid_cons
             for (int i = 0; i < 2; ++i) {
                 mb_init(bar_s + 8 * i, 1);
                 mb_init(bar_p + 8 * i, 4);
-                mb_init(bar_o + 8 * i, 1);
             }
+            for (int i = 0; i < 4; ++i) mb_init(bar_o + 8 * i, 1);
             mb_init(bar_drain, 1);
             *abort_flag = 0;
             asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+            for (int j = 0; j < n_first; ++j) issue_unit(j);
         }
-        // the zeros (generic proxy) are ordered before the TMA writes and MMA
-        // reads (async proxy) of the same bytes
+        // 6 * NSTG blocks x 512 bytes (slots 56 .. 63)
+        for (int i = threadIdx.x; i < 6 * NSTG * 32; i += kThreads) {
+            uint4 *z = reinterpret_cast<uint4 *>(smem + (i >> 5) * kBlk + kRowsBytes) + (i & 31);
+            *z = make_uint4(0, 0, 0, 0);
+        }
+        const T *rpb = reinterpret_cast<const T *>(p.rpb);
+        for (int i = threadIdx.x; i < p.heads * kTabHead; i += kThreads) {
+            const int h = i / kTabHead, a = (i / kTabPitch) % 13, b = i % kTabPitch;
+            float v = 0.f;
+            if (rpb && b < 13) v = Elem<T>::to_f(rpb[(h * 13 + a) * 13 + b]) * p.sqrt_d;
+            tab[i] = v;
+        }
+        // the zeros (generic proxy) are ordered before the MMA reads (async
+        // proxy) of the same bytes
         asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
         if (warp == kWarpMma) tmem_alloc(smem_u32(tmem_slot));
         tc_fence_before();
@@ -283,28 +316,16 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_umma_kernel(const __grid_cons
     if (warp == kWarpTma) {
         // =================== TMA producer ===================
         if (lane == 0) {
-            int issued = 0;
-            for (int j = 0; j < nst; ++j) {
+            int issued = n_first;
+            for (int j = n_first; j < nst; ++j) {
                 const int s = j % NSTG;
-                if (j >= NSTG && !mb_wait(bar_empty + 8 * s, (uint32_t)(((j / NSTG) - 1) & 1))) {
+                if (!mb_wait(bar_empty + 8 * s, (uint32_t)(((j / NSTG) - 1) & 1))) {
                     atomicAdd(&g_umma_timeouts, 1u);
                     *abort_flag = 1;
                     break;
                 }
                 if (*abort_flag) break;
-                const int g0 = 2 * (u_begin + j);
-                const int ng = g0 + 1 < p.GU ? 2 : 1;
-                const uint32_t fb = bar_full + 8 * s;
-                const uint32_t st = sbase + (uint32_t)s * kStage;
-                mb_expect_tx(fb, (uint32_t)(3 * ng) * kBlk);
-                for (int e = 0; e < ng; ++e) {
-                    const int g = g0 + e;
-                    const int bh = g / dd, rem = g - bh * dd, gy = rem / p.d, gx = rem - gy * p.d;
-                    const int row = bh * KW;   // merged (plane, group row) coordinate of group row 0
-                    tma_load_5d(st + (uint32_t)e * kBlk, &p.tq, fb, gx, 0, gy, row);
-                    tma_load_5d(st + kTile + (uint32_t)e * kBlk, &p.tk, fb, gx, 0, gy, row);
-                    tma_load_5d(st + 2 * kTile + (uint32_t)e * kBlk, &p.tv, fb, gx, 0, gy, row);
-                }
+                issue_unit(j);
                 ++issued;
             }
             // copies still in flight land before shared memory is released
@@ -313,51 +334,49 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_umma_kernel(const __grid_cons
         }
     } else if (warp == kWarpMma) {
         // =================== MMA issuer ===================
+        // Order: S_0, S_1, then per unit j: O_j = P_j V_j, S_{j+2} = Q K^T.
+        // S_{j+2} reuses S / P buffer j & 1 after the P.V that reads P_j
+        // (tcgen05.mma of one thread execute in issue order).
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_f16<T>(128, 0);
             constexpr uint32_t idesc_pv = idesc_f16<T>(32, 1);
-            for (int j = 0; j <= nst; ++j) {
-                if (j < nst) {
-                    // S_j = Q K^T into S buffer j & 1 (free: its previous
-                    // unit's P was consumed by a P.V issued earlier)
-                    const int s = j % NSTG;
-                    if (!mb_wait(bar_full + 8 * s, (uint32_t)((j / NSTG) & 1))) {
-                        atomicAdd(&g_umma_timeouts, 1u);
-                        *abort_flag = 1;
-                        break;
-                    }
-                    if (*abort_flag) break;
-                    tc_fence_after();
-                    const uint32_t st = sbase + (uint32_t)s * kStage;
-                    // K-major, 64-byte rows: 8-row groups 512 bytes apart; the
-                    // second K = 16 step starts 32 bytes into the rows
-                    const uint64_t da = sw64_desc(st, 16, 512), db = sw64_desc(st + kTile, 16, 512);
-                    const uint32_t dS = tmem + (uint32_t)(j & 1) * 128;
-                    umma_ss(dS, da, db, idesc_qk, 0);
-                    umma_ss(dS, da + 2, db + 2, idesc_qk, 1);
-                    umma_commit(bar_s + 8 * (j & 1));
+            auto issue_qk = [&](int j) -> bool {
+                const int s = j % NSTG;
+                if (!mb_wait(bar_full + 8 * s, (uint32_t)((j / NSTG) & 1)) || *abort_flag) return false;
+                tc_fence_after();
+                const uint32_t st = sbase + (uint32_t)s * kStage;
+                // K-major, 64-byte rows: 8-row groups 512 bytes apart; the
+                // second K = 16 step starts 32 bytes into the rows
+                const uint64_t da = sw64_desc(st, 16, 512), db = sw64_desc(st + kTile, 16, 512);
+                const uint32_t dS = tmem + (uint32_t)(j & 1) * 128;
+                umma_ss(dS, da, db, idesc_qk, 0);
+                umma_ss(dS, da + 2, db + 2, idesc_qk, 1);
+                umma_commit(bar_s + 8 * (j & 1));
+                return true;
+            };
+            bool ok = issue_qk(0) && (nst < 2 || issue_qk(1));
+            for (int j = 0; ok && j < nst; ++j) {
+                const int b = j & 1, s = j % NSTG;
+                if (!mb_wait(bar_p + 8 * b, (uint32_t)((j >> 1) & 1)) || *abort_flag) {
+                    ok = false;
+                    break;
                 }
-                if (j >= 1) {
-                    // O_{j-1} = P V
-                    const int jp = j - 1, b = jp & 1, s = jp % NSTG;
-                    if (!mb_wait(bar_p + 8 * b, (uint32_t)((jp >> 1) & 1))) {
-                        atomicAdd(&g_umma_timeouts, 1u);
-                        *abort_flag = 1;
-                        break;
-                    }
-                    if (*abort_flag) break;
-                    tc_fence_after();
-                    const uint32_t vt = sbase + (uint32_t)s * kStage + 2 * kTile;
-                    const uint32_t dO = tmem + 256u + (uint32_t)b * 32;
-                    const uint32_t aP = tmem + (uint32_t)b * 128;
-                    // V MN-major: 64-byte rows of 32 channels, 8-key groups
-                    // 512 bytes apart; k-step t takes keys 16t .. 16t + 15
+                tc_fence_after();
+                const uint32_t vt = sbase + (uint32_t)s * kStage + 2 * kTile;
+                const uint32_t dO = tmem + 256u + (uint32_t)(j & 3) * 32;
+                const uint32_t aP = tmem + (uint32_t)b * 128;
+                // V MN-major: 64-byte rows of 32 channels, 8-key groups 512
+                // bytes apart; k-step t takes keys 16t .. 16t + 15
 #pragma unroll
-                    for (int t = 0; t < 8; ++t)
-                        umma_ts(dO, aP + 8u * t, sw64_desc(vt + 1024u * t, 16, 512), idesc_pv, t > 0 ? 1u : 0u);
-                    umma_commit(bar_o + 8 * b);
-                    umma_commit(bar_empty + 8 * s);
-                }
+                for (int t = 0; t < 8; ++t)
+                    umma_ts(dO, aP + 8u * t, sw64_desc(vt + 1024u * t, 16, 512), idesc_pv, t > 0 ? 1u : 0u);
+                umma_commit(bar_o + 8 * (j & 3));
+                umma_commit(bar_empty + 8 * s);
+                if (j + 2 < nst && !issue_qk(j + 2)) ok = false;
+            }
+            if (!ok) {
+                atomicAdd(&g_umma_timeouts, 1u);
+                *abort_flag = 1;
             }
             // every MMA issued has completed before TMEM is released
             umma_commit(bar_drain);
@@ -365,7 +384,10 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_umma_kernel(const __grid_cons
         }
     } else {
         // =================== softmax warpgroups ===================
-        const int w = warp >> 2;                      // warpgroup = TMEM buffer set
+        // Warpgroup w takes units j = w, w + 2, ...: softmax of unit j, then
+        // the epilogue of its previous unit j - 2 (whose P.V has had the
+        // softmax's time to complete); O buffers rotate over 4 (j & 3).
+        const int w = warp >> 2;                      // warpgroup = S / P buffer
         const int q4 = warp & 3;                      // lane quarter of this warp
         const int m = q4 * 32 + lane;                 // tile row = TMEM lane
         const int e = m >> 6;                         // group A (0) or B (1); uniform per warp
@@ -375,88 +397,29 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_umma_kernel(const __grid_cons
         const uint32_t tl = tmem + ((uint32_t)(32 * q4) << 16);
         const uint32_t tS = tl + (uint32_t)w * 128 + (uint32_t)e * 64;
         const uint32_t tP = tl + (uint32_t)w * 128;
-        const uint32_t tO = tl + 256u + (uint32_t)w * 32;
         const float c = p.c_log2;
         float bias[KW * KW];
         int cur_h = -1;
-        for (int j = w, k = 0; j < nst; j += 2, ++k) {
-            const int g = 2 * (u_begin + j) + e;
-            const bool gok = g < p.GU;
-            const int bh = gok ? g / dd : 0;
-            const int h = bh % p.heads;
-            if (h != cur_h) {
-                cur_h = h;
-                // bias of key (ky, kx): table row ky - qy + 6, column kx - qx + 6
-                const float *tb = tab + h * kTabHead + (6 - qyc) * kTabPitch + (6 - qxc);
-#pragma unroll
-                for (int ky = 0; ky < KW; ++ky)
-#pragma unroll
-                    for (int kx = 0; kx < KW; ++kx) bias[ky * KW + kx] = tb[ky * kTabPitch + kx];
-            }
-            bool ok = mb_wait(bar_s + 8 * w, (uint32_t)(k & 1));
-            if (!__all_sync(0xffffffffu, ok) || __any_sync(0xffffffffu, *abort_flag != 0)) {
-                if (lane == 0) {
-                    atomicAdd(&g_umma_timeouts, 1u);
-                    *abort_flag = 1;
-                }
-                break;
-            }
-            tc_fence_after();
-            // scores of keys 8 * ky + kx, ky, kx < 8 (kx = 7 and ky = 7 are pads)
-            float s[56];
-            tmem_ld32(tS, s);
-            tmem_ld16(tS + 32, s + 32);
-            tmem_ld8(tS + 48, s + 48);
-            tmem_ld_wait();
-            float mx = -3.0e38f;
-#pragma unroll
-            for (int ky = 0; ky < KW; ++ky) {
-#pragma unroll
-                for (int kx = 0; kx < KW; ++kx) s[ky * 8 + kx] += bias[ky * KW + kx];
-                mx = max3(mx, max3(s[ky * 8 + 0], s[ky * 8 + 1], s[ky * 8 + 2]),
-                          max3(s[ky * 8 + 3], s[ky * 8 + 4], fmaxf(s[ky * 8 + 5], s[ky * 8 + 6])));
-            }
-            const float nm = -mx * c;
-            float l = 0.f;
-            uint32_t pk[32];
-#pragma unroll
-            for (int i = 0; i < 28; ++i) {
-                const float p0 = ex2(fmaf(s[2 * i], c, nm));
-                const float p1 = ((2 * i + 1) & 7) < KW ? ex2(fmaf(s[2 * i + 1], c, nm)) : 0.f;
-                l += p0 + p1;
-                pk[i] = Pack2<T>::run(p0, p1);
-            }
-#pragma unroll
-            for (int i = 28; i < 32; ++i) pk[i] = 0u;
-            uint32_t zero[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) zero[i] = 0u;
-            // own group's keys: P columns 32e .. 32e + 31; the other group's: zeros
-            tmem_st16(tP + (uint32_t)e * 32, pk);
-            tmem_st16(tP + (uint32_t)e * 32 + 16, pk + 16);
-            tmem_st16(tP + (uint32_t)(e ^ 1) * 32, zero);
-            tmem_st16(tP + (uint32_t)(e ^ 1) * 32 + 16, zero);
-            tmem_st_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mb_arrive(bar_p + 8 * w);
-            // ---- epilogue
-            ok = mb_wait(bar_o + 8 * w, (uint32_t)(k & 1));
+        float l_prev = 1.f;
+        // O of unit jj (ready once its P.V completed) / row sum -> 64 bytes
+        auto epilogue_store = [&](int jj) -> bool {
+            const bool ok = mb_wait(bar_o + 8 * (jj & 3), (uint32_t)((jj >> 2) & 1));
             if (!__all_sync(0xffffffffu, ok)) {
                 if (lane == 0) {
                     atomicAdd(&g_umma_timeouts, 1u);
                     *abort_flag = 1;
                 }
-                break;
+                return false;
             }
             tc_fence_after();
             float o[32];
-            tmem_ld32(tO, o);
+            tmem_ld32(tl + 256u + (uint32_t)(jj & 3) * 32, o);
             tmem_ld_wait();
-            if (gok && qok) {
+            const int g = 2 * (u_begin + jj) + e;
+            if (g < p.GU && qok) {
                 float inv;
-                asm("rcp.approx.ftz.f32 %0, %1;\n" : "=f"(inv) : "f"(l));
-                const int rem = g - bh * dd, gy = rem / p.d, gx = rem - gy * p.d;
+                asm("rcp.approx.ftz.f32 %0, %1;\n" : "=f"(inv) : "f"(l_prev));
+                const int bh = g / dd, rem = g - bh * dd, gy = rem / p.d, gx = rem - gy * p.d;
                 uint4 *dst = reinterpret_cast<uint4 *>(
                     p.out + ((((size_t)bh * p.H + gy + (size_t)p.d * qy) * p.W) + gx + (size_t)p.d * qx) * 64);
 #pragma unroll
@@ -465,6 +428,80 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_umma_kernel(const __grid_cons
                                         Pack2<T>::run(o[8 * i + 2] * inv, o[8 * i + 3] * inv),
                                         Pack2<T>::run(o[8 * i + 4] * inv, o[8 * i + 5] * inv),
                                         Pack2<T>::run(o[8 * i + 6] * inv, o[8 * i + 7] * inv));
+            }
+            return true;
+        };
+        for (int j = w;; j += 2) {
+            if (j < nst) {
+                const int g = 2 * (u_begin + j) + e;
+                const int h = (min(g, p.GU - 1) / dd) % p.heads;
+                if (h != cur_h) {
+                    cur_h = h;
+                    // bias of key (ky, kx): table row ky - qy + 6, column kx - qx + 6
+                    const float *tb = tab + h * kTabHead + (6 - qyc) * kTabPitch + (6 - qxc);
+#pragma unroll
+                    for (int ky = 0; ky < KW; ++ky)
+#pragma unroll
+                        for (int kx = 0; kx < KW; ++kx) bias[ky * KW + kx] = tb[ky * kTabPitch + kx];
+                }
+                const bool ok = mb_wait(bar_s + 8 * w, (uint32_t)((j >> 1) & 1));
+                if (!__all_sync(0xffffffffu, ok) || __any_sync(0xffffffffu, *abort_flag != 0)) {
+                    if (lane == 0) {
+                        atomicAdd(&g_umma_timeouts, 1u);
+                        *abort_flag = 1;
+                    }
+                    break;
+                }
+                tc_fence_after();
+                // scores of keys 8 * ky + kx, ky, kx < 8 (kx = 7 and ky = 7 are pads)
+                float s[56];
+                tmem_ld32(tS, s);
+                tmem_ld16(tS + 32, s + 32);
+                tmem_ld8(tS + 48, s + 48);
+                tmem_ld_wait();
+                float mx = -3.0e38f;
+#pragma unroll
+                for (int ky = 0; ky < KW; ++ky) {
+#pragma unroll
+                    for (int kx = 0; kx < KW; ++kx) s[ky * 8 + kx] += bias[ky * KW + kx];
+                    mx = max3(mx, max3(s[ky * 8 + 0], s[ky * 8 + 1], s[ky * 8 + 2]),
+                              max3(s[ky * 8 + 3], s[ky * 8 + 4], fmaxf(s[ky * 8 + 5], s[ky * 8 + 6])));
+                }
+                const float nm = -mx * c;
+                float l0 = 0.f, l1 = 0.f;
+                uint32_t pk[32];
+#pragma unroll
+                for (int i = 0; i < 28; ++i) {
+                    const float p0 = ex2(fmaf(s[2 * i], c, nm));
+                    const float p1 = ((2 * i + 1) & 7) < KW ? ex2(fmaf(s[2 * i + 1], c, nm)) : 0.f;
+                    if (i & 1) l1 += p0 + p1; else l0 += p0 + p1;
+                    pk[i] = Pack2<T>::run(p0, p1);
+                }
+#pragma unroll
+                for (int i = 28; i < 32; ++i) pk[i] = 0u;
+                uint32_t zero[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) zero[i] = 0u;
+                // own group's keys: P columns 32e .. 32e + 31; the other group's: zeros
+                tmem_st16(tP + (uint32_t)e * 32, pk);
+                tmem_st16(tP + (uint32_t)e * 32 + 16, pk + 16);
+                tmem_st16(tP + (uint32_t)(e ^ 1) * 32, zero);
+                tmem_st16(tP + (uint32_t)(e ^ 1) * 32 + 16, zero);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mb_arrive(bar_p + 8 * w);
+                if (j < 2) {
+                    l_prev = l0 + l1;
+                    continue;
+                }
+                // ---- epilogue of unit j - 2 below, then keep this unit's sum
+                const float l_this = l0 + l1;
+                if (!epilogue_store(j - 2)) break;
+                l_prev = l_this;
+            } else {
+                if (j >= 2 && j - 2 < nst) epilogue_store(j - 2);
+                break;
             }
         }
     }
@@ -528,9 +565,9 @@ cudaError_t launch_umma_t(const Problem &pr, const void *q, const void *k, const
     const int64_t bh = pr.bh();
     const int64_t gu = bh * pr.d * pr.d;
     if (gu <= 0 || gu >= INT32_MAX || bh * KW >= INT32_MAX) return cudaSuccess;
-    if (!encode_group_map(&up.tq, q, pr.dtype, bh, pr.H, pr.W, pr.d, 8, 8) ||
-        !encode_group_map(&up.tk, k, pr.dtype, bh, pr.H, pr.W, pr.d, 8, 8) ||
-        !encode_group_map(&up.tv, v, pr.dtype, bh, pr.H, pr.W, pr.d, 8, 8))
+    if (!encode_group_map(&up.tq, q, pr.dtype, bh, pr.H, pr.W, pr.d, 8, 7, 1) ||
+        !encode_group_map(&up.tk, k, pr.dtype, bh, pr.H, pr.W, pr.d, 8, 7, 1) ||
+        !encode_group_map(&up.tv, v, pr.dtype, bh, pr.H, pr.W, pr.d, 8, 7, 1))
         return cudaSuccess;
     up.out = static_cast<unsigned char *>(out);
     up.rpb = rpb;
@@ -543,7 +580,7 @@ cudaError_t launch_umma_t(const Problem &pr, const void *q, const void *k, const
     up.off_bar = align_up(up.off_tab + (uint32_t)(pr.heads * kTabHead * 4), 16);
     // + 1024 bytes for aligning the base; at least 116 KB so that two blocks
     // never share an SM (each takes all 512 TMEM columns)
-    const uint32_t smem = std::max<uint32_t>(up.off_bar + 16 * NSTG + 64 + 1024, 116u * 1024u);
+    const uint32_t smem = std::max<uint32_t>(up.off_bar + 16 * NSTG + 80 + 1024, 116u * 1024u);
     if ((int)smem > cap) return cudaSuccess;
     const int grid = std::min(up.NU, sms);
     fwd_umma_kernel<T><<<grid, kThreads, smem, st>>>(up);
