@@ -74,7 +74,7 @@ struct StreamParams {
     unsigned char *out;
     const void *rpb;
     int H, W, heads, d;
-    int nsteps;
+    int nsteps;      // DENSE: steps; SLIDE: query-row pairs (split over the CTAs)
     // SLIDE schedule
     int MX, SP, NP, SPI, NR;
     // DENSE schedule
@@ -223,22 +223,32 @@ __device__ __forceinline__ int win_start(int y, int L) { return clampi(y - KW / 
 __device__ __forceinline__ int pair_halo(int pair, int H) { return min(win_start(2 * pair, H), H - 8); }
 
 // SLIDE walk: the CTA's steps in order, with the K / V ring bookkeeping.
-// Rows of one image are loaded in increasing order, each once, into
-// consecutive ring rows; the next image continues after the last ring row of
-// the previous one.  Producer and consumers run the same walk.  Only the
-// image, the step within it and the ring row of the step's first key row are
-// kept; the rest is recomputed from them.
+// A CTA owns a contiguous range of query-row pairs in (image, pair) order
+// (global pair index bh * NP + pair), which may start and end inside an
+// image; a step is up to SP consecutive pairs of one image.  Rows of one
+// image are loaded in increasing order, each once, into consecutive ring
+// rows; the next image continues after the last ring row of the previous
+// one.  Producer and consumers run the same walk.  Only the image, the step's
+// pairs and the ring row of the step's first key row are kept; the rest is
+// recomputed from them.
 struct SlideWalk {
-    int bh, k;        // image and step index within it
+    int bh;           // image
+    int pa, pe;       // the step's first pair and one past its last
+    int ge;           // end of the CTA's range (global pair index)
     int h;            // head of image bh
     int ring_lo;      // ring row of lo()
-    __device__ __forceinline__ int p0(const StreamParams &p) const { return k * p.SP; }
-    __device__ __forceinline__ int plast(const StreamParams &p) const { return min(k * p.SP + p.SP, p.NP) - 1; }
-    __device__ __forceinline__ int lo(const StreamParams &p) const { return pair_halo(p0(p), p.H); }
-    __device__ __forceinline__ int hi(const StreamParams &p) const { return pair_halo(plast(p), p.H) + 7; }
-    __device__ __forceinline__ void init(const StreamParams &p, int s) {
-        bh = s / p.SPI;
-        k = s - bh * p.SPI;
+    __device__ __forceinline__ int p0(const StreamParams &) const { return pa; }
+    __device__ __forceinline__ int plast(const StreamParams &) const { return pe - 1; }
+    __device__ __forceinline__ int lo(const StreamParams &p) const { return pair_halo(pa, p.H); }
+    __device__ __forceinline__ int hi(const StreamParams &p) const { return pair_halo(pe - 1, p.H) + 7; }
+    __device__ __forceinline__ int step_end(const StreamParams &p) const {
+        return min(pa + p.SP, min(p.NP, ge - bh * p.NP));
+    }
+    __device__ __forceinline__ void init(const StreamParams &p, int gb, int gend) {
+        ge = gend;
+        bh = gb / p.NP;
+        pa = gb - bh * p.NP;
+        pe = step_end(p);
         h = bh % p.heads;
         ring_lo = 0;
     }
@@ -250,17 +260,31 @@ struct SlideWalk {
     __device__ __forceinline__ int next(const StreamParams &p) {
         const int old_lo = lo(p), old_hi = hi(p);
         const int hi_ring = wrap(ring_lo + old_hi - old_lo, p.NR);
-        if (++k == p.SPI) {
-            k = 0;
+        if (pe == p.NP) {
             ++bh;
             if (++h == p.heads) h = 0;
+            pa = 0;
+            pe = step_end(p);
             ring_lo = wrap(hi_ring + 1, p.NR);
             return lo(p);
         }
+        pa = pe;
+        pe = step_end(p);
         ring_lo = wrap(ring_lo + (lo(p) - old_lo), p.NR);
         return old_hi + 1;
     }
 };
+
+// Number of SLIDE steps in the pair range [gb, ge): per image, ceil(pairs / SP).
+__device__ __forceinline__ int slide_steps(const StreamParams &p, int gb, int ge) {
+    int n = 0;
+    while (gb < ge) {
+        const int bh = gb / p.NP, pa = gb - bh * p.NP, pe = min(p.NP, ge - bh * p.NP);
+        n += (pe - pa + p.SP - 1) / p.SP;
+        gb = bh * p.NP + pe;
+    }
+    return n;
+}
 
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(dst),
@@ -440,10 +464,12 @@ template <typename T, bool DENSE, int NWC>
 __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __grid_constant__ StreamParams p) {
     extern __shared__ __align__(1024) unsigned char smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // this CTA's range: DENSE steps, or SLIDE query-row pairs (finer, so that
+    // the CTAs' loads differ by at most one pair)
     const int s_begin = (int)((int64_t)p.nsteps * blockIdx.x / gridDim.x);
     const int s_end = (int)((int64_t)p.nsteps * (blockIdx.x + 1) / gridDim.x);
     if (s_begin >= s_end) return;
-    const int nst = s_end - s_begin;
+    const int nst = DENSE ? s_end - s_begin : slide_steps(p, s_begin, s_end);
     constexpr int GPS = NWC / 4;   // DENSE groups per step
 
     const uint32_t sbase = smem_u32(smem);
@@ -493,7 +519,7 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
             if (lane == 0) {
                 const uint32_t rowbytes = (uint32_t)p.W * kPixB;
                 SlideWalk w;
-                w.init(p, s_begin);
+                w.init(p, s_begin, s_end);
                 int issued = 0;
                 for (int i = 0; i < nst; ++i) {
                     const int stage = i % NS;
@@ -602,7 +628,7 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
             const uint32_t dv = (p.off_v - p.off_k) + 16u * (uint32_t)((lane >> 4) - lch);
             const int qsel = (lane >> 3) & 1;
             SlideWalk w;
-            w.init(p, s_begin);
+            w.init(p, s_begin, s_end);
             for (int i = 0; i < nst; ++i) {
                 const int stage = i % NS;
                 if (i) w.next(p);
@@ -825,9 +851,9 @@ cudaError_t launch_slide(StreamParams &sp, const Problem &pr, cudaStream_t st, b
     for (int SP = std::max(1, NWC / MX); SP >= 1; --SP) {
         const uint32_t smem = plan_slide(sp, pr, SP);
         if ((int)smem > cap) continue;
-        const int64_t nsteps = pr.bh() * sp.SPI;
-        if (nsteps >= INT32_MAX || nsteps <= 0) return cudaSuccess;
-        sp.nsteps = (int)nsteps;
+        const int64_t npairs = pr.bh() * sp.NP;
+        if (npairs >= INT32_MAX || npairs <= 0) return cudaSuccess;
+        sp.nsteps = (int)npairs;
         return launch_stream_t<T, false, NWC>(sp, smem, sms, st, launched);
     }
     return cudaSuccess;
