@@ -813,8 +813,7 @@ cudaError_t stream_device(int *sms, int *smem_cap, const void *kern) {
 uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
 template <typename T, bool DENSE, int NWC>
-cudaError_t launch_stream_t(const StreamParams &sp, uint32_t smem, int sms, cudaStream_t st, bool *launched) {
-    const int grid = std::min(sp.nsteps, sms);
+cudaError_t launch_stream_t(const StreamParams &sp, uint32_t smem, int grid, cudaStream_t st, bool *launched) {
     fwd_stream_kernel<T, DENSE, NWC><<<grid, (NWC + 1) * 32, smem, st>>>(sp);
     *launched = true;
     return cudaGetLastError();
@@ -854,7 +853,19 @@ cudaError_t launch_slide(StreamParams &sp, const Problem &pr, cudaStream_t st, b
         const int64_t npairs = pr.bh() * sp.NP;
         if (npairs >= INT32_MAX || npairs <= 0) return cudaSuccess;
         sp.nsteps = (int)npairs;
-        return launch_stream_t<T, false, NWC>(sp, smem, sms, st, launched);
+        // CTAs: one per SM with an even split of the pairs, or, when the
+        // images fit on the SMs, a whole number c of CTAs per image, so that
+        // every CTA's range lies inside one image (no second halo and no
+        // second clamped image top, which cost about a step).  The aligned
+        // split is taken while it gives a CTA at most one pair more.
+        const int64_t images = pr.bh();
+        int grid = (int)std::min<int64_t>(npairs, sms);
+        if (images <= sms) {
+            const int64_t c = std::min<int64_t>(sms / images, sp.NP);
+            const int64_t aligned = (sp.NP + c - 1) / c, even = (npairs + sms - 1) / sms;
+            if (aligned <= even + 1) grid = (int)(images * c);
+        }
+        return launch_stream_t<T, false, NWC>(sp, smem, grid, st, launched);
     }
     return cudaSuccess;
 }
@@ -893,7 +904,7 @@ cudaError_t launch_stream_impl(const Problem &pr, const void *q, const void *k, 
         sp.off_bar = align_up(sp.off_tab + 128 + (uint32_t)(pr.heads * kTabHead * 4), 16);
         const uint32_t smem = sp.off_bar + 16 * NS + 16;
         if ((int)smem > cap) return cudaSuccess;
-        return launch_stream_t<T, true, NWC>(sp, smem, sms, st, launched);
+        return launch_stream_t<T, true, NWC>(sp, smem, std::min(sp.nsteps, sms), st, launched);
     }
     // SLIDE: 14 consumer warps (SP query-row pairs of MX column tiles each)
     // and a producer warp; 15 warps keep 128 registers per thread
