@@ -632,20 +632,15 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
             for (int i = 0; i < nst; ++i) {
                 const int stage = i % NS;
                 if (i) w.next(p);
-                if (!sb_wait(bar_full + 8 * stage, (uint32_t)((i / NS) & 1))) {
-                    if (lane == 0) {
-                        atomicAdd(&g_stream_timeouts, 1u);
-                        *abort_flag = 1;
-                    }
-                    break;
-                }
-                if (*abort_flag) break;
                 const int pair = w.p0(p) + pw;
-                if (active && pair <= w.plast(p)) {
-                    const int qy0 = 2 * pair, qy1 = min(qy0 + 1, H - 1);
-                    const int hy = pair_halo(pair, H);
+                const bool work = active && pair <= w.plast(p);
+                const int qy0 = 2 * pair, qy1 = min(qy0 + 1, H - 1);
+                const int hy = pair_halo(pair, H);
+                if (work) {
                     const int sy0 = win_start(qy0, H), sy1 = win_start(qy1, H);
-                    // bias: rewritten when the head or the row geometry changes
+                    // bias: rewritten when the head or the row geometry
+                    // changes, before the wait for the step's rows (it needs
+                    // none of them), so that it overlaps the copies
                     const int key = ((w.h * 8 + (qy0 - hy)) * 2 + (qy1 - qy0)) * 4 + (sy0 - hy) * 2 + (sy1 - hy);
                     if (key != bias_key) {
                         bias_key = key;
@@ -673,6 +668,16 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
                         }
                         tmem_store_bias<NJ>(tb, bias);
                     }
+                }
+                if (!sb_wait(bar_full + 8 * stage, (uint32_t)((i / NS) & 1))) {
+                    if (lane == 0) {
+                        atomicAdd(&g_stream_timeouts, 1u);
+                        *abort_flag = 1;
+                    }
+                    break;
+                }
+                if (*abort_flag) break;
+                if (work) {
                     // Q fragment addresses: lanes 0-7 / 16-23 row qy0, 8-15 /
                     // 24-31 row qy1; lanes 16-31 take the odd 16-byte chunk
                     const int qr = stage * 2 * p.SP + (qsel ? qy1 : qy0) - 2 * w.p0(p);
