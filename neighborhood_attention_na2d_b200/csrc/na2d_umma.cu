@@ -268,10 +268,14 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_umma_kernel(const __grid_cons
             tma_load_5d(st + 2 * kTile + (uint32_t)e * kBlk, &p.tv, fb, gx, 0, gy, row);
         }
     };
-    const int n_first = min(NSTG, nst);   // units whose copies start in the prologue
+    // Units whose copies start in the prologue: two.  With every stage
+    // requested at once by every block, the first unit's bytes and the bias
+    // table's reads queue behind all of them (measured: 18.5 us per launch at
+    // B = 32, DiNAT stage 1, against 16.7 us with two and 17.3 us with none).
+    const int n_first = min(2, nst);
 
     // ---- prologue.  The producer thread initialises the barriers and starts
-    // the first NSTG units' copies at once; meanwhile the other threads zero
+    // the first units' copies; meanwhile the other threads zero
     // the spare slot row 7 of every block, which the 7-row copies never write
     // (V's must be finite: P is 0 there, and 0 * NaN would not be), build the
     // bias table and allocate TMEM.
