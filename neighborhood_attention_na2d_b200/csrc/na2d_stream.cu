@@ -524,7 +524,13 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
                 for (int i = 0; i < nst; ++i) {
                     const int stage = i % NS;
                     const int first = i ? w.next(p) : w.lo(p);
-                    if (i >= NS && !sb_wait(bar_empty + 8 * stage, (uint32_t)(((i / NS) - 1) & 1))) {
+                    // ramp-up: each of the first NS steps is requested once
+                    // the previous step's rows have landed, so that the first
+                    // step's rows do not queue behind the next steps'; later,
+                    // a step waits for its stage to be released
+                    const bool ok = i >= NS ? sb_wait(bar_empty + 8 * stage, (uint32_t)(((i / NS) - 1) & 1))
+                                            : (i == 0 || sb_wait(bar_full + 8 * (i - 1), 0u));
+                    if (!ok) {
                         atomicAdd(&g_stream_timeouts, 1u);
                         *abort_flag = 1;
                         break;
