@@ -117,6 +117,15 @@ __device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(bar) : "memory");
 }
 
+// ---- programmatic dependent launch ------------------------------------------
+// The kernels are launched with programmatic stream serialisation: a grid
+// may be scheduled while the previous kernel on the stream finishes, runs its
+// prologue (barriers, tensor-memory allocation), and reads no global memory
+// before grid_dep_wait() returns, i.e. before that kernel has completed and
+// its writes are visible.  grid_dep_launch() lets the next grid be scheduled.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
 // ---- tensor memory (TMEM) helpers -------------------------------------------
 constexpr int kTmemCols = 256;   // 4 column slots of 64, one per warp of a lane quarter
 
@@ -468,6 +477,7 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
     // the CTAs' loads differ by at most one pair)
     const int s_begin = (int)((int64_t)p.nsteps * blockIdx.x / gridDim.x);
     const int s_end = (int)((int64_t)p.nsteps * (blockIdx.x + 1) / gridDim.x);
+    grid_dep_launch();
     if (s_begin >= s_end) return;
     const int nst = DENSE ? s_end - s_begin : slide_steps(p, s_begin, s_end);
     constexpr int GPS = NWC / 4;   // DENSE groups per step
@@ -488,6 +498,7 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
             const int n16 = (int)(p.off_tab / 16);
             for (int i = threadIdx.x; i < n16; i += blockDim.x) z[i] = make_uint4(0, 0, 0, 0);
         }
+        grid_dep_wait();   // first global read: the bias table
         const T *rpb = reinterpret_cast<const T *>(p.rpb);
         for (int i = threadIdx.x; i < p.heads * kTabHead; i += blockDim.x) {
             const int h = i / kTabHead, a = (i / kTabPitch) % 13, b = i % kTabPitch;
@@ -825,9 +836,19 @@ uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
 template <typename T, bool DENSE, int NWC>
 cudaError_t launch_stream_t(const StreamParams &sp, uint32_t smem, int grid, cudaStream_t st, bool *launched) {
-    fwd_stream_kernel<T, DENSE, NWC><<<grid, (NWC + 1) * 32, smem, st>>>(sp);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3((NWC + 1) * 32);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, fwd_stream_kernel<T, DENSE, NWC>, sp);
     *launched = true;
-    return cudaGetLastError();
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 // SLIDE plan for SP query-row pairs per step; returns the shared-memory bytes.

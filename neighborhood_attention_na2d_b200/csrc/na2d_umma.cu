@@ -109,6 +109,15 @@ __device__ __forceinline__ void mb_expect_tx(uint32_t bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
 }
 
+// ---- programmatic dependent launch ------------------------------------------
+// The kernels are launched with programmatic stream serialisation: a grid
+// may be scheduled while the previous kernel on the stream finishes, runs its
+// prologue (barriers, tensor-memory allocation), and reads no global memory
+// before grid_dep_wait() returns, i.e. before that kernel has completed and
+// its writes are visible.  grid_dep_launch() lets the next grid be scheduled.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
 // ---- TMA ---------------------------------------------------------------------
 __device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap *map, uint32_t bar, int c1, int c2,
                                             int c3, int c4) {
@@ -236,6 +245,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_umma_kernel(const __grid_cons
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int u_begin = (int)((int64_t)p.NU * blockIdx.x / gridDim.x);
     const int u_end = (int)((int64_t)p.NU * (blockIdx.x + 1) / gridDim.x);
+    grid_dep_launch();
     if (u_begin >= u_end) return;
     const int nst = u_end - u_begin;
     const int dd = p.d * p.d;
@@ -293,6 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_umma_kernel(const __grid_cons
             mb_init(bar_drain, 1);
             *abort_flag = 0;
             asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+            grid_dep_wait();   // before the first copy
             for (int j = 0; j < n_first; ++j) issue_unit(j);
         }
         // 6 * NSTG blocks x 512 bytes (slots 56 .. 63)
@@ -300,6 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_umma_kernel(const __grid_cons
             uint4 *z = reinterpret_cast<uint4 *>(smem + (i >> 5) * kBlk + kRowsBytes) + (i & 31);
             *z = make_uint4(0, 0, 0, 0);
         }
+        grid_dep_wait();   // before the bias table's reads
         const T *rpb = reinterpret_cast<const T *>(p.rpb);
         for (int i = threadIdx.x; i < p.heads * kTabHead; i += kThreads) {
             const int h = i / kTabHead, a = (i / kTabPitch) % 13, b = i % kTabPitch;
@@ -586,10 +598,19 @@ cudaError_t launch_umma_t(const Problem &pr, const void *q, const void *k, const
     // never share an SM (each takes all 512 TMEM columns)
     const uint32_t smem = std::max<uint32_t>(up.off_bar + 16 * NSTG + 80 + 1024, 116u * 1024u);
     if ((int)smem > cap) return cudaSuccess;
-    const int grid = std::min(up.NU, sms);
-    fwd_umma_kernel<T><<<grid, kThreads, smem, st>>>(up);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)std::min(up.NU, sms));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t el = cudaLaunchKernelEx(&cfg, fwd_umma_kernel<T>, up);
     *launched = true;
-    return cudaGetLastError();
+    return el != cudaSuccess ? el : cudaGetLastError();
 }
 
 }  // namespace
