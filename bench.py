@@ -53,10 +53,18 @@ def log(*a):
     print(*a, file=sys.stderr, flush=True)
 
 
+def code_only(text: str) -> str:
+    """C++ source without comments and blank lines, so that an edit of the
+    comments alone does not count as a kernel change."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = (re.sub(r"//.*$", "", ln).rstrip() for ln in text.splitlines())
+    return "\n".join(ln for ln in lines if ln)
+
+
 def kernel_sha() -> str:
     h = hashlib.sha256()
     for p in KERNEL_SOURCES:
-        h.update((ROOT / p).read_bytes())
+        h.update(code_only((ROOT / p).read_text()).encode())
     return h.hexdigest()[:16]
 
 

@@ -7,23 +7,29 @@
 // only changes how the work is scheduled and staged.
 //
 // Two schedules:
-//  * SLIDE (d = 1, 14 <= W <= 64, H >= 8): the map is walked in "steps" of SP
-//    query-row pairs.  A query-row pair needs 8 consecutive key rows (the union
-//    of its two clamped windows), and consecutive pairs share 6 of them, so
-//    every K / V row is brought into a shared-memory ring once per CTA and
-//    reused by up to four pairs.  One CTA per SM owns a contiguous range of
-//    steps (whole image rows in (batch*head, row) order).
-//  * DENSE (H = W = 7d, every dilation group exactly 7 x 7; DiNAT's layers
-//    whose dilated window spans the map): a group is a dense 49 x 49
-//    attention.  A step is NWC / 4 consecutive groups, staged whole.
+//  * SLIDE (d = 1, 14 <= W <= 64, H >= 8): the map is walked in "steps" of up
+//    to SP query-row pairs of one image.  A query-row pair needs 8 consecutive
+//    key rows (the union of its two clamped windows), and consecutive pairs
+//    share 6 of them, so every K / V row is brought into a shared-memory ring
+//    once per CTA and reused by up to four pairs.  A CTA owns a contiguous
+//    range of pairs in (batch*head, pair) order: c CTAs per image when the
+//    images fit on the SMs (no range then crosses an image), else an even
+//    split over one CTA per SM.
+//  * DENSE (H = W = 7d, every dilation group exactly 7 x 7): a group is a
+//    dense 49 x 49 attention.  A step is NWC / 4 consecutive groups, staged
+//    whole.  These maps normally run on the tcgen05 kernel (na2d_umma.cu);
+//    this schedule is its fallback.
 //
-// Loading: every warp issues its share of the 16-byte cp.async copies of the
-// step NS - 1 ahead (many warps keep enough requests in flight to stream at
-// HBM speed; a single issuing thread does not), and every thread arrives on
-// the stage's "full" mbarrier once its copies have landed
-// (cp.async.mbarrier.arrive.noinc).  A warp refills a stage only after all
-// warps released it on its "empty" mbarrier, which keeps the warps within
-// one step of each other.  All waits are bounded.
+// Loading, by a producer warp NS - 1 steps ahead through full / empty
+// mbarriers: SLIDE issues one bulk copy (cp.async.bulk) per new image row of
+// K, V and Q from one thread, with the byte count on the stage's full
+// barrier; DENSE issues 16-byte cp.async with fixed per-lane offsets, each
+// lane arriving once its copies have landed.  In the ramp-up each of the
+// first NS steps is requested once the previous step's rows have landed, so
+// that the first step's rows do not queue behind the next ones.  All waits
+// are bounded.  The kernel is launched with programmatic stream
+// serialisation and reads no global memory before the previous kernel on
+// the stream has completed.
 //
 // Per warp, one 16-query tile per step: 2 query rows x 8 query columns.  Its
 // keys form n-tiles of 4 key rows x 2 key columns (14 n-tiles = 8 x 14 keys for
