@@ -116,6 +116,12 @@ def _stream_cases():
         for dtype in ("f16", "bf16"):
             cases.append((Shape(B, heads, 7 * d, 7 * d, 32, 7, d, dtype, 7000 + n), n % 3 != 2))
             n += 1
+    # 64 heads (the largest bias table of the dense kernel), more units than
+    # SMs with an odd group count, and more sliding-row images than SMs (the
+    # pairs are then split evenly across images)
+    cases.append((Shape(1, 64, 7, 7, 32, 7, 1, "bf16", 7100), True))
+    cases.append((Shape(3, 101, 7, 7, 32, 7, 1, "f16", 7101), True))
+    cases.append((Shape(75, 2, 14, 14, 32, 7, 1, "f16", 7102), True))
     return cases
 
 
