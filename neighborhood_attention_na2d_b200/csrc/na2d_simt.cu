@@ -56,17 +56,24 @@ __device__ __forceinline__ QueryWin query_window(int i, int j, int H, int W, int
 }
 
 // ---------------------------------------------------------------------------
-// Fused forward, one thread per (b, head, i, j) query.  Two passes over the
-// k*k window: the row maximum first, then exp, sum and the weighted values.
+// Fused forward, one warp per (b, head, i, j) query.  Scores: lane t takes
+// neighbours n = t, t + 32, ... (n = ty * k + tx, up to six per lane for
+// k <= 13), each a full D = 32 dot product.  The row max and sum are warp
+// reductions.  Weighted values: lane c accumulates channel c over the
+// neighbours in order, each probability taken from its lane by a shuffle, so
+// the value rows are read coalesced.
 // ---------------------------------------------------------------------------
+constexpr int kMaxPerLane = (13 * 13 + 31) / 32;
+
 template <typename T>
 __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k,
                                                             const T *__restrict__ v, const T *__restrict__ rpb,
                                                             T *__restrict__ out, int heads, int H, int W, int K,
                                                             int d, int64_t nq, float scale) {
-    const int nb = 2 * K - 1;
-    for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < nq;
-         idx += (int64_t)gridDim.x * blockDim.x) {
+    const int nb = 2 * K - 1, KK = K * K;
+    const int lane = threadIdx.x & 31;
+    const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t idx = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5; idx < nq; idx += nwarps) {
         const int j = (int)(idx % W);
         const int64_t t = idx / W;
         const int i = (int)(t % H);
@@ -74,44 +81,49 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(const T *__restrict_
         const int h = (int)(bh % heads);
         const QueryWin w = query_window(i, j, H, W, K, d);
         const size_t base = (size_t)bh * H * W;
+        const T *bias = rpb ? rpb + (size_t)h * nb * nb : nullptr;
         float qf[kHeadDim];
         load_row<T>(q + (size_t)idx * kHeadDim, qf);
-        const T *bias = rpb ? rpb + (size_t)h * nb * nb : nullptr;
 
+        float sc[kMaxPerLane];
         float m = -FLT_MAX;
-        for (int ty = 0; ty < K; ++ty) {
-            const int ky = w.gy + d * (w.sy + ty);
-            const int by = w.sy + ty - w.iy + K - 1;
-            for (int tx = 0; tx < K; ++tx) {
-                const int kx = w.gx + d * (w.sx + tx);
-                float s = dot_row<T>(qf, k + (base + (size_t)ky * W + kx) * kHeadDim) * scale;
-                if (bias) s += Elem<T>::to_f(bias[by * nb + (w.sx + tx - w.ix + K - 1)]);
-                m = fmaxf(m, s);
+#pragma unroll
+        for (int r = 0; r < kMaxPerLane; ++r) {
+            const int n = lane + 32 * r;
+            sc[r] = -FLT_MAX;
+            if (n < KK) {
+                const int ty = n / K, tx = n - ty * K;
+                const int ky = w.gy + d * (w.sy + ty), kx = w.gx + d * (w.sx + tx);
+                float sv = dot_row<T>(qf, k + (base + (size_t)ky * W + kx) * kHeadDim) * scale;
+                if (bias) sv += Elem<T>::to_f(bias[(w.sy + ty - w.iy + K - 1) * nb + (w.sx + tx - w.ix + K - 1)]);
+                sc[r] = sv;
+                m = fmaxf(m, sv);
             }
         }
-        float l = 0.f, acc[kHeadDim];
 #pragma unroll
-        for (int c = 0; c < kHeadDim; ++c) acc[c] = 0.f;
-        for (int ty = 0; ty < K; ++ty) {
-            const int ky = w.gy + d * (w.sy + ty);
-            const int by = w.sy + ty - w.iy + K - 1;
-            for (int tx = 0; tx < K; ++tx) {
-                const int kx = w.gx + d * (w.sx + tx);
-                const size_t key = (base + (size_t)ky * W + kx) * kHeadDim;
-                float s = dot_row<T>(qf, k + key) * scale;
-                if (bias) s += Elem<T>::to_f(bias[by * nb + (w.sx + tx - w.ix + K - 1)]);
-                const float p = expf(s - m);
-                l += p;
-                float vf[kHeadDim];
-                load_row<T>(v + key, vf);
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        float l = 0.f;
 #pragma unroll
-                for (int c = 0; c < kHeadDim; ++c) acc[c] = fmaf(p, vf[c], acc[c]);
+        for (int r = 0; r < kMaxPerLane; ++r) {
+            sc[r] = lane + 32 * r < KK ? expf(sc[r] - m) : 0.f;
+            l += sc[r];
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+        float acc = 0.f;
+#pragma unroll
+        for (int r = 0; r < kMaxPerLane; ++r) {
+            if (32 * r >= KK) break;
+            const int cnt = min(32, KK - 32 * r);
+            for (int tl = 0; tl < cnt; ++tl) {
+                const int n = 32 * r + tl;
+                const float pn = __shfl_sync(0xffffffffu, sc[r], tl);
+                const int ty = n / K, tx = n - ty * K;
+                const int ky = w.gy + d * (w.sy + ty), kx = w.gx + d * (w.sx + tx);
+                acc = fmaf(pn, Elem<T>::to_f(v[(base + (size_t)ky * W + kx) * kHeadDim + lane]), acc);
             }
         }
-        const float inv = 1.f / l;
-        T *o = out + (size_t)idx * kHeadDim;
-#pragma unroll
-        for (int c = 0; c < kHeadDim; ++c) o[c] = Elem<T>::from_f(acc[c] * inv);
+        out[(size_t)idx * kHeadDim + lane] = Elem<T>::from_f(acc / l);
     }
 }
 
@@ -203,7 +215,7 @@ template <typename T>
 cudaError_t fwd_simt_impl(const Problem &p, const void *q, const void *k, const void *v, const void *rpb, void *out,
                           cudaStream_t st) {
     const int64_t nq = p.bh() * p.H * p.W;
-    fwd_simt_kernel<T><<<grid_for(nq), kThreads, 0, st>>>(
+    fwd_simt_kernel<T><<<grid_for(nq * 32), kThreads, 0, st>>>(
         static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v),
         static_cast<const T *>(rpb), static_cast<T *>(out), p.heads, p.H, p.W, p.k, p.d, nq,
         1.0f / sqrtf((float)p.D));
