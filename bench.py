@@ -43,10 +43,13 @@ UNIT = "queries*heads/s"
 FALLBACK_HBM_GBS = 6650.0
 PEAKS_FILE = ROOT / "MEASURED_PEAKS.json"
 PROFILES = ROOT / "profiles"
-KERNEL_SOURCES = ["neighborhood_attention_na2d_b200/csrc/na2d_tc.cu",
-                  "neighborhood_attention_na2d_b200/csrc/na2d_stream.cu",
-                  "neighborhood_attention_na2d_b200/csrc/na2d_umma.cu",
-                  "neighborhood_attention_na2d_b200/csrc/na2d_device.cuh"]
+CSRC = "neighborhood_attention_na2d_b200/csrc/"
+# The sources each profiled kernel is built from (device code and the host
+# code that plans and launches it).
+KERNEL_SOURCES = {
+    "fwd_stream_kernel": [CSRC + "na2d_stream.cu", CSRC + "na2d_device.cuh", CSRC + "na2d_launch.h"],
+    "fwd_umma_kernel": [CSRC + "na2d_umma.cu", CSRC + "na2d_tc.cu", CSRC + "na2d_device.cuh", CSRC + "na2d_launch.h"],
+}
 
 
 def log(*a):
@@ -61,9 +64,10 @@ def code_only(text: str) -> str:
     return "\n".join(ln for ln in lines if ln)
 
 
-def kernel_sha() -> str:
+def kernel_sha(kernel: str) -> str:
+    """Hash of a kernel's sources without their comments."""
     h = hashlib.sha256()
-    for p in KERNEL_SOURCES:
+    for p in KERNEL_SOURCES[kernel]:
         h.update(code_only((ROOT / p).read_text()).encode())
     return h.hexdigest()[:16]
 
@@ -94,7 +98,7 @@ def recorded_traffic(kernel: str, workload: str) -> int | None:
         return None
     text = f.read_text()
     m = re.search(r"traffic_per_launch_bytes\s*=\s*(\d+)\s*;\s*kernel_sha\s*=\s*([0-9a-f]+)", text)
-    if not m or m.group(2) != kernel_sha():
+    if not m or m.group(2) != kernel_sha(kernel):
         return None
     return int(m.group(1))
 
