@@ -80,16 +80,6 @@ def hbm_peak() -> tuple[float, str]:
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def dominant_kernel(wl) -> str:
-    """The kernel that runs a workload's forward (one launch per shape): maps
-    whose dilation groups are all exactly 7 x 7 take the tcgen05 kernel, other
-    k = 7 maps the streaming kernel."""
-    s = wl.shapes[0]
-    if s.k == 7 and s.H == 7 * s.d and s.W == 7 * s.d:
-        return "fwd_umma_kernel"
-    return "fwd_stream_kernel"
-
-
 def recorded_traffic(kernel: str, workload: str) -> int | None:
     """DRAM bytes per launch from the committed ncu summary of this kernel on
     this workload, only if it was taken on the current kernel source."""
@@ -256,10 +246,147 @@ def cpu_baseline(wl):
             "sample": "; ".join(parts) + "; one pass, fp64"}
 
 
+def graph_plan(K: int, G_max: int = 200) -> tuple[int, int, int]:
+    """How K timed steps are split into CUDA-graph replays: a graph of G steps
+    replayed `full` times, then a graph of `rest` steps (rest < G), so that one
+    timed run is exactly K steps."""
+    if K < 1:
+        raise ValueError("--steps must be at least 1")
+    G = min(K, G_max)
+    full, rest = divmod(K, G)
+    return G, full, rest
+
+
+def make_sets(wl, dev, rank, l2):
+    """Resident input/output sets, rotated so that every step misses L2."""
+    import torch
+    elem = {"f32": 4, "f16": 2, "bf16": 2}
+    set_bytes = sum(4 * s.B * s.heads * s.H * s.W * s.D * elem[s.dtype] for s in wl.shapes)
+    R = max(2, math.ceil(3 * l2 / set_bytes))
+    sets = []
+    for r in range(R):
+        one = []
+        for s in wl.shapes:
+            q, k, v, rpb = make_inputs(s, s.seed + 1000 * r + 100000 * rank)
+            q, k, v, rpb = (t.to(dev) for t in (q, k, v, rpb))
+            one.append((s, q, k, v, rpb, torch.empty_like(q)))
+        sets.append(one)
+    torch.cuda.synchronize()
+    return sets, set_bytes
+
+
+def time_steps(wl, sets, K, warmup, dev, pg=None, min_seconds=0.25, min_runs=5, clocks=None):
+    """Times K steps of the workload (one na2d_forward per shape per step,
+    rotating the input sets).  The K steps are replayed from CUDA graphs (see
+    graph_plan) between CUDA events on the launching stream, bracketed by a
+    barrier and device synchronisation; the run is repeated until about
+    min_seconds have been timed and the median run is returned, as ms per step,
+    with the run count and the spread."""
+    import torch
+    import neighborhood_attention_na2d_b200 as na
+
+    R = len(sets)
+
+    def step(i):
+        for (s, q, k, v, rpb, out) in sets[i % R]:
+            na.na2d_forward(q, k, v, rpb, s.k, s.d, out=out)
+
+    for i in range(max(warmup, 3)):
+        step(i)
+    torch.cuda.synchronize()
+    G, full, rest = graph_plan(K)
+    stream = torch.cuda.Stream(dev)
+    stream.wait_stream(torch.cuda.current_stream(dev))
+    graphs = []
+    with torch.cuda.stream(stream):
+        for n in ([G] + ([rest] if rest else [])):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for i in range(n):
+                    step(i)
+            graphs.append(g)
+        torch.cuda.synchronize()
+        for g in graphs:      # one untimed replay of each graph
+            g.replay()
+        torch.cuda.synchronize()
+        runs = []
+        t_total = 0.0
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ctx = clocks if clocks is not None else _Null()
+        with ctx:
+            while len(runs) < min_runs or t_total < min_seconds * 1e3:
+                if pg:
+                    pg.barrier()
+                torch.cuda.synchronize()
+                start.record(stream)
+                for _ in range(full):
+                    graphs[0].replay()
+                if rest:
+                    graphs[1].replay()
+                end.record(stream)
+                end.synchronize()
+                ms = start.elapsed_time(end)
+                if pg:
+                    t = torch.tensor([ms], device=dev)
+                    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+                    ms = float(t.item())
+                runs.append(ms)
+                t_total += ms
+                if len(runs) >= 10000:
+                    break
+    torch.cuda.synchronize()
+    del graphs
+    med = statistics.median(runs)
+    return {"ms_per_step": med / K, "runs": len(runs), "graph_steps": G, "replays_per_run": full + (1 if rest else 0),
+            "min_ms_per_step": min(runs) / K, "max_ms_per_step": max(runs) / K}
+
+
+class _Null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        return False
+
+
+def tensor_peak() -> tuple[float, str]:
+    """Dense bf16 tensor peak (TFLOP/s) from MEASURED_PEAKS.json (burst figure;
+    fp16 runs at the same rate)."""
+    try:
+        d = json.loads(PEAKS_FILE.read_text())
+        return float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
+def roofline(wl, ms_per_step, kern):
+    """Roofline of one step: the slower of the algorithmic bytes at the HBM
+    peak and the useful FLOPs at the tensor peak; achieved is measured against
+    that bound."""
+    alg_bytes = sum(s.algorithmic_bytes() for s in wl.shapes)
+    flops = sum(s.useful_flops() for s in wl.shapes)
+    hbm, hbm_kind = hbm_peak()
+    tc, tc_kind = tensor_peak()
+    t_hbm = alg_bytes / (hbm * 1e9)
+    t_tc = flops / (tc * 1e12)
+    sec = ms_per_step / 1e3
+    if t_hbm >= t_tc:
+        achieved = alg_bytes / sec / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                "peak_source": f"{hbm_kind} hbm_gbs (copy)"}
+    else:
+        achieved = flops / sec / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": tc, "unit": "TFLOP/s", "frac": achieved / tc,
+                "peak_source": f"{tc_kind} bf16_tflops (burst)"}
+    roof.update({"traffic": recorded_traffic(kern, wl.name) if kern else None,
+                 "algorithmic_bytes_per_step": alg_bytes, "useful_flops_per_step": flops,
+                 "t_hbm_us": t_hbm * 1e6, "t_tensor_us": t_tc * 1e6, "kernel": kern})
+    return roof
+
+
 def run_ours(args, world, rank, local):
     import torch
     import neighborhood_attention_na2d_b200 as na
-    from neighborhood_attention_na2d_b200 import _native
 
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA GPU")
@@ -274,98 +401,82 @@ def run_ours(args, world, rank, local):
     na.lib()
     wl = workload(args)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    elem = {"f32": 4, "f16": 2, "bf16": 2}
 
-    # ---- resident input sets, rotated so that every step misses L2
-    set_bytes = sum(4 * s.B * s.heads * s.H * s.W * s.D * elem[s.dtype] for s in wl.shapes)
-    R = max(2, math.ceil(3 * l2 / set_bytes))
-    sets = []
-    for r in range(R):
-        one = []
-        for s in wl.shapes:
-            q, k, v, rpb = make_inputs(s, s.seed + 1000 * r + 100000 * rank)
-            q, k, v, rpb = (t.to(dev) for t in (q, k, v, rpb))
-            one.append((s, q, k, v, rpb, torch.empty_like(q)))
-        sets.append(one)
-    torch.cuda.synchronize()
+    sets, set_bytes = make_sets(wl, dev, rank, l2)
+    R = len(sets)
     log(f"rank {rank}: {R} input sets x {set_bytes / 1e6:.1f} MB (L2 {l2 / 1e6:.0f} MB)")
-
-    def step(r):
-        for (s, q, k, v, rpb, out) in sets[r % R]:
-            na.na2d_forward(q, k, v, rpb, s.k, s.d, out=out)
-
-    # ---- warm-up (eager), then capture graphs of whole rotations
-    for i in range(max(args.warmup, 3)):
-        step(i)
-    torch.cuda.synchronize()
-    per_graph = R * max(1, 64 // R)
-    graph = torch.cuda.CUDAGraph()
-    cap_stream = torch.cuda.Stream(dev)
-    cap_stream.wait_stream(torch.cuda.current_stream(dev))
-    with torch.cuda.stream(cap_stream):
-        with torch.cuda.graph(graph, stream=cap_stream):
-            for i in range(per_graph):
-                step(i)
-    torch.cuda.synchronize()
-    for _ in range(2):
-        graph.replay()
-    torch.cuda.synchronize()
-
     K = args.steps
-    full, rest = divmod(K, per_graph)
-    stream = torch.cuda.current_stream(dev)
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if pg:
-        pg.barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clocks:
-        start.record(stream)
-        for _ in range(full):
-            graph.replay()
-        for i in range(rest):
-            step(i)
-        end.record(stream)
-        end.synchronize()
-    torch.cuda.synchronize()
-    ms = start.elapsed_time(end)
-    if pg:
-        t = torch.tensor([ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms = float(t.item())
-        pg.barrier()
-    ms_per_step = ms / K
+    clocks = ClockSampler(local)
+    t = time_steps(wl, sets, K, args.warmup, dev, pg, clocks=clocks)
+    ms_per_step = t["ms_per_step"]
     units_rank = sum(s.B * s.heads * s.H * s.W for s in wl.shapes)
     value = world * units_rank / (ms_per_step / 1e3)
+    kern = kernels_of(wl)
+    roof = roofline(wl, ms_per_step, kern[0] if len(set(kern)) == 1 else None)
+    del sets
 
-    # ---- roofline of the dominant kernel (the fused forward; one launch per shape per step)
-    alg_bytes = sum(s.algorithmic_bytes() for s in wl.shapes)
-    achieved = alg_bytes / (ms_per_step / 1e3) / 1e9
-    peak, peak_kind = hbm_peak()
-    kern = dominant_kernel(wl)
-    roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-            "traffic": recorded_traffic(kern, wl.name), "peak_source": f"{peak_kind} hbm_gbs (copy)",
-            "algorithmic_bytes_per_step": alg_bytes, "kernel": kern}
+    # ---- the other workloads of the same problem, each timed the same way (1 GPU)
+    per_wl = {}
+    if world == 1 and not args.no_per_workload:
+        for name in PER_WORKLOAD:
+            if name == wl.name:
+                continue
+            w2 = WORKLOADS[name]
+            s2, _ = make_sets(w2, dev, rank, l2)
+            t2 = time_steps(w2, s2, K, args.warmup, dev, None)
+            k2 = kernels_of(w2)
+            r2 = roofline(w2, t2["ms_per_step"], k2[0] if len(set(k2)) == 1 else None)
+            per_wl[name] = {"ms_per_step": t2["ms_per_step"],
+                            "value": sum(s.B * s.heads * s.H * s.W for s in w2.shapes) / (t2["ms_per_step"] / 1e3),
+                            "frac": r2["frac"], "bound": r2["bound"], "achieved": r2["achieved"],
+                            "traffic": r2["traffic"], "kernels": k2, "shapes": [s.describe() for s in w2.shapes],
+                            "runs": t2["runs"]}
+            del s2
+        torch.cuda.empty_cache()
 
     # ---- end to end through the public API: pinned host -> device, forward, device -> host
     e2e = run_e2e(args, wl, dev, rank, world, pg)
 
     cfg = config_dict(wl, world)
     cfg.update({"l2": f"rotating {R} input sets ({R * set_bytes / 1e6:.0f} MB) > 3x L2 ({l2 / 1e6:.0f} MB)",
-                "timing": f"CUDA graphs of {per_graph} steps, CUDA events on the launching stream"})
+                "timing": (f"each timed run is exactly {K} steps: a CUDA graph of {t['graph_steps']} steps "
+                           f"replayed {t['replays_per_run']} time(s) (a second graph holds the remainder); "
+                           f"CUDA events on the launching stream; median of {t['runs']} runs"),
+                "ms_per_step_min_max": [t["min_ms_per_step"], t["max_ms_per_step"]]})
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": wl.shapes[0].dtype, "data": "synthetic (seeded N(0,1) q/k/v, N(0,0.02) rpb)", "config": cfg,
         "roofline": roof, "e2e": e2e, "gpu_launches": K * len(wl.shapes), "clocks": clocks.summary(),
     }
+    if per_wl:
+        line["per_workload"] = per_wl
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
-    del graph
     if pg:
         pg.barrier()
         pg.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+# workloads timed beside the headline in a 1-GPU run (the second stage-1
+# target first)
+PER_WORKLOAD = ("dinat_s1_bf16", "dinat_sweep_bf16", "seg_bf16")
+
+
+def kernels_of(wl) -> list[str]:
+    """The kernel the library launched for each shape of the workload (asked
+    from the library after a call, not predicted)."""
+    import torch
+    import neighborhood_attention_na2d_b200 as na
+    names = []
+    for s in wl.shapes:
+        q, k, v, rpb = (t.cuda() for t in make_inputs(replace(s, B=1)))
+        na.na2d_forward(q, k, v, rpb, s.k, s.d)
+        names.append(na.na2d_last_kernel())
+    torch.cuda.synchronize()
+    return names
 
 
 def run_e2e(args, wl, dev, rank, world, pg):
@@ -418,11 +529,12 @@ def run_e2e(args, wl, dev, rank, world, pg):
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=HEADLINE)
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed oracle leg")
+    ap.add_argument("--no-per-workload", action="store_true", help="time only the selected workload")
     ap.add_argument("--batch", type=int, default=None,
                     help="override B of every shape (a larger or smaller case of the same kernels)")
     args = ap.parse_args()

@@ -122,6 +122,13 @@ NA2D_API const char *na2d_status_str(na2d_status s);
 /* Library version: major * 10000 + minor * 100 + patch. */
 NA2D_API int na2d_version(void);
 
+/* Diagnostic.  The name of the kernel that the calling host thread's most
+ * recent na2d_forward call launched (a static string such as
+ * "fwd_stream_kernel"), or NULL if that call launched nothing (an argument
+ * error or an empty problem) or no call was made on this thread yet.  Used by
+ * the tests to record which kernel each problem shape reaches. */
+NA2D_API const char *na2d_last_kernel(void);
+
 #ifdef __cplusplus
 }
 #endif

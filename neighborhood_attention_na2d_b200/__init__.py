@@ -19,7 +19,10 @@ from __future__ import annotations
 from ._native import Na2dError, Problem, check, device_faults, lib, status_str  # noqa: F401
 
 __all__ = ["na2d_qk_rpb", "na2d_softmax", "na2d_av", "na2d_forward", "na2d_status_str", "na2d_device_faults",
-           "Na2dError", "make_problem"]
+           "na2d_last_kernel", "Na2dError", "make_problem"]
+
+# status codes used for argument errors raised before the library is called
+_ERR_NULL, _ERR_DTYPE, _ERR_SHAPE = 1, 2, 3
 
 
 def _torch():
@@ -44,10 +47,43 @@ def _ptr(t) -> int | None:
     if t is None:
         return None
     if not t.is_cuda:
-        raise Na2dError(1, "device", "tensors must be CUDA tensors (there is no CPU path)")
+        raise Na2dError(_ERR_NULL, "device", "tensors must be CUDA tensors (there is no CPU path)")
     if not t.is_contiguous():
-        raise Na2dError(3, "layout", "tensors must be contiguous")
+        raise Na2dError(_ERR_SHAPE, "layout", "tensors must be contiguous")
     return t.data_ptr()
+
+
+def _like(name: str, t, ref, shape=None, dtype=None) -> None:
+    """Checks on the host that tensor `t` has the given shape (default: ref's),
+    dtype (default: ref's) and ref's device; the library receives raw pointers
+    and could not detect a mismatch, so a short or foreign buffer is refused
+    here, before any launch."""
+    if t is None:
+        raise Na2dError(_ERR_NULL, name, f"{name} is required")
+    want_shape = tuple(ref.shape) if shape is None else tuple(shape)
+    want_dtype = ref.dtype if dtype is None else dtype
+    if t.dim() != len(want_shape) or tuple(t.shape) != want_shape:
+        raise Na2dError(_ERR_SHAPE, name, f"{name} has shape {tuple(t.shape)}, expected {want_shape}")
+    if t.dtype != want_dtype:
+        raise Na2dError(_ERR_DTYPE, name, f"{name} is {t.dtype}, expected {want_dtype}")
+    if t.device != ref.device:
+        raise Na2dError(_ERR_NULL, name, f"{name} is on {t.device}, expected {ref.device}")
+
+
+def _check_qkv(q, kernel_size: int) -> None:
+    if q.dim() != 5:
+        raise Na2dError(_ERR_SHAPE, "q", f"q must be [B, heads, H, W, D], got shape {tuple(q.shape)}")
+
+
+def _check_rpb(rpb, q, kernel_size: int) -> None:
+    if rpb is None:
+        return
+    nb = 2 * kernel_size - 1
+    _like("rpb", rpb, q, shape=(q.shape[1], nb, nb))
+
+
+def _attn_shape(x, kernel_size: int):
+    return tuple(x.shape[:4]) + (kernel_size * kernel_size,)
 
 
 def _stream(t) -> int:
@@ -67,11 +103,23 @@ def na2d_device_faults(device=None) -> int:
         return device_faults(torch.cuda.current_stream(dev).cuda_stream)
 
 
+def na2d_last_kernel() -> str | None:
+    """Name of the kernel that this thread's last na2d_forward call launched
+    (None if it launched nothing)."""
+    r = lib().na2d_last_kernel()
+    return r.decode() if r else None
+
+
 def na2d_forward(q, k, v, rpb, kernel_size: int, dilation: int = 1, out=None):
     """Fused forward: softmax(q.k/sqrt(D) + rpb) . v over each query's window."""
+    _check_qkv(q, kernel_size)
     p = make_problem(q.shape, kernel_size, dilation, q.dtype)
+    _like("k", k, q)
+    _like("v", v, q)
+    _check_rpb(rpb, q, kernel_size)
     if out is None:
         out = _torch().empty_like(q)
+    _like("out", out, q)
     ptrs = (_ptr(q), _ptr(k), _ptr(v), _ptr(rpb), _ptr(out))
     with _torch().cuda.device(q.device):
         check(lib().na2d_forward(p, *ptrs, _stream(q)), "na2d_forward")
@@ -80,10 +128,13 @@ def na2d_forward(q, k, v, rpb, kernel_size: int, dilation: int = 1, out=None):
 
 def na2d_qk_rpb(q, k, rpb, kernel_size: int, dilation: int = 1, attn=None):
     """Scores (fp32): q.k/sqrt(D) + rpb for each query's k*k neighbours."""
+    _check_qkv(q, kernel_size)
     p = make_problem(q.shape, kernel_size, dilation, q.dtype)
+    _like("k", k, q)
+    _check_rpb(rpb, q, kernel_size)
     if attn is None:
-        attn = _torch().empty(tuple(q.shape[:4]) + (kernel_size * kernel_size,), dtype=_torch().float32,
-                              device=q.device)
+        attn = _torch().empty(_attn_shape(q, kernel_size), dtype=_torch().float32, device=q.device)
+    _like("attn", attn, q, shape=_attn_shape(q, kernel_size), dtype=_torch().float32)
     ptrs = (_ptr(q), _ptr(k), _ptr(rpb), _ptr(attn))
     with _torch().cuda.device(q.device):
         check(lib().na2d_qk_rpb(p, *ptrs, _stream(q)), "na2d_qk_rpb")
@@ -92,6 +143,11 @@ def na2d_qk_rpb(q, k, rpb, kernel_size: int, dilation: int = 1, attn=None):
 
 def na2d_softmax(attn, kernel_size: int, dilation: int = 1, D: int = 32, dtype=None):
     """In-place softmax over the last (k*k) axis of an fp32 score tensor."""
+    if attn.dim() != 5 or attn.shape[4] != kernel_size * kernel_size:
+        raise Na2dError(_ERR_SHAPE, "attn", f"attn must be [B, heads, H, W, {kernel_size * kernel_size}], "
+                        f"got {tuple(attn.shape)}")
+    if attn.dtype != _torch().float32:
+        raise Na2dError(_ERR_DTYPE, "attn", f"attn must be float32, got {attn.dtype}")
     B, heads, H, W, _ = attn.shape
     p = make_problem((B, heads, H, W, D), kernel_size, dilation, dtype or _torch().float32)
     ptr = _ptr(attn)
@@ -102,9 +158,12 @@ def na2d_softmax(attn, kernel_size: int, dilation: int = 1, D: int = 32, dtype=N
 
 def na2d_av(attn, v, kernel_size: int, dilation: int = 1, out=None):
     """Weighted sum of values: out = sum_n attn[..., n] * v[key_n]."""
+    _check_qkv(v, kernel_size)
     p = make_problem(v.shape, kernel_size, dilation, v.dtype)
+    _like("attn", attn, v, shape=_attn_shape(v, kernel_size), dtype=_torch().float32)
     if out is None:
         out = _torch().empty_like(v)
+    _like("out", out, v)
     ptrs = (_ptr(attn), _ptr(v), _ptr(out))
     with _torch().cuda.device(v.device):
         check(lib().na2d_av(p, *ptrs, _stream(v)), "na2d_av")

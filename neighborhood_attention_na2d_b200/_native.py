@@ -19,7 +19,7 @@ STATUS_NAMES = {
 
 # every symbol the header declares
 EXPORTS = ("na2d_qk_rpb", "na2d_softmax", "na2d_av", "na2d_forward", "na2d_device_faults", "na2d_status_str",
-           "na2d_version")
+           "na2d_version", "na2d_last_kernel")
 
 
 class Problem(ctypes.Structure):
@@ -61,6 +61,8 @@ def lib() -> ctypes.CDLL:
         L.na2d_status_str.restype = ctypes.c_char_p
         L.na2d_version.argtypes = []
         L.na2d_version.restype = ctypes.c_int
+        L.na2d_last_kernel.argtypes = []
+        L.na2d_last_kernel.restype = ctypes.c_char_p
         _lib = L
     return _lib
 

@@ -58,6 +58,9 @@ bool rpb_aligned(const na2d_problem *p, const void *rpb) {
     return !rpb || (reinterpret_cast<uintptr_t>(rpb) % elem_size(p->dtype)) == 0;
 }
 
+// Name of the kernel the calling thread's last forward call launched.
+thread_local const char *t_last_kernel = nullptr;
+
 na2d_status from_cuda(cudaError_t e) {
     if (e == cudaSuccess) return NA2D_OK;
     cudaGetLastError();   // clear a sticky launch error for the caller's next call
@@ -65,6 +68,10 @@ na2d_status from_cuda(cudaError_t e) {
 }
 
 }  // namespace
+
+namespace na2d {
+void note_kernel(const char *name) { t_last_kernel = name; }
+}  // namespace na2d
 
 extern "C" {
 
@@ -82,6 +89,7 @@ na2d_status na2d_forward(const na2d_problem *p, const void *q, const void *k, co
     if (overlap(out, n, q, n) || overlap(out, n, k, n) || overlap(out, n, v, n) || overlap(out, n, rpb, rpb_bytes(p)))
         return NA2D_ERR_ALIAS;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    t_last_kernel = nullptr;
     if (na2d::tc_supported(pr)) {
         bool launched = false;
         cudaError_t e = na2d::launch_forward_umma(pr, q, k, v, rpb, out, st, &launched);
@@ -159,6 +167,8 @@ const char *na2d_status_str(na2d_status s) {
     return "unknown status";
 }
 
-int na2d_version(void) { return 100; }
+int na2d_version(void) { return 200; }
+
+const char *na2d_last_kernel(void) { return t_last_kernel; }
 
 }  // extern "C"

@@ -29,6 +29,10 @@ cudaError_t launch_qk_rpb(const Problem &p, const void *q, const void *k, const 
 cudaError_t launch_softmax(const Problem &p, float *attn, cudaStream_t stream);
 cudaError_t launch_av(const Problem &p, const float *attn, const void *v, void *out, cudaStream_t stream);
 
+// Records, for the calling host thread, the name of the kernel a forward call
+// has just launched (a static string); read back by na2d_last_kernel.
+void note_kernel(const char *name);
+
 // Reads and clears the count of device-side bounded waits that ran out;
 // synchronises the stream.
 cudaError_t read_device_faults(unsigned int *count, cudaStream_t stream);

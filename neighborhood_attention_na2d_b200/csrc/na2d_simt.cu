@@ -219,6 +219,7 @@ cudaError_t fwd_simt_impl(const Problem &p, const void *q, const void *k, const 
         static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v),
         static_cast<const T *>(rpb), static_cast<T *>(out), p.heads, p.H, p.W, p.k, p.d, nq,
         1.0f / sqrtf((float)p.D));
+    note_kernel("fwd_simt_kernel");
     return cudaGetLastError();
 }
 

@@ -857,6 +857,7 @@ cudaError_t launch_mode(const Args &a, int smem, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     const int64_t grid = std::min<int64_t>(a.nblocks, (int64_t)sms * occ);
     kern<<<(unsigned)grid, kThreads, smem, st>>>(a);
+    note_kernel(MODE == kFull ? "fwd_tc_kernel/full" : MODE == kDense ? "fwd_tc_kernel/dense" : "fwd_tc_kernel/generic");
     return cudaGetLastError();
 }
 
@@ -950,6 +951,7 @@ cudaError_t launch_tma(const Problem &p, const Args &base, cudaStream_t st, bool
     const int64_t grid = std::min<int64_t>((t.ntiles + t.tpb - 1) / t.tpb, (int64_t)sms * occ);
     kern<<<(unsigned)grid, R::NWC * 32, R::SMEM, st>>>(t);
     *launched = true;
+    note_kernel(MODE == kFullTma ? "fwd_sync_kernel/full_tma" : "fwd_sync_kernel/dense_tma");
     return cudaGetLastError();
 }
 

@@ -610,6 +610,7 @@ cudaError_t launch_umma_t(const Problem &pr, const void *q, const void *k, const
     cfg.numAttrs = 1;
     const cudaError_t el = cudaLaunchKernelEx(&cfg, fwd_umma_kernel<T>, up);
     *launched = true;
+    note_kernel("fwd_umma_kernel");
     return el != cudaSuccess ? el : cudaGetLastError();
 }
 

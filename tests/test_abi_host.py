@@ -101,7 +101,7 @@ def test_exports_match_header():
 
 def test_version_and_status_strings():
     build()
-    assert _native.lib().na2d_version() == 100
+    assert _native.lib().na2d_version() == 200
     names = [_native.status_str(s) for s in range(10)]
     assert names[0] == "ok" and len(set(names)) == 10
     assert _native.status_str(99) == "unknown status"
@@ -129,3 +129,67 @@ def test_binding_refuses_cpu_tensors():
     x = torch.zeros(1, 1, 7, 7, 32, dtype=torch.float16)
     with pytest.raises(na.Na2dError):
         na.na2d_forward(x, x, x, None, 7, 1, out=torch.empty_like(x))
+
+
+# ---------------------------------------------------------------------------
+# The Python binding checks every tensor against q before calling the library
+# (which receives raw pointers and cannot detect a short or mistyped buffer).
+# CPU tensors suffice: the checks run before any device work.
+def _t(*shape, dtype=None):
+    import torch
+    return torch.zeros(*shape, dtype=dtype or torch.float16)
+
+
+@pytest.mark.parametrize("case,status", [
+    ("short_k", 3), ("short_v", 3), ("k_dtype", 2), ("out_short", 3), ("out_dtype", 2),
+    ("rpb_small", 3), ("rpb_dtype", 2), ("rpb_heads", 3), ("q_4d", 3),
+])
+def test_binding_forward_mismatch(case, status):
+    import torch
+    import neighborhood_attention_na2d_b200 as na
+    q = _t(1, 2, 14, 14, 32)
+    k, v, out, rpb = _t(1, 2, 14, 14, 32), _t(1, 2, 14, 14, 32), _t(1, 2, 14, 14, 32), _t(2, 13, 13)
+    if case == "short_k":
+        k = _t(1, 2, 14, 13, 32)
+    elif case == "short_v":
+        v = _t(1, 1, 14, 14, 32)
+    elif case == "k_dtype":
+        k = _t(1, 2, 14, 14, 32, dtype=torch.bfloat16)
+    elif case == "out_short":
+        out = _t(1, 2, 14, 14, 16)
+    elif case == "out_dtype":
+        out = _t(1, 2, 14, 14, 32, dtype=torch.float32)
+    elif case == "rpb_small":
+        rpb = _t(2, 11, 11)
+    elif case == "rpb_dtype":
+        rpb = _t(2, 13, 13, dtype=torch.float32)
+    elif case == "rpb_heads":
+        rpb = _t(3, 13, 13)
+    elif case == "q_4d":
+        q = _t(2, 14, 14, 32)
+    with pytest.raises(na.Na2dError) as e:
+        na.na2d_forward(q, k, v, rpb, 7, 1, out=out)
+    assert e.value.status == status
+
+
+@pytest.mark.parametrize("case,status", [("attn_short", 3), ("attn_dtype", 2), ("av_out", 3), ("sm_shape", 3),
+                                         ("sm_dtype", 2), ("qk_k", 3)])
+def test_binding_split_mismatch(case, status):
+    import torch
+    import neighborhood_attention_na2d_b200 as na
+    q = _t(1, 2, 14, 14, 32)
+    attn = torch.zeros(1, 2, 14, 14, 49)
+    with pytest.raises(na.Na2dError) as e:
+        if case == "attn_short":
+            na.na2d_av(torch.zeros(1, 2, 14, 14, 25), q, 7, 1)
+        elif case == "attn_dtype":
+            na.na2d_av(attn.half(), q, 7, 1)
+        elif case == "av_out":
+            na.na2d_av(attn, q, 7, 1, out=_t(1, 2, 14, 14, 8))
+        elif case == "sm_shape":
+            na.na2d_softmax(torch.zeros(1, 2, 14, 14, 48), 7, 1)
+        elif case == "sm_dtype":
+            na.na2d_softmax(attn.double(), 7, 1)
+        elif case == "qk_k":
+            na.na2d_qk_rpb(q, _t(1, 2, 13, 14, 32), None, 7, 1)
+    assert e.value.status == status

@@ -1,6 +1,8 @@
 """bench.py's host-side bookkeeping (no GPU): which kernel a workload runs on,
 and the source hash that ties a committed ncu summary to the kernel code (a
 summary's DRAM traffic is reported only while that hash matches)."""
+import pytest
+
 import bench
 from neighborhood_attention_na2d_b200.inputs import WORKLOADS
 
@@ -12,6 +14,19 @@ def test_code_only_ignores_comments_and_blank_lines():
     assert bench.code_only(a) != bench.code_only(a.replace("2 * x", "3 * x"))
 
 
-def test_dominant_kernel_per_workload():
-    assert bench.dominant_kernel(WORKLOADS["nat_tiny_s1_fp16"]) == "fwd_stream_kernel"
-    assert bench.dominant_kernel(WORKLOADS["dinat_s1_bf16"]) == "fwd_umma_kernel"
+@pytest.mark.parametrize("K", [1, 3, 20, 199, 200, 201, 450, 20000])
+def test_graph_plan_times_exactly_k_steps(K):
+    """A timed run replays graphs covering exactly --steps steps, at least one
+    graph replay (the driver's --steps 20 must replay a graph, not launch
+    eagerly)."""
+    G, full, rest = bench.graph_plan(K)
+    assert 1 <= G <= 200 and 0 <= rest < G
+    assert full * G + rest == K
+    assert full >= 1
+
+
+def test_roofline_picks_the_slower_limit():
+    wl = WORKLOADS["nat_tiny_s1_fp16"]
+    r = bench.roofline(wl, 0.010, None)
+    assert r["bound"] == "hbm" and r["t_hbm_us"] > r["t_tensor_us"]
+    assert abs(r["achieved"] - wl.shapes[0].algorithmic_bytes() / 1e-5 / 1e9) < 1e-6 * r["achieved"]

@@ -181,12 +181,6 @@ def test_split_path(dtype, k, d, H, W):
     assert max_err(out.double().cpu().numpy(), oracle.forward(f64(q), f64(kk), f64(v), f64(rpb), k, d)) <= TOL[dtype]
 
 
-def test_no_device_wait_timed_out():
-    """Runs after the parity tests above (same module): no kernel gave up on a
-    bounded wait."""
-    assert na.na2d_device_faults() == 0
-
-
 def test_empty_batch():
     x = torch.empty(0, 2, 14, 14, 32, dtype=torch.float16, device="cuda")
     out = na.na2d_forward(x, x, x, None, 7, 1)
@@ -228,3 +222,81 @@ def test_bench_buffers_sampled(name):
         for (b, h, i, j) in pts:
             want = oracle.forward_query(q64, k64, v64, r64, shape.k, shape.d, b, h, i, j)
             assert float(np.abs(out[b, h, i, j] - want).max()) <= TOL[shape.dtype]
+
+
+# ---------------------------------------------------------------------------
+# Dispatch: which kernel each kind of problem reaches (na2d_last_kernel), with
+# parity.  Every branch of na2d_forward's dispatch has a row here.
+DISPATCH = [
+    (Shape(1, 3, 14, 14, 32, 7, 2, "bf16", 601), "fwd_umma_kernel"),            # every group exactly 7 x 7
+    (Shape(1, 2, 16, 16, 32, 7, 1, "f16", 602), "fwd_stream_kernel"),           # k = 7 sliding rows
+    (Shape(1, 2, 28, 28, 32, 7, 2, "bf16", 603), "fwd_sync_kernel/full_tma"),   # k <= 7, equal groups >= 14 long
+    (Shape(1, 2, 12, 12, 32, 3, 1, "f16", 604), "fwd_sync_kernel/full_tma"),
+    (Shape(1, 2, 6, 6, 32, 3, 2, "bf16", 605), "fwd_sync_kernel/dense_tma"),    # k <= 5, every group exactly k
+    (Shape(1, 2, 30, 30, 32, 9, 1, "f16", 606), "fwd_tc_kernel/full"),          # k >= 9, long groups
+    (Shape(1, 2, 13, 13, 32, 13, 1, "bf16", 607), "fwd_tc_kernel/dense"),       # k >= 9, every group exactly k
+    (Shape(1, 2, 20, 18, 32, 7, 2, "bf16", 608), "fwd_tc_kernel/generic"),      # short groups
+    (Shape(1, 2, 23, 19, 32, 5, 2, "f16", 609), "fwd_tc_kernel/full"),          # ragged groups (H, W not multiples of d)
+    (Shape(1, 2, 15, 17, 32, 5, 2, "bf16", 612), "fwd_tc_kernel/generic"),      # ragged short groups
+    (Shape(1, 2, 14, 14, 32, 7, 1, "f32", 610), "fwd_simt_kernel"),             # fp32
+    (Shape(1, 2, 5, 6, 32, 1, 1, "f16", 611), "fwd_simt_kernel"),               # k = 1
+]
+
+
+@pytest.mark.parametrize("shape,kernel", DISPATCH, ids=[f"{k}:{s.describe()}" for s, k in DISPATCH])
+def test_dispatch_table(shape, kernel):
+    (q, k, v, rpb), got = run_forward(shape)
+    assert na.na2d_last_kernel() == kernel
+    want = oracle.forward(f64(q), f64(k), f64(v), f64(rpb), shape.k, shape.d)
+    assert max_err(got, want) <= TOL[shape.dtype]
+
+
+def _chain_cases():
+    return [s for s, _ in DISPATCH[:3]] + [DISPATCH[5][0], DISPATCH[7][0], DISPATCH[9][0]]
+
+
+@pytest.mark.parametrize("graph", [False, True], ids=["eager", "graph"])
+@pytest.mark.parametrize("shape", _chain_cases(), ids=lambda s: s.describe())
+def test_chained_calls_same_stream(shape, graph):
+    """out1 = f(q, k, v); out2 = f(out1, k, v); out3 = f(out2, k, v), queued on
+    one stream with no host synchronisation (and, in the graph variant,
+    captured in one CUDA graph).  The streaming and tcgen05 kernels are
+    launched with programmatic stream serialisation; a global read placed
+    before their wait for the previous grid would read a stale out1 / out2
+    here.  Each output is checked against the oracle applied to the previous
+    GPU output."""
+    q, k, v, rpb = make_inputs(shape)
+    qd, kd, vd, rd = (t.cuda() for t in (q, k, v, rpb))
+    outs = [torch.full_like(qd, float("nan")) for _ in range(3)]
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+
+    def chain():
+        x = qd
+        for o in outs:
+            na.na2d_forward(x, kd, vd, rd, shape.k, shape.d, out=o)
+            x = o
+
+    with torch.cuda.stream(s):
+        if graph:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s):
+                chain()
+            for o in outs:
+                o.fill_(float("nan"))
+            g.replay()
+        else:
+            chain()
+    s.synchronize()
+    prev = q
+    for o in outs:
+        got = o.cpu()
+        want = oracle.forward(f64(prev), f64(k), f64(v), f64(rpb), shape.k, shape.d)
+        assert max_err(got.double().numpy(), want) <= TOL[shape.dtype]
+        prev = got
+
+
+def test_no_device_wait_timed_out():
+    """Runs after the parity tests above (same module): no kernel gave up on a
+    bounded wait."""
+    assert na.na2d_device_faults() == 0
