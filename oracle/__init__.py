@@ -92,8 +92,9 @@ class Oracle:
         lib.oracle_na2d_softmax.argtypes = [i] * 7 + [_DP, i]
         lib.oracle_na2d_av.argtypes = [i] * 7 + [_DP, _DP, _DP, i]
         lib.oracle_na2d_forward.argtypes = [i] * 7 + [_DP, _DP, _DP, _DP, _DP, i]
+        lib.oracle_na2d_backward.argtypes = [i] * 7 + [_DP] * 9 + [i]
         for f in ("oracle_axis_window", "oracle_axis_neighbors", "oracle_na2d_qk_rpb",
-                  "oracle_na2d_softmax", "oracle_na2d_av", "oracle_na2d_forward"):
+                  "oracle_na2d_softmax", "oracle_na2d_av", "oracle_na2d_forward", "oracle_na2d_backward"):
             getattr(lib, f).restype = ctypes.c_int
         self._lib = lib
 
@@ -151,6 +152,21 @@ class Oracle:
                                              nthreads or default_threads()), "forward")
         return out
 
+    def backward(self, q, k, v, rpb, dout, kernel_size: int, dilation: int, nthreads: int | None = None):
+        """Gradients (dq, dk, dv, drpb) of the fused forward for the output
+        gradient dout; drpb is returned even when rpb is None (the gradient
+        with respect to a zero bias)."""
+        q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+        rpb = None if rpb is None else _f64(rpb)
+        shp = _shape(q, kernel_size, dilation)
+        dq, dk, dv = (np.empty(q.shape, dtype=np.float64) for _ in range(3))
+        nb = 2 * kernel_size - 1
+        drpb = np.empty((q.shape[1], nb, nb), dtype=np.float64)
+        _check(self._lib.oracle_na2d_backward(*shp, _ptr(q), _ptr(k), _ptr(v), _ptr(rpb), _ptr(dout), _ptr(dq),
+                                              _ptr(dk), _ptr(dv), _ptr(drpb), nthreads or default_threads()),
+               "backward")
+        return dq, dk, dv, drpb
+
     def forward_query(self, q, k, v, rpb, kernel_size: int, dilation: int,
                       b: int, h: int, i: int, j: int) -> np.ndarray:
         """One output row from the definition, with numpy on the window that
@@ -206,3 +222,7 @@ def forward(q, k, v, rpb, kernel_size, dilation, nthreads=None):
 
 def forward_query(q, k, v, rpb, kernel_size, dilation, b, h, i, j):
     return get().forward_query(q, k, v, rpb, kernel_size, dilation, b, h, i, j)
+
+
+def backward(q, k, v, rpb, dout, kernel_size, dilation, nthreads=None):
+    return get().backward(q, k, v, rpb, dout, kernel_size, dilation, nthreads)

@@ -338,3 +338,156 @@ int oracle_na2d_forward(int B, int heads, int H, int W, int D, int k, int d,
     jb.out = out;
     return dispatch(jb, nthreads);
 }
+
+/* ---------------------------------------------------------------------------
+ * Backward of the fused definition.  The layer is trained end to end (gitcode
+ * DiNAT article, section "微调示例：加载预训练权重继续训练", fine-tuning; the
+ * HF tests it describes in "源码与测试导览" run forward and backward), so the
+ * gradients of out with respect to q, k, v and rpb are part of the method.
+ * They are the chain rule through the three stages, for one query with
+ * scores s_n, weights p_n = softmax(s)_n and output o = sum_n p_n v_n, given
+ * the output gradient g = dL/do:
+ *     dL/dv_n    += p_n g                 (key n's value, from every query
+ *                                          whose window holds key n)
+ *     dL/dp_n     = g . v_n
+ *     dL/ds_n     = p_n (dL/dp_n - sum_m p_m dL/dp_m)    (softmax Jacobian)
+ *     dL/dq      += sum_n dL/ds_n k_n / sqrt(D)
+ *     dL/dk_n    += dL/ds_n q / sqrt(D)
+ *     dL/drpb[h, by_n, bx_n] += dL/ds_n
+ * One query at a time, recomputing the forward's scores and softmax exactly
+ * as forward_slice does.  dq, dk, dv of the slice are overwritten; the bias
+ * gradient is added into drpb_acc ([heads, 2k-1, 2k-1]).
+ * ------------------------------------------------------------------------- */
+static void backward_slice(const oracle_shape *p, int bh, const double *q,
+                           const double *kk, const double *v, const double *rpb,
+                           const double *dout, double *dq, double *dk, double *dv,
+                           double *drpb_acc)
+{
+    const int H = p->H, W = p->W, D = p->D, k = p->k, d = p->d;
+    const int h = bh % p->heads;
+    const int nb = 2 * k - 1;
+    const double scale = 1.0 / sqrt((double)D);
+    const size_t base = (size_t)bh * H * W * D;
+    int *ky = malloc(sizeof(int) * k), *by = malloc(sizeof(int) * k);
+    int *kx = malloc(sizeof(int) * k), *bx = malloc(sizeof(int) * k);
+    double *sc = malloc(sizeof(double) * k * k);
+    double *dp = malloc(sizeof(double) * k * k);
+    for (size_t e = 0; e < (size_t)H * W * D; ++e) {
+        dq[base + e] = 0.0;
+        dk[base + e] = 0.0;
+        dv[base + e] = 0.0;
+    }
+    for (int i = 0; i < H; ++i) {
+        oracle_axis_neighbors(H, k, d, i, ky, by);
+        for (int j = 0; j < W; ++j) {
+            oracle_axis_neighbors(W, k, d, j, kx, bx);
+            const double *qv = q + base + ((size_t)i * W + j) * D;
+            const double *g = dout + base + ((size_t)i * W + j) * D;
+            /* scores and softmax, as in the forward */
+            for (int ty = 0; ty < k; ++ty)
+                for (int tx = 0; tx < k; ++tx) {
+                    const double *kv = kk + base + ((size_t)ky[ty] * W + kx[tx]) * D;
+                    double dot = 0.0;
+                    for (int c = 0; c < D; ++c) dot += qv[c] * kv[c];
+                    double bias = 0.0;
+                    if (rpb) bias = rpb[((size_t)h * nb + by[ty]) * nb + bx[tx]];
+                    sc[ty * k + tx] = dot * scale + bias;
+                }
+            double m = sc[0];
+            for (int t = 1; t < k * k; ++t)
+                if (sc[t] > m) m = sc[t];
+            double sum = 0.0;
+            for (int t = 0; t < k * k; ++t) {
+                sc[t] = exp(sc[t] - m);
+                sum += sc[t];
+            }
+            for (int t = 0; t < k * k; ++t) sc[t] /= sum;       /* p_n */
+            /* dL/dp_n = g . v_n, and the weighted mean sum_m p_m dL/dp_m */
+            double pdp = 0.0;
+            for (int ty = 0; ty < k; ++ty)
+                for (int tx = 0; tx < k; ++tx) {
+                    const double *vv = v + base + ((size_t)ky[ty] * W + kx[tx]) * D;
+                    double dot = 0.0;
+                    for (int c = 0; c < D; ++c) dot += g[c] * vv[c];
+                    dp[ty * k + tx] = dot;
+                    pdp += sc[ty * k + tx] * dot;
+                }
+            double *dqv = dq + base + ((size_t)i * W + j) * D;
+            for (int ty = 0; ty < k; ++ty)
+                for (int tx = 0; tx < k; ++tx) {
+                    const int n = ty * k + tx;
+                    const size_t key = base + ((size_t)ky[ty] * W + kx[tx]) * D;
+                    const double ds = sc[n] * (dp[n] - pdp);        /* dL/ds_n */
+                    for (int c = 0; c < D; ++c) {
+                        dv[key + c] += sc[n] * g[c];
+                        dqv[c] += ds * kk[key + c] * scale;
+                        dk[key + c] += ds * qv[c] * scale;
+                    }
+                    drpb_acc[((size_t)h * nb + by[ty]) * nb + bx[tx]] += ds;
+                }
+        }
+    }
+    free(ky); free(by); free(kx); free(bx); free(sc); free(dp);
+}
+
+typedef struct {
+    const oracle_shape *p;
+    int bh_begin, bh_end;
+    const double *q, *k, *v, *rpb, *dout;
+    double *dq, *dk, *dv, *drpb_acc;
+} bjob;
+
+static void *run_bjob(void *arg)
+{
+    bjob *jb = (bjob *)arg;
+    for (int bh = jb->bh_begin; bh < jb->bh_end; ++bh)
+        backward_slice(jb->p, bh, jb->q, jb->k, jb->v, jb->rpb, jb->dout, jb->dq, jb->dk, jb->dv,
+                       jb->drpb_acc);
+    return NULL;
+}
+
+/* Gradients of the fused forward.  dq, dk, dv: [B, heads, H, W, D]; drpb:
+ * [heads, 2k-1, 2k-1] or NULL (not wanted).  Threads split the (b, head)
+ * slices; each thread sums its bias gradient privately and the sums are added
+ * in thread order, so the result does not depend on timing. */
+int oracle_na2d_backward(int B, int heads, int H, int W, int D, int k, int d,
+                         const double *q, const double *kk, const double *v,
+                         const double *rpb, const double *dout, double *dq,
+                         double *dk, double *dv, double *drpb, int nthreads)
+{
+    oracle_shape p = make_shape(B, heads, H, W, D, k, d);
+    if (!shape_ok(&p)) return -1;
+    const int nb = 2 * k - 1;
+    const size_t ntab = (size_t)heads * nb * nb;
+    if (drpb)
+        for (size_t e = 0; e < ntab; ++e) drpb[e] = 0.0;
+    const int nbh = B * heads;
+    if (nbh == 0) return 0;
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > nbh) nthreads = nbh;
+    pthread_t *tid = malloc(sizeof(pthread_t) * nthreads);
+    int *created = calloc(nthreads, sizeof(int));
+    bjob *jobs = malloc(sizeof(bjob) * nthreads);
+    double *acc = calloc((size_t)nthreads * (ntab ? ntab : 1), sizeof(double));
+    for (int t = 0; t < nthreads; ++t) {
+        bjob jb = {&p, (int)((long long)nbh * t / nthreads), (int)((long long)nbh * (t + 1) / nthreads),
+                   q, kk, v, rpb, dout, dq, dk, dv, acc + (size_t)t * ntab};
+        jobs[t] = jb;
+        if (t == nthreads - 1)
+            run_bjob(&jobs[t]);
+        else if (pthread_create(&tid[t], NULL, run_bjob, &jobs[t]) == 0)
+            created[t] = 1;
+        else
+            run_bjob(&jobs[t]);
+    }
+    for (int t = 0; t < nthreads - 1; ++t)
+        if (created[t]) pthread_join(tid[t], NULL);
+    if (drpb)
+        for (int t = 0; t < nthreads; ++t)
+            for (size_t e = 0; e < ntab; ++e) drpb[e] += acc[(size_t)t * ntab + e];
+    free(acc);
+    free(tid);
+    free(created);
+    free(jobs);
+    return 0;
+}

@@ -20,7 +20,13 @@ What fixes each expected value (never the oracle's own formula retyped):
   * a one-hot bias with zero q, k: closed form of the weights, which fixes the
     bias table's orientation (row = vertical offset key' - i' + k - 1);
   * translation equivariance of unclamped queries (NA abstract, HF NAT page);
-  * the pages' DiNAT stage table (tests/golden/dinat_stage_table.txt).
+  * the pages' DiNAT stage table (tests/golden/dinat_stage_table.txt);
+  * backward: central finite differences of the (pinned) forward, exhaustively
+    on tiny maps; gradients of dense softmax attention from torch autograd in
+    fp64 when the window covers the image; calculus identities (softmax
+    gradients sum to zero, so every head's bias gradient sums to zero; the
+    weights sum to one, so the value gradients sum to the output gradients);
+    the dilation decomposition carried over to the gradients.
 """
 from __future__ import annotations
 
@@ -280,6 +286,105 @@ def pin_forward_query(orc):
                                    rtol=0, atol=TOL)
 
 
+# ---------------------------------------------------------------------------
+# Backward.
+def _loss(orc, q, kk, v, rpb, dout, k, d):
+    return float((orc.forward(q, kk, v, rpb, k, d) * dout).sum())
+
+
+def pin_backward_finite_differences(orc):
+    """Every entry of dq, dk, dv and drpb equals the central difference of
+    L = sum(dout * forward) with step 1e-5 (error O(1e-10)), on tiny maps with
+    clamped edges and dilation."""
+    rng = np.random.default_rng(21)
+    for (B, heads, H, W, D, k, d) in [(1, 2, 5, 6, 3, 3, 1), (1, 1, 7, 6, 2, 3, 2), (2, 1, 5, 5, 2, 5, 1)]:
+        q, kk, v, rpb = _rand(rng, B, heads, H, W, D, k)
+        dout = rng.standard_normal(q.shape)
+        dq, dk, dv, drpb = orc.backward(q, kk, v, rpb, dout, k, d)
+        eps = 1e-5
+        for name, x, grad in (("q", q, dq), ("k", kk, dk), ("v", v, dv), ("rpb", rpb, drpb)):
+            num = np.empty_like(x)
+            flat, nflat = x.reshape(-1), num.reshape(-1)
+            for e in range(flat.size):
+                old = flat[e]
+                flat[e] = old + eps
+                up = _loss(orc, q, kk, v, rpb, dout, k, d)
+                flat[e] = old - eps
+                dn = _loss(orc, q, kk, v, rpb, dout, k, d)
+                flat[e] = old
+                nflat[e] = (up - dn) / (2 * eps)
+            np.testing.assert_allclose(grad, num, rtol=1e-6, atol=1e-7, err_msg=f"d{name} {(H, W, k, d)}")
+
+
+def pin_backward_dense_autograd(orc):
+    """k = H = W, d = 1: NA is dense softmax attention with the bias matrix
+    Bias[(iy, ix), (jy, jx)] = rpb[h, jy - iy + k - 1, jx - ix + k - 1]; its
+    gradients come from torch autograd (fp64), not from the oracle."""
+    import torch
+    rng = np.random.default_rng(22)
+    for k in (3, 5):
+        B, heads, D = 2, 2, 4
+        q, kk, v, rpb = _rand(rng, B, heads, k, k, D, k)
+        dout = rng.standard_normal(q.shape)
+        T = [torch.tensor(a, dtype=torch.float64, requires_grad=True) for a in (q, kk, v, rpb)]
+        iy, ix = np.divmod(np.arange(k * k), k)
+        ry = torch.tensor(iy[None, :] - iy[:, None] + k - 1)
+        rx = torch.tensor(ix[None, :] - ix[:, None] + k - 1)
+        bias = T[3][:, ry, rx]                                   # [heads, k*k, k*k]
+        Q, K, V = (t.reshape(B, heads, k * k, D) for t in T[:3])
+        S = Q @ K.transpose(-1, -2) / math.sqrt(D) + bias
+        O = torch.softmax(S, dim=-1) @ V
+        O.reshape(q.shape).backward(torch.tensor(dout))
+        got = orc.backward(q, kk, v, rpb, dout, k, 1)
+        for g, t in zip(got, T):
+            np.testing.assert_allclose(g, t.grad.numpy(), rtol=0, atol=1e-11)
+
+
+def pin_backward_identities(orc):
+    """Softmax gradients sum to zero over a window, so each head's bias
+    gradient sums to zero; the weights of every window sum to one, so per
+    (b, head) the value gradients sum to the output gradients; with q = 0
+    and no bias (uniform weights) dv at a key is dout summed over the queries
+    whose (searched) window holds it, divided by k*k."""
+    rng = np.random.default_rng(23)
+    H, W, k, d = 9, 11, 3, 2
+    q, kk, v, rpb = _rand(rng, 2, 3, H, W, 4, k)
+    dout = rng.standard_normal(q.shape)
+    dq, dk, dv, drpb = orc.backward(q, kk, v, rpb, dout, k, d)
+    np.testing.assert_allclose(drpb.sum(axis=(1, 2)), 0.0, rtol=0, atol=1e-11)
+    np.testing.assert_allclose(dv.sum(axis=(2, 3)), dout.sum(axis=(2, 3)), rtol=0, atol=1e-11)
+    _, _, dv0, _ = orc.backward(np.zeros_like(q), kk, v, None, dout, k, d)
+    want = np.zeros_like(dv0)
+    for i in range(H):
+        ky, _ = axis_window_search(H, k, d, i)
+        for j in range(W):
+            kx, _ = axis_window_search(W, k, d, j)
+            for y in ky:
+                for x in kx:
+                    want[:, :, y, x] += dout[:, :, i, j] / (k * k)
+    np.testing.assert_allclose(dv0, want, rtol=0, atol=1e-12)
+
+
+def pin_backward_dilation_decomposition(orc):
+    """Gradients of NA(x; k, d) are the d x d interleave of the gradients of
+    NA(x[gy::d, gx::d]; k, 1); the bias gradient is their sum."""
+    rng = np.random.default_rng(24)
+    for H, W, k, d in [(14, 13, 3, 2), (16, 16, 5, 3)]:
+        q, kk, v, rpb = _rand(rng, 1, 2, H, W, 3, k)
+        dout = rng.standard_normal(q.shape)
+        got = orc.backward(q, kk, v, rpb, dout, k, d)
+        drpb_sum = np.zeros_like(got[3])
+        for gy in range(d):
+            for gx in range(d):
+                sub = [np.ascontiguousarray(a[:, :, gy::d, gx::d]) for a in (q, kk, v, dout)]
+                want = orc.backward(sub[0], sub[1], sub[2], rpb, sub[3], k, 1)
+                for g, w in zip(got[:3], want[:3]):
+                    np.testing.assert_allclose(g[:, :, gy::d, gx::d], w, rtol=0, atol=TOL)
+                drpb_sum += want[3]
+        np.testing.assert_allclose(got[3], drpb_sum, rtol=0, atol=1e-11)
+
+
 ALL_PINS = [pin_window_keyset, pin_full_attention, pin_brute_force, pin_dilation_decomposition,
             pin_invariants, pin_rpb_orientation, pin_translation, pin_split_stages, pin_stage_table,
-            pin_forward_query]
+            pin_forward_query, pin_backward_finite_differences, pin_backward_dense_autograd,
+            pin_backward_identities, pin_backward_dilation_decomposition]

@@ -45,6 +45,17 @@ MUTANTS = {
                              ("const double *vv = vs + ((size_t)ky[ty] * W + kx[tx]) * D;",
                               "const double *vv = vs + ((size_t)ky[tx] * W + kx[ty]) * D;")],
     "av_uses_keys": [("const double *vv = v + base +", "const double *vv = kk + base +")],
+    # backward (every index unchanged, only the arithmetic)
+    "bwd_drops_softmax_mean": [("const double ds = sc[n] * (dp[n] - pdp);", "const double ds = sc[n] * dp[n];")],
+    "bwd_mean_unweighted": [("pdp += sc[ty * k + tx] * dot;", "pdp += dot;")],
+    "bwd_dp_uses_query": [("dot += g[c] * vv[c];", "dot += g[c] * qv[c];")],
+    "bwd_dq_unscaled": [("dqv[c] += ds * kk[key + c] * scale;", "dqv[c] += ds * kk[key + c];")],
+    "bwd_dk_uses_key": [("dk[key + c] += ds * qv[c] * scale;", "dk[key + c] += ds * kk[key + c] * scale;")],
+    "bwd_dv_uses_ds": [("dv[key + c] += sc[n] * g[c];", "dv[key + c] += ds * g[c];")],
+    "bwd_drpb_transposed": [("drpb_acc[((size_t)h * nb + by[ty]) * nb + bx[tx]] += ds;",
+                             "drpb_acc[((size_t)h * nb + bx[tx]) * nb + by[ty]] += ds;")],
+    "bwd_drpb_uses_p": [("drpb_acc[((size_t)h * nb + by[ty]) * nb + bx[tx]] += ds;",
+                         "drpb_acc[((size_t)h * nb + by[ty]) * nb + bx[tx]] += sc[n];")],
 }
 
 
