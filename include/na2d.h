@@ -107,6 +107,34 @@ NA2D_API na2d_status na2d_av(const na2d_problem *p, const float *attn, const voi
 NA2D_API na2d_status na2d_forward(const na2d_problem *p, const void *q, const void *k, const void *v,
                          const void *rpb, void *out, void *stream);
 
+/* Bytes of device workspace na2d_backward needs for problem p: fp32
+ * log-sum-exp and delta per query and head (8 bytes each pair) plus an fp32
+ * bias-gradient table of heads * (2k-1)^2 floats.  Writes 0 for an empty
+ * problem.  Host-only; launches nothing. */
+NA2D_API na2d_status na2d_backward_workspace_size(const na2d_problem *p, size_t *bytes);
+
+/* Backward of na2d_forward.  The layer is trained end to end ("Dilated
+ * Neighborhood Attention Transformer", gitcode DiNAT article, section
+ * "微调示例：加载预训练权重继续训练"), and its gradients are the chain rule through
+ * scores -> softmax -> weighted sum: for a query with weights p_n and output
+ * gradient g, dp_n = g . v_n, ds_n = p_n (dp_n - sum_m p_m dp_m),
+ *     dq = sum_n ds_n key_n / sqrt(D),  dk_n += ds_n q / sqrt(D),
+ *     dv_n += p_n g,  drpb[h, key' - i' + k - 1 (both axes)] += ds_n.
+ * Inputs: q, k, v, dout [B,heads,H,W,D] and rpb [heads,2k-1,2k-1] (or NULL
+ * for a zero bias), in the problem's dtype.  Outputs: dq, dk, dv
+ * [B,heads,H,W,D] and drpb [heads,2k-1,2k-1] (or NULL if not wanted), in the
+ * problem's dtype, fully overwritten.  workspace: a caller-owned device buffer
+ * of at least na2d_backward_workspace_size() bytes, 16-byte aligned, used as
+ * scratch (its contents are undefined afterwards).  Same supported set,
+ * ownership, threading and error rules as na2d_forward; no output or the
+ * workspace may overlap an input or another output (NA2D_ERR_ALIAS); a
+ * workspace smaller than required returns NA2D_ERR_SHAPE.  fp32 arithmetic;
+ * the bias gradient is summed in fp32 with atomics, so its last bits may vary
+ * from run to run. */
+NA2D_API na2d_status na2d_backward(const na2d_problem *p, const void *q, const void *k, const void *v,
+                                   const void *rpb, const void *dout, void *dq, void *dk, void *dv, void *drpb,
+                                   void *workspace, size_t workspace_bytes, void *stream);
+
 /* Diagnostic.  Kernels that wait on shared-memory barriers for their own
  * tensor copies give up after about a second of device time (a wait that long
  * means the copy will never arrive), skip their remaining work and count the

@@ -8,6 +8,8 @@ in the library's sm_100a kernels):
     na2d_softmax(attn, kernel_size, dilation)            -> attn  (in place)
     na2d_av(attn, v, kernel_size, dilation)              -> out   [B,heads,H,W,D]
     na2d_forward(q, k, v, rpb, kernel_size, dilation)    -> out   (fused)
+    na2d_backward(q, k, v, rpb, dout, kernel_size, dilation) -> (dq, dk, dv, drpb)
+    na2d(q, k, v, rpb, kernel_size, dilation)            -> out   (autograd: backward via na2d_backward)
 
 q, k, v are contiguous [B, heads, H, W, D] tensors in float32, float16 or
 bfloat16 on one CUDA device; rpb is [heads, 2k-1, 2k-1] in the same dtype, or
@@ -16,10 +18,10 @@ from the library raises ``Na2dError``; there is no CPU fallback.
 """
 from __future__ import annotations
 
-from ._native import Na2dError, Problem, check, device_faults, lib, status_str  # noqa: F401
+from ._native import Na2dError, Problem, backward_workspace_size, check, device_faults, lib, status_str  # noqa: F401
 
 __all__ = ["na2d_qk_rpb", "na2d_softmax", "na2d_av", "na2d_forward", "na2d_status_str", "na2d_device_faults",
-           "na2d_last_kernel", "Na2dError", "make_problem"]
+           "na2d_last_kernel", "na2d_backward", "na2d", "Na2dError", "make_problem"]
 
 # status codes used for argument errors raised before the library is called
 _ERR_NULL, _ERR_DTYPE, _ERR_SHAPE = 1, 2, 3
@@ -168,3 +170,73 @@ def na2d_av(attn, v, kernel_size: int, dilation: int = 1, out=None):
     with _torch().cuda.device(v.device):
         check(lib().na2d_av(p, *ptrs, _stream(v)), "na2d_av")
     return out
+
+
+def na2d_backward(q, k, v, rpb, dout, kernel_size: int, dilation: int = 1, dq=None, dk=None, dv=None, drpb=None,
+                  workspace=None):
+    """Gradients (dq, dk, dv, drpb) of na2d_forward for the output gradient
+    dout; drpb is None when rpb is None.  The fp32 workspace is allocated with
+    torch unless given (a uint8 CUDA tensor of at least
+    backward_workspace_size bytes)."""
+    torch = _torch()
+    _check_qkv(q, kernel_size)
+    p = make_problem(q.shape, kernel_size, dilation, q.dtype)
+    for name, t in (("k", k), ("v", v), ("dout", dout)):
+        _like(name, t, q)
+    _check_rpb(rpb, q, kernel_size)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        _like(name, t, q)
+    if rpb is not None and drpb is None:
+        drpb = torch.empty_like(rpb)
+    if drpb is not None:
+        _check_rpb(drpb, q, kernel_size)
+    need = backward_workspace_size(p)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    if workspace.device != q.device:
+        raise Na2dError(_ERR_NULL, "workspace", f"workspace is on {workspace.device}, expected {q.device}")
+    nbytes = workspace.numel() * workspace.element_size()
+    ptrs = (_ptr(q), _ptr(k), _ptr(v), _ptr(rpb), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(drpb),
+            _ptr(workspace))
+    with torch.cuda.device(q.device):
+        check(lib().na2d_backward(p, *ptrs, nbytes, _stream(q)), "na2d_backward")
+    return dq, dk, dv, drpb
+
+
+def _autograd_function():
+    torch = _torch()
+
+    class _NA2D(torch.autograd.Function):
+        """Autograd wrapper: forward = na2d_forward, backward = na2d_backward
+        (both in the library's kernels)."""
+
+        @staticmethod
+        def forward(ctx, q, k, v, rpb, kernel_size, dilation):
+            q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+            rpb = None if rpb is None else rpb.contiguous()
+            ctx.save_for_backward(q, k, v, rpb)
+            ctx.kd = (kernel_size, dilation)
+            return na2d_forward(q, k, v, rpb, kernel_size, dilation)
+
+        @staticmethod
+        def backward(ctx, dout):
+            q, k, v, rpb = ctx.saved_tensors
+            dq, dk, dv, drpb = na2d_backward(q, k, v, rpb, dout.contiguous(), *ctx.kd)
+            return dq, dk, dv, drpb, None, None
+
+    return _NA2D
+
+
+_NA2D = None
+
+
+def na2d(q, k, v, rpb, kernel_size: int, dilation: int = 1):
+    """Differentiable neighborhood attention (forward and backward in the
+    library's kernels), for training with torch autograd."""
+    global _NA2D
+    if _NA2D is None:
+        _NA2D = _autograd_function()
+    return _NA2D.apply(q, k, v, rpb, kernel_size, dilation)

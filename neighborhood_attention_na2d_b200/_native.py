@@ -19,7 +19,7 @@ STATUS_NAMES = {
 
 # every symbol the header declares
 EXPORTS = ("na2d_qk_rpb", "na2d_softmax", "na2d_av", "na2d_forward", "na2d_device_faults", "na2d_status_str",
-           "na2d_version", "na2d_last_kernel")
+           "na2d_version", "na2d_last_kernel", "na2d_backward_workspace_size", "na2d_backward")
 
 
 class Problem(ctypes.Structure):
@@ -61,6 +61,10 @@ def lib() -> ctypes.CDLL:
         L.na2d_status_str.restype = ctypes.c_char_p
         L.na2d_version.argtypes = []
         L.na2d_version.restype = ctypes.c_int
+        L.na2d_backward_workspace_size.argtypes = [P, ctypes.POINTER(ctypes.c_size_t)]
+        L.na2d_backward_workspace_size.restype = ctypes.c_int
+        L.na2d_backward.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
+        L.na2d_backward.restype = ctypes.c_int
         L.na2d_last_kernel.argtypes = []
         L.na2d_last_kernel.restype = ctypes.c_char_p
         _lib = L
@@ -92,6 +96,18 @@ def softmax_ptr(p: Problem, attn: int, stream: int = 0) -> int:
 
 def av_ptr(p: Problem, attn: int, v: int, out: int, stream: int = 0) -> int:
     return lib().na2d_av(ctypes.byref(p), attn, v, out, stream)
+
+
+def backward_workspace_size(p: Problem) -> int:
+    n = ctypes.c_size_t(0)
+    check(lib().na2d_backward_workspace_size(ctypes.byref(p), ctypes.byref(n)), "na2d_backward_workspace_size")
+    return n.value
+
+
+def backward_ptr(p: Problem, q: int, k: int, v: int, rpb: int | None, dout: int, dq: int, dk: int, dv: int,
+                 drpb: int | None, workspace: int, workspace_bytes: int, stream: int = 0) -> int:
+    return lib().na2d_backward(ctypes.byref(p), q, k, v, rpb, dout, dq, dk, dv, drpb, workspace, workspace_bytes,
+                               stream)
 
 
 def device_faults(stream: int = 0) -> int:

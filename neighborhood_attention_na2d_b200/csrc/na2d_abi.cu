@@ -140,6 +140,46 @@ na2d_status na2d_av(const na2d_problem *p, const float *attn, const void *v, voi
     return from_cuda(na2d::launch_av(pr, attn, v, out, static_cast<cudaStream_t>(stream)));
 }
 
+na2d_status na2d_backward_workspace_size(const na2d_problem *p, size_t *bytes) {
+    Problem pr;
+    bool empty = false;
+    if (!bytes) return NA2D_ERR_NULL;
+    na2d_status s = check_problem(p, &pr, &empty);
+    if (s != NA2D_OK) return s;
+    *bytes = empty ? 0 : na2d::backward_workspace_bytes(pr);
+    return NA2D_OK;
+}
+
+na2d_status na2d_backward(const na2d_problem *p, const void *q, const void *k, const void *v, const void *rpb,
+                          const void *dout, void *dq, void *dk, void *dv, void *drpb, void *workspace,
+                          size_t workspace_bytes, void *stream) {
+    Problem pr;
+    bool empty = false;
+    na2d_status s = check_problem(p, &pr, &empty);
+    if (s != NA2D_OK) return s;
+    if (empty) return NA2D_OK;
+    if (!q || !k || !v || !dout || !dq || !dk || !dv || !workspace) return NA2D_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dq) || !aligned16(dk) ||
+        !aligned16(dv) || !aligned16(workspace) || !rpb_aligned(p, rpb) || !rpb_aligned(p, drpb))
+        return NA2D_ERR_ALIGN;
+    const size_t need = na2d::backward_workspace_bytes(pr);
+    if (workspace_bytes < need) return NA2D_ERR_SHAPE;
+    const size_t n = tensor_bytes(p), nr = rpb_bytes(p);
+    const void *ins[5] = {q, k, v, dout, rpb};
+    const size_t in_n[5] = {n, n, n, n, nr};
+    const void *outs[5] = {dq, dk, dv, drpb, workspace};
+    const size_t out_n[5] = {n, n, n, nr, need};
+    for (int o = 0; o < 5; ++o) {
+        for (int i = 0; i < 5; ++i)
+            if (overlap(outs[o], out_n[o], ins[i], in_n[i])) return NA2D_ERR_ALIAS;
+        for (int o2 = o + 1; o2 < 5; ++o2)
+            if (overlap(outs[o], out_n[o], outs[o2], out_n[o2])) return NA2D_ERR_ALIAS;
+    }
+    t_last_kernel = nullptr;
+    return from_cuda(na2d::launch_backward(pr, q, k, v, rpb, dout, dq, dk, dv, drpb, workspace,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
 na2d_status na2d_device_faults(unsigned int *count, void *stream) {
     if (!count) return NA2D_ERR_NULL;
     unsigned int a = 0, b = 0, c = 0;

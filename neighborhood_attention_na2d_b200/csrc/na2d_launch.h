@@ -29,6 +29,13 @@ cudaError_t launch_qk_rpb(const Problem &p, const void *q, const void *k, const 
 cudaError_t launch_softmax(const Problem &p, float *attn, cudaStream_t stream);
 cudaError_t launch_av(const Problem &p, const float *attn, const void *v, void *out, cudaStream_t stream);
 
+// Backward (dq, dk, dv, drpb) of the fused forward; workspace holds
+// backward_workspace_bytes(p) bytes of fp32 scratch.
+size_t backward_workspace_bytes(const Problem &p);
+cudaError_t launch_backward(const Problem &p, const void *q, const void *k, const void *v, const void *rpb,
+                            const void *dout, void *dq, void *dk, void *dv, void *drpb, void *workspace,
+                            cudaStream_t stream);
+
 // Records, for the calling host thread, the name of the kernel a forward call
 // has just launched (a static string); read back by na2d_last_kernel.
 void note_kernel(const char *name);

@@ -67,6 +67,19 @@ def _host_checks() -> dict:
     r["empty_softmax"] = _native.softmax_ptr(prob(B=0), 0)
     r["empty_av"] = _native.av_ptr(prob(B=0), 0, 0, 0)
     r["faults_null"] = L.na2d_device_faults(None, None)
+    ws = _native.backward_workspace_size(p)
+    r["ws_bytes"] = ws
+    r["ws_empty"] = _native.backward_workspace_size(prob(B=0))
+    F = [FAKE + 0x100000 * i for i in range(1, 10)]   # disjoint, 16-byte aligned
+    r["bwd_null_dout"] = _native.backward_ptr(p, F[0], F[1], F[2], None, 0, F[3], F[4], F[5], None, F[6], ws)
+    r["bwd_null_ws"] = _native.backward_ptr(p, F[0], F[1], F[2], None, F[7], F[3], F[4], F[5], None, 0, ws)
+    r["bwd_small_ws"] = _native.backward_ptr(p, F[0], F[1], F[2], None, F[7], F[3], F[4], F[5], None, F[6], ws - 4)
+    r["bwd_align"] = _native.backward_ptr(p, F[0], F[1], F[2], None, F[7], F[3] + 8, F[4], F[5], None, F[6], ws)
+    r["bwd_alias_in"] = _native.backward_ptr(p, F[0], F[1], F[2], None, F[7], F[0], F[4], F[5], None, F[6], ws)
+    r["bwd_alias_out"] = _native.backward_ptr(p, F[0], F[1], F[2], None, F[7], F[3], F[3], F[5], None, F[6], ws)
+    r["bwd_alias_ws"] = _native.backward_ptr(p, F[0], F[1], F[2], None, F[7], F[3], F[4], F[5], None, F[7], ws)
+    r["bwd_bad_k"] = _native.backward_ptr(prob(k=4), F[0], F[1], F[2], None, F[7], F[3], F[4], F[5], None, F[6], ws)
+    r["bwd_empty"] = _native.backward_ptr(prob(B=0), 0, 0, 0, None, 0, 0, 0, 0, None, 0, 0)
     return r
 
 
@@ -79,6 +92,12 @@ def host_results():
     out = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=300)
     assert out.returncode == 0, out.stderr
     return json.loads(out.stdout.strip().splitlines()[-1])
+
+
+def test_backward_workspace_size(host_results):
+    """[lse, delta] fp32 per query and head plus the fp32 bias table."""
+    assert host_results["ws_bytes"] == (2 * 2 * 2 * 14 * 14 + 2 * 13 * 13) * 4
+    assert host_results["ws_empty"] == 0
 
 
 def header_functions():
@@ -117,6 +136,8 @@ def test_forward_rejects_bad_problems(host_results, i):
     ("align_q", 6), ("align_rpb", 6), ("align_attn", 6), ("align_softmax", 6), ("align_av", 6),
     ("alias_out_q", 7), ("alias_partial", 7), ("alias_av", 7),
     ("empty_B", 0), ("empty_heads", 0), ("empty_qk", 0), ("empty_softmax", 0), ("empty_av", 0), ("faults_null", 1),
+    ("bwd_null_dout", 1), ("bwd_null_ws", 1), ("bwd_small_ws", 3), ("bwd_align", 6), ("bwd_alias_in", 7),
+    ("bwd_alias_out", 7), ("bwd_alias_ws", 7), ("bwd_bad_k", 4), ("bwd_empty", 0),
 ])
 def test_host_checks(host_results, case, status):
     assert host_results[case] == status
