@@ -135,6 +135,28 @@ NA2D_API na2d_status na2d_backward(const na2d_problem *p, const void *q, const v
                                    const void *rpb, const void *dout, void *dq, void *dk, void *dv, void *drpb,
                                    void *workspace, size_t workspace_bytes, void *stream);
 
+/* na2d_backward without a workspace argument, for callers that cannot
+ * allocate device memory: code whose host framework owns every device
+ * allocation and allows none during execution, or a loop that cannot accept
+ * the device-wide synchronisation a cudaMalloc / cudaFree may cause.  The
+ * papers have no counterpart to this call; it exists only for such callers.
+ * It computes exactly what na2d_backward computes, but its scratch is a
+ * 16 MiB array built into the library, which every GPU that loads the
+ * library holds until the process exits.  Problems whose workspace
+ * (na2d_backward_workspace_size: 8 bytes per query and head plus
+ * 4 * heads * (2k-1)^2 bytes) exceeds 16 MiB are refused with NA2D_ERR_SHAPE
+ * before any launch.  The call allocates nothing.  Its first call on a device
+ * looks up the array's device address with that device current (a host-side
+ * step done once per device); make that first call before any stream capture.
+ * All calls share the one array and it keeps the last call's contents (the
+ * call clears what must start at zero), so calls whose work can overlap on
+ * the GPU, e.g. on two streams without ordering between them, race on it and
+ * give wrong results.  Arguments, outputs and errors otherwise as for
+ * na2d_backward. */
+NA2D_API na2d_status na2d_backward_noalloc(const na2d_problem *p, const void *q, const void *k, const void *v,
+                                           const void *rpb, const void *dout, void *dq, void *dk, void *dv,
+                                           void *drpb, void *stream);
+
 /* Diagnostic.  Kernels that wait on shared-memory barriers for their own
  * tensor copies give up after about a second of device time (a wait that long
  * means the copy will never arrive), skip their remaining work and count the

@@ -19,7 +19,8 @@ STATUS_NAMES = {
 
 # every symbol the header declares
 EXPORTS = ("na2d_qk_rpb", "na2d_softmax", "na2d_av", "na2d_forward", "na2d_device_faults", "na2d_status_str",
-           "na2d_version", "na2d_last_kernel", "na2d_backward_workspace_size", "na2d_backward")
+           "na2d_version", "na2d_last_kernel", "na2d_backward_workspace_size", "na2d_backward",
+           "na2d_backward_noalloc")
 
 
 class Problem(ctypes.Structure):
@@ -65,6 +66,8 @@ def lib() -> ctypes.CDLL:
         L.na2d_backward_workspace_size.restype = ctypes.c_int
         L.na2d_backward.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
         L.na2d_backward.restype = ctypes.c_int
+        L.na2d_backward_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.na2d_backward_noalloc.restype = ctypes.c_int
         L.na2d_last_kernel.argtypes = []
         L.na2d_last_kernel.restype = ctypes.c_char_p
         _lib = L
@@ -108,6 +111,12 @@ def backward_ptr(p: Problem, q: int, k: int, v: int, rpb: int | None, dout: int,
                  drpb: int | None, workspace: int, workspace_bytes: int, stream: int = 0) -> int:
     return lib().na2d_backward(ctypes.byref(p), q, k, v, rpb, dout, dq, dk, dv, drpb, workspace, workspace_bytes,
                                stream)
+
+
+def backward_noalloc_ptr(p: Problem, q: int, k: int, v: int, rpb: int | None, dout: int, dq: int, dk: int, dv: int,
+                         drpb: int | None, stream: int = 0) -> int:
+    """na2d_backward with the library's built-in scratch (no workspace)."""
+    return lib().na2d_backward_noalloc(ctypes.byref(p), q, k, v, rpb, dout, dq, dk, dv, drpb, stream)
 
 
 def device_faults(stream: int = 0) -> int:

@@ -180,6 +180,36 @@ na2d_status na2d_backward(const na2d_problem *p, const void *q, const void *k, c
                                            static_cast<cudaStream_t>(stream)));
 }
 
+na2d_status na2d_backward_noalloc(const na2d_problem *p, const void *q, const void *k, const void *v,
+                                  const void *rpb, const void *dout, void *dq, void *dk, void *dv, void *drpb,
+                                  void *stream) {
+    Problem pr;
+    bool empty = false;
+    na2d_status s = check_problem(p, &pr, &empty);
+    if (s != NA2D_OK) return s;
+    if (empty) return NA2D_OK;
+    if (!q || !k || !v || !dout || !dq || !dk || !dv) return NA2D_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dq) || !aligned16(dk) ||
+        !aligned16(dv) || !rpb_aligned(p, rpb) || !rpb_aligned(p, drpb))
+        return NA2D_ERR_ALIGN;
+    // the built-in scratch has a fixed size: larger problems are refused here
+    if (na2d::backward_workspace_bytes(pr) > na2d::noalloc_scratch_bytes()) return NA2D_ERR_SHAPE;
+    const size_t n = tensor_bytes(p), nr = rpb_bytes(p);
+    const void *ins[5] = {q, k, v, dout, rpb};
+    const size_t in_n[5] = {n, n, n, n, nr};
+    void *outs[4] = {dq, dk, dv, drpb};
+    const size_t out_n[4] = {n, n, n, nr};
+    for (int o = 0; o < 4; ++o) {
+        for (int i = 0; i < 5; ++i)
+            if (overlap(outs[o], out_n[o], ins[i], in_n[i])) return NA2D_ERR_ALIAS;
+        for (int o2 = o + 1; o2 < 4; ++o2)
+            if (overlap(outs[o], out_n[o], outs[o2], out_n[o2])) return NA2D_ERR_ALIAS;
+    }
+    t_last_kernel = nullptr;
+    return from_cuda(na2d::launch_backward_noalloc(pr, q, k, v, rpb, dout, dq, dk, dv, drpb,
+                                                   static_cast<cudaStream_t>(stream)));
+}
+
 na2d_status na2d_device_faults(unsigned int *count, void *stream) {
     if (!count) return NA2D_ERR_NULL;
     unsigned int a = 0, b = 0, c = 0;

@@ -28,6 +28,8 @@
 #include <cuda_runtime.h>
 
 #include <cfloat>
+#include <map>
+#include <mutex>
 
 #include "na2d_device.cuh"
 #include "na2d_launch.h"
@@ -267,6 +269,23 @@ template <typename T> cudaError_t launch_bwd_t(const BwdArgs &a, int64_t bh, cud
     return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// Built-in scratch for na2d_backward_noalloc: the same workspace as above
+// ([lse, delta] per query and head, then the fp32 bias table), held in a
+// fixed array that every GPU loading the library keeps until the process
+// exits, for callers that cannot allocate device memory themselves.
+constexpr size_t kNoAllocScratchBytes = (size_t)16 << 20;   // 16 MiB
+static __device__ __align__(256) unsigned char g_bwd_noalloc_scratch[kNoAllocScratchBytes];
+
+struct NoAllocAddrs {
+    std::mutex mu;
+    std::map<int, void *> dev;   // device -> device address of g_bwd_noalloc_scratch
+};
+NoAllocAddrs &noalloc_addrs() {
+    static NoAllocAddrs a;
+    return a;
+}
+
 }  // namespace
 
 size_t backward_workspace_bytes(const Problem &p) {
@@ -295,6 +314,33 @@ cudaError_t launch_backward(const Problem &p, const void *q, const void *k, cons
     case DType::F16: return launch_bwd_t<__half>(a, p.bh(), st);
     default: return launch_bwd_t<__nv_bfloat16>(a, p.bh(), st);
     }
+}
+
+
+size_t noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
+
+// The array's name is only a host-side stand-in in host code; its device
+// address is looked up once per device, with that device current, on the
+// first call there.
+cudaError_t launch_backward_noalloc(const Problem &p, const void *q, const void *k, const void *v, const void *rpb,
+                                    const void *dout, void *dq, void *dk, void *dv, void *drpb, cudaStream_t st) {
+    if (backward_workspace_bytes(p) > kNoAllocScratchBytes) return cudaErrorInvalidValue;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    void *scratch = nullptr;
+    {
+        NoAllocAddrs &a = noalloc_addrs();
+        std::lock_guard<std::mutex> lock(a.mu);
+        auto it = a.dev.find(dev);
+        if (it == a.dev.end()) {
+            e = cudaGetSymbolAddress(&scratch, g_bwd_noalloc_scratch);
+            if (e != cudaSuccess) return e;
+            it = a.dev.emplace(dev, scratch).first;
+        }
+        scratch = it->second;
+    }
+    return launch_backward(p, q, k, v, rpb, dout, dq, dk, dv, drpb, scratch, st);
 }
 
 }  // namespace na2d

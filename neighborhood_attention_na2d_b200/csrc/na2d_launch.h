@@ -36,6 +36,13 @@ cudaError_t launch_backward(const Problem &p, const void *q, const void *k, cons
                             const void *dout, void *dq, void *dk, void *dv, void *drpb, void *workspace,
                             cudaStream_t stream);
 
+// The backward with the library's built-in scratch array instead of a
+// caller workspace (no allocation); problems whose workspace exceeds
+// noalloc_scratch_bytes() are refused by the caller of this function.
+size_t noalloc_scratch_bytes();
+cudaError_t launch_backward_noalloc(const Problem &p, const void *q, const void *k, const void *v, const void *rpb,
+                                    const void *dout, void *dq, void *dk, void *dv, void *drpb, cudaStream_t stream);
+
 // Records, for the calling host thread, the name of the kernel a forward call
 // has just launched (a static string); read back by na2d_last_kernel.
 void note_kernel(const char *name);
