@@ -65,6 +65,10 @@ constexpr int kTabHead = 13 * kTabPitch;
 constexpr int kTileCols = 4;          // query columns of a tile
 constexpr int kHaloCols = kTileCols + KW - 1;   // 10 key columns per tile
 constexpr int kKG = kHaloCols / 2;    // 5 key groups of 16 keys (8 rows x 2 columns)
+#ifndef NAT_NWC
+#define NAT_NWC 14                    // consumer warps
+#define NAT_NT 2                      // 4-column tiles per consumer warp and step
+#endif
 
 // Counts bounded waits of this file's kernels that ran out.
 __device__ unsigned int g_stream_timeouts;
@@ -162,7 +166,7 @@ __device__ __forceinline__ void tmem_ld4(uint32_t taddr, float (&v)[4]) {
 // (the mma / ldmatrix fragment layout) across the warp.
 __device__ __forceinline__ uint32_t movm_t(uint32_t x) {
     uint32_t y;
-    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
+    asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
     return y;
 }
 
@@ -194,6 +198,21 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
     float r;
     asm("max.f32 %0, %1, %2, %3;\n" : "=f"(r) : "f"(a), "f"(b), "f"(c));
     return r;
+}
+
+// d = a * b + c on two fp32 lanes at once (packed f32x2 FMA).
+__device__ __forceinline__ void fma2(float &d0, float &d1, float a0, float a1, float b, float c0, float c1) {
+    asm("{\n .reg .b64 ra, rb, rc, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %4};\n mov.b64 rc, {%5, %6};\n"
+        " fma.rn.f32x2 rd, ra, rb, rc;\n mov.b64 {%0, %1}, rd;\n}\n"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b), "f"(c0), "f"(c1));
+}
+// (a0 * b0, a1 * b1) on two fp32 lanes at once.
+__device__ __forceinline__ void mul2(float &d0, float &d1, float a0, float a1, float b0, float b1) {
+    asm("{\n .reg .b64 ra, rb, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n"
+        " mul.rn.f32x2 rd, ra, rb;\n mov.b64 {%0, %1}, rd;\n}\n"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
 __device__ __forceinline__ int clampi(int x, int lo, int hi) { return x < lo ? lo : (x > hi ? hi : x); }
@@ -286,8 +305,24 @@ __device__ __forceinline__ void sb_expect_tx(uint32_t bar, uint32_t bytes) {
 // bank groups.
 __device__ __forceinline__ uint32_t row_base(int r, uint32_t pitch) { return (uint32_t)r * pitch + 16u * (r & 3); }
 
+// One P.V k-step of a tile: O^T += V^T P^T (channels 0-15 and 16-31) and the
+// row sums l += 1^T P^T; `first` starts the accumulators at zero.
+template <typename T>
+__device__ __forceinline__ void pv_step(float (&o)[2][4], float (&l)[4], const uint32_t (&v0)[4], const uint32_t (&v1)[4],
+                                        const uint32_t (&b)[2], const uint32_t (&ones)[4], bool first) {
+    if (first) {
+        Mma<T>::run0(o[0], v0, b[0], b[1]);
+        Mma<T>::run0(o[1], v1, b[0], b[1]);
+        Mma<T>::run0(l, ones, b[0], b[1]);
+    } else {
+        Mma<T>::run(o[0], v0, b[0], b[1]);
+        Mma<T>::run(o[1], v1, b[0], b[1]);
+        Mma<T>::run(l, ones, b[0], b[1]);
+    }
+}
+
 // ---------------------------------------------------------------------------
-// Two 8-query tiles (u = 0, 1) of one warp: S^T = K Q^T + bias, softmax,
+// NT 8-query tiles (u < NT) of one warp: S^T = K Q^T + bias, softmax,
 // O^T = V^T P^T, store.  Fragment roles, with g = lane / 4 and c = lane % 4:
 //   key group t (16 keys): key m < 8 is halo row m / 2, column 2t + m % 2;
 //     key m >= 8 is halo row 4 + (m - 8) / 2, column 2t + m % 2;
@@ -300,36 +335,60 @@ __device__ __forceinline__ uint32_t row_base(int r, uint32_t pitch) { return (ui
 //          chunk (lane / 8) % 2); channels 16-31 are + 32;
 //   tb: this warp's TMEM bias columns (tile u at + 32 u);
 //   out[u]: this lane's output pixel (query lane / 4 of tile u), or null.
+// All exponentials of the tiles are issued before their P.V products, so the
+// MUFU work of one warp forms one long independent run.
 // ---------------------------------------------------------------------------
-template <typename T>
-__device__ __forceinline__ void tile_pair(const uint32_t (&qa)[2], const uint32_t (&ka)[2], const uint32_t (&va)[2],
-                                          uint32_t tb, float c_log2, unsigned char *const (&out)[2], int lane) {
-    float s[2][kKG][4];
-    uint32_t qb[2][4];
+template <typename T, int NT, bool SHARED>
+__device__ __forceinline__ void tile_run(const uint32_t (&qa)[NT], const uint32_t (&ka)[NT], const uint32_t (&va)[NT],
+                                         uint32_t tb, float c_log2, unsigned char *const (&out)[NT], int lane) {
+    // SHARED (NT = 2, halo columns of tile 1 = those of tile 0 + 4): the two
+    // tiles' 14 halo columns are 7 key groups; tile 0 uses groups 0-4 and
+    // tile 1 groups 2-6, so each K / V fragment is loaded once for both.
+    static_assert(!SHARED || NT == 2, "shared key groups pair two adjacent tiles");
+    constexpr int NG = SHARED ? kKG + 2 : kKG;   // key groups loaded per tile set
+    float s[NT][kKG][4];
+    uint32_t qb[NT][4];
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
+    for (int u = 0; u < NT; ++u) {
         tmem_ld16(tb + 32u * u, *reinterpret_cast<float(*)[kKG][4]>(&s[u][0][0]));
         tmem_ld4(tb + 32u * u + 16u, s[u][4]);
     }
 #pragma unroll
-    for (int u = 0; u < 2; ++u) ldsm_x4(qb[u], qa[u]);
+    for (int u = 0; u < NT; ++u) ldsm_x4(qb[u], qa[u]);
     tmem_ld_wait();
     // ---- S^T = K Q^T + bias (C-init)
+    if constexpr (SHARED) {
 #pragma unroll
-    for (int t = 0; t < kKG; ++t)
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
+        for (int gi = 0; gi < NG; ++gi) {
             uint32_t k0[4], k1[4];
-            ldsm_x4(k0, ka[u] + 128u * t);
-            ldsm_x4(k1, ka[u] + 128u * t + 32u);
-            Mma<T>::run(s[u][t], k0, qb[u][0], qb[u][1]);
-            Mma<T>::run(s[u][t], k1, qb[u][2], qb[u][3]);
+            ldsm_x4(k0, ka[0] + 128u * gi);
+            ldsm_x4(k1, ka[0] + 128u * gi + 32u);
+            if (gi < kKG) {
+                Mma<T>::run(s[0][gi], k0, qb[0][0], qb[0][1]);
+                Mma<T>::run(s[0][gi], k1, qb[0][2], qb[0][3]);
+            }
+            if (gi >= 2) {
+                Mma<T>::run(s[1][gi - 2], k0, qb[1][0], qb[1][1]);
+                Mma<T>::run(s[1][gi - 2], k1, qb[1][2], qb[1][3]);
+            }
         }
+    } else {
+#pragma unroll
+        for (int t = 0; t < kKG; ++t)
+#pragma unroll
+            for (int u = 0; u < NT; ++u) {
+                uint32_t k0[4], k1[4];
+                ldsm_x4(k0, ka[u] + 128u * t);
+                ldsm_x4(k1, ka[u] + 128u * t + 32u);
+                Mma<T>::run(s[u][t], k0, qb[u][0], qb[u][1]);
+                Mma<T>::run(s[u][t], k1, qb[u][2], qb[u][3]);
+            }
+    }
     // ---- row max of queries 2c (m[u][0]) and 2c + 1 (m[u][1]): registers, then
     // the 8 lanes that hold the other keys of the same queries
-    float m[2][2];
+    float m[NT][2];
 #pragma unroll
-    for (int u = 0; u < 2; ++u)
+    for (int u = 0; u < NT; ++u)
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
             float x = max3(s[u][0][e], s[u][0][e + 2], s[u][1][e]);
@@ -341,32 +400,47 @@ __device__ __forceinline__ void tile_pair(const uint32_t (&qa)[2], const uint32_
 #pragma unroll
     for (int sh = 4; sh <= 16; sh <<= 1)
 #pragma unroll
-        for (int u = 0; u < 2; ++u)
+        for (int u = 0; u < NT; ++u)
 #pragma unroll
             for (int e = 0; e < 2; ++e) m[u][e] = fmaxf(m[u][e], __shfl_xor_sync(0xffffffffu, m[u][e], sh));
-    // ---- P = exp2((S - max) log2(e) / sqrt(D)), transposed into the B
-    // operand of O^T += V^T P^T; l += 1^T P^T gives the row sums
-    constexpr uint32_t ONE = OnesBits<T>::v;
-    const uint32_t ones[4] = {ONE, ONE, ONE, ONE};
-    float o[2][2][4], l[2][4];
+    // ---- P = exp2((S - max) log2(e) / sqrt(D)), packed and transposed into
+    // the B operands of the P.V k-steps
+    uint32_t bp[NT][kKG][2];
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
+    for (int u = 0; u < NT; ++u) {
         const float n0 = -m[u][0] * c_log2, n1 = -m[u][1] * c_log2;
 #pragma unroll
         for (int t = 0; t < kKG; ++t) {
-            const uint32_t b0 = movm_t(Exp2Pair<T>::run(fmaf(s[u][t][0], c_log2, n0), fmaf(s[u][t][1], c_log2, n1)));
-            const uint32_t b1 = movm_t(Exp2Pair<T>::run(fmaf(s[u][t][2], c_log2, n0), fmaf(s[u][t][3], c_log2, n1)));
+            float x0, x1, x2, x3;
+            fma2(x0, x1, s[u][t][0], s[u][t][1], c_log2, n0, n1);
+            fma2(x2, x3, s[u][t][2], s[u][t][3], c_log2, n0, n1);
+            bp[u][t][0] = movm_t(Exp2Pair<T>::run(x0, x1));
+            bp[u][t][1] = movm_t(Exp2Pair<T>::run(x2, x3));
+        }
+    }
+    // ---- O^T += V^T P^T; l += 1^T P^T gives the row sums
+    constexpr uint32_t ONE = OnesBits<T>::v;
+    const uint32_t ones[4] = {ONE, ONE, ONE, ONE};
+    float o[NT][2][4], l[NT][4];
+#pragma unroll
+    for (int gi = 0; gi < NG; ++gi) {
+        if constexpr (SHARED) {
             uint32_t v0[4], v1[4];
-            ldsm_x4_t(v0, va[u] + 128u * t);
-            ldsm_x4_t(v1, va[u] + 128u * t + 32u);
-            if (t == 0) {
-                Mma<T>::run0(o[u][0], v0, b0, b1);
-                Mma<T>::run0(o[u][1], v1, b0, b1);
-                Mma<T>::run0(l[u], ones, b0, b1);
-            } else {
-                Mma<T>::run(o[u][0], v0, b0, b1);
-                Mma<T>::run(o[u][1], v1, b0, b1);
-                Mma<T>::run(l[u], ones, b0, b1);
+            ldsm_x4_t(v0, va[0] + 128u * gi);
+            ldsm_x4_t(v1, va[0] + 128u * gi + 32u);
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int t = gi - 2 * u;
+                if (t < 0 || t >= kKG) continue;
+                pv_step<T>(o[u], l[u], v0, v1, bp[u][t], ones, t == 0);
+            }
+        } else {
+#pragma unroll
+            for (int u = 0; u < NT; ++u) {
+                uint32_t v0[4], v1[4];
+                ldsm_x4_t(v0, va[u] + 128u * gi);
+                ldsm_x4_t(v1, va[u] + 128u * gi + 32u);
+                pv_step<T>(o[u], l[u], v0, v1, bp[u][gi], ones, gi == 0);
             }
         }
     }
@@ -374,15 +448,18 @@ __device__ __forceinline__ void tile_pair(const uint32_t (&qa)[2], const uint32_
     // each 8-channel chunk) and store 4 bytes per chunk
     const uint32_t cofs = 4u * (uint32_t)(lane & 3);
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
+    for (int u = 0; u < NT; ++u) {
         float i0, i1;
         asm("rcp.approx.ftz.f32 %0, %1;\n" : "=f"(i0) : "f"(l[u][0]));
         asm("rcp.approx.ftz.f32 %0, %1;\n" : "=f"(i1) : "f"(l[u][1]));
         uint32_t y[4];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-            y[2 * h] = movm_t(Elem<T>::pack2(o[u][h][0] * i0, o[u][h][1] * i1));
-            y[2 * h + 1] = movm_t(Elem<T>::pack2(o[u][h][2] * i0, o[u][h][3] * i1));
+            float a0, a1, a2, a3;
+            mul2(a0, a1, o[u][h][0], o[u][h][1], i0, i1);
+            mul2(a2, a3, o[u][h][2], o[u][h][3], i0, i1);
+            y[2 * h] = movm_t(Elem<T>::pack2(a0, a1));
+            y[2 * h + 1] = movm_t(Elem<T>::pack2(a2, a3));
         }
         if (out[u]) {
 #pragma unroll
@@ -391,14 +468,23 @@ __device__ __forceinline__ void tile_pair(const uint32_t (&qa)[2], const uint32_
     }
 }
 
+// Named barrier among the consumer warps only (id 1; id 0 is __syncthreads).
+__device__ __forceinline__ void consumers_sync(int nthreads) {
+    asm volatile("bar.sync 1, %0;\n" ::"r"(nthreads) : "memory");
+}
+
 // ---------------------------------------------------------------------------
 // Kernel.  Warps 0 .. NWC-1 consume; warp NWC produces (one thread issues one
 // bulk copy per image row).  Each consumer warp owns a fixed position in
-// every step: pair warp / MX of the step and the 8 query columns starting at
-// 8 (warp % MX), as two 4-column tiles, so its column geometry is set up once.
+// every step: pair warp / MX of the step and the 4 NT query columns starting
+// at 4 NT (warp % MX), as NT 4-column tiles, so its column geometry (halo
+// columns, the column part of its window masks and bias-table columns) is set
+// up once.  The producer starts copying right after the barriers are set up;
+// the consumers build the bias table and allocate tensor memory meanwhile.
 // ---------------------------------------------------------------------------
-template <typename T, int NWC>
+template <typename T, int NWC, int NT>
 __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __grid_constant__ StreamParams p) {
+    static_assert(32 * NT * ((NWC + 3) / 4) <= kTmemCols, "bias columns of all consumer warps fit in TMEM");
     extern __shared__ __align__(1024) unsigned char smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // this CTA's range of query-row pairs (the CTAs' loads differ by at most one pair)
@@ -416,35 +502,22 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
     float *tab = reinterpret_cast<float *>(smem + p.off_tab + 64);
     const uint32_t pitch = (uint32_t)(p.W + 1) * kPixB;   // row pitch in bytes
 
-    // ---- prologue: build the bias table; init the barriers; allocate TMEM.
-    {
-        grid_dep_wait();   // first global read: the bias table
-        const T *rpb = reinterpret_cast<const T *>(p.rpb);
-        for (int i = threadIdx.x; i < p.heads * kTabHead; i += blockDim.x) {
-            const int h = i / kTabHead, a = (i / kTabPitch) % 13, b = i % kTabPitch;
-            float v = 0.f;
-            if (rpb && b < 13) v = Elem<T>::to_f(rpb[(h * 13 + a) * 13 + b]) * p.sqrt_d;
-            tab[i] = v;
+    if (threadIdx.x == NWC * 32) {
+        for (int i = 0; i < NS; ++i) {
+            sb_init(bar_full + 8 * i, 1);     // one expect_tx arrival per step
+            sb_init(bar_empty + 8 * i, NWC);
         }
-        if (threadIdx.x == 0) {
-            for (int i = 0; i < NS; ++i) {
-                sb_init(bar_full + 8 * i, 1);     // one expect_tx arrival per step
-                sb_init(bar_empty + 8 * i, NWC);
-            }
-            *abort_flag = 0;
-            asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-        }
-        if (warp == 0) tmem_alloc(smem_u32(tmem_slot));
-        tmem_fence_before();
-        __syncthreads();
-        tmem_fence_after();
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     }
+    __syncthreads();
 
     if (warp == NWC) {
         // =================== producer ===================
         // one thread issues one bulk copy per image row: the step's new K and
         // V rows into the ring, its query rows into the stage
         if (lane == 0) {
+            grid_dep_wait();   // no global read before the previous kernel completes
             const uint32_t rowbytes = (uint32_t)p.W * kPixB;
             SlideWalk w;
             w.init(p, s_begin, s_end);
@@ -486,25 +559,61 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
         }
     } else {
         // =================== consumers ===================
+        // prologue (overlaps the first copies): bias table, tensor memory
+        {
+            grid_dep_wait();   // first global read: the bias table
+            const T *rpb = reinterpret_cast<const T *>(p.rpb);
+            for (int i = threadIdx.x; i < p.heads * kTabHead; i += NWC * 32) {
+                const int h = i / kTabHead, a = (i / kTabPitch) % 13, b = i % kTabPitch;
+                float v = 0.f;
+                if (rpb && b < 13) v = Elem<T>::to_f(rpb[(h * 13 + a) * 13 + b]) * p.sqrt_d;
+                tab[i] = v;
+            }
+            if (warp == 0) tmem_alloc(smem_u32(tmem_slot));
+            tmem_fence_before();
+            consumers_sync(NWC * 32);
+            tmem_fence_after();
+        }
         const int H = p.H, W = p.W;
         const int g = lane >> 2, c = lane & 3;
         // this warp's TMEM bias columns: lane quarter warp % 4, column slot warp / 4
-        const uint32_t tb = *tmem_slot + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(64 * (warp >> 2));
-        // fixed per warp: its pair within the step and its two 4-column tiles
-        const int pw = warp / p.MX, x0 = 8 * (warp - pw * p.MX);
+        const uint32_t tb = *tmem_slot + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(32 * NT * (warp >> 2));
+        // fixed per warp: its pair within the step and its NT 4-column tiles
+        const int pw = warp / p.MX, x0 = kTileCols * NT * (warp - pw * p.MX);
         const bool active = warp < p.SP * p.MX;
         const int mk = lane & 15, mv = (lane & 7) + ((lane >> 4) << 3);
         const int krow = ((mk >> 3) << 2) + ((mk & 7) >> 1), vrow = ((mv >> 3) << 2) + ((mv & 7) >> 1);
-        int xq[2], hx[2];
-        uint32_t qcol[2], kcol[2], vcol[2];
+        uint32_t qcol[NT], kcol[NT], vcol[NT];
+        int xq[NT];
+        // bias rewrite, column part: table column of key group 0 for this lane's
+        // two queries (jlo = 0, 1), and which of the 10 (t, jlo) keys lie in
+        // the query's window along x
+        int cb[NT][2];
+        uint32_t xin[NT];
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
+        for (int u = 0; u < NT; ++u) {
             xq[u] = x0 + kTileCols * u;
-            hx[u] = tile_halo(xq[u], W);
+            const int hx = tile_halo(xq[u], W);
             qcol[u] = (uint32_t)min(xq[u] + (lane & 3), W - 1) * kPixB + 16u * (uint32_t)(lane >> 3);
-            kcol[u] = (uint32_t)(hx[u] + (mk & 1)) * kPixB + 16u * (uint32_t)(lane >> 4);
-            vcol[u] = (uint32_t)(hx[u] + (mv & 1)) * kPixB + 16u * (uint32_t)((lane >> 3) & 1);
+            kcol[u] = (uint32_t)(hx + (mk & 1)) * kPixB + 16u * (uint32_t)(lane >> 4);
+            vcol[u] = (uint32_t)(hx + (mv & 1)) * kPixB + 16u * (uint32_t)((lane >> 3) & 1);
+            xin[u] = 0;
+#pragma unroll
+            for (int jlo = 0; jlo < 2; ++jlo) {
+                const int qx = min(xq[u] + 2 * (c & 1) + jlo, W - 1), sx = win_start(qx, W);
+                // kx - qx + 6 for key column kx = hx + 2t + (g & 1): within
+                // [-3, 15], inside the padded table
+                cb[u][jlo] = hx + (g & 1) - qx + 6;
+#pragma unroll
+                for (int t = 0; t < kKG; ++t) {
+                    const int kx = hx + 2 * t + (g & 1);
+                    xin[u] |= ((unsigned)(kx - sx) < (unsigned)KW ? 1u : 0u) << (2 * t + jlo);
+                }
+            }
         }
+        // the two tiles' halos are 4 columns apart (away from the image's
+        // left and right edges): their key groups can be shared
+        const bool shared_cols = NT == 2 && tile_halo(xq[NT - 1], W) == tile_halo(xq[0], W) + kTileCols;
         const int qsel = (lane >> 2) & 1;
         // output pixel of this lane's epilogue query (lane / 4): tile row g / 4, column g % 4
         const int orow = g >> 2, ocol0 = g & 3;
@@ -526,29 +635,28 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
                 const int key = ((w.h * 8 + (qy0 - hy)) * 2 + (qy1 - qy0)) * 4 + (sy0 - hy) * 2 + (sy1 - hy);
                 if (key != bias_key) {
                     bias_key = key;
-                    const float *th = tab + w.h * kTabHead;
-                    // this lane's queries 2c, 2c + 1 share tile row c / 2
+                    // this lane's queries 2c, 2c + 1 share tile row c / 2; its
+                    // keys lie on halo rows g / 2 (j < 2) and 4 + g / 2 (j >= 2)
                     const int qy = (c >> 1) ? qy1 : qy0, sy = (c >> 1) ? sy1 : sy0;
+                    const float *rows[2];
+                    bool yin[2];
 #pragma unroll
-                    for (int u = 0; u < 2; ++u) {
+                    for (int jh = 0; jh < 2; ++jh) {
+                        const int ky = hy + 4 * jh + (g >> 1);
+                        yin[jh] = (unsigned)(ky - sy) < (unsigned)KW;
+                        rows[jh] = tab + w.h * kTabHead + clampi(ky - qy + 6, 0, 12) * kTabPitch;
+                    }
+#pragma unroll
+                    for (int u = 0; u < NT; ++u) {
                         float b[kKG][4];
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const int ky = hy + 4 * (j >> 1) + (g >> 1);
-                            const bool yin = (unsigned)(ky - sy) < (unsigned)KW;
-                            const int qx = min(xq[u] + 2 * (c & 1) + (j & 1), W - 1), sx = win_start(qx, W);
-                            // table row of this key row; the column offsets
-                            // kx - qx + 6 stay within [-3, 15], inside the
-                            // padded table, so the loads need no clamp
-                            const float *row = th + clampi(ky - qy + 6, 0, 12) * kTabPitch - qx + 6;
+                        for (int t = 0; t < kKG; ++t)
 #pragma unroll
-                            for (int t = 0; t < kKG; ++t) {
-                                const int kx = hx[u] + 2 * t + (g & 1);
-                                const bool in = yin && (unsigned)(kx - sx) < (unsigned)KW;
-                                const float v = row[kx];
+                            for (int j = 0; j < 4; ++j) {
+                                const float v = rows[j >> 1][cb[u][j & 1] + 2 * t];
+                                const bool in = yin[j >> 1] && ((xin[u] >> (2 * t + (j & 1))) & 1u);
                                 b[t][j] = in ? v : kMaskC;
                             }
-                        }
 #pragma unroll
                         for (int t = 0; t < kKG; ++t) tmem_st4(tb + 32u * u + 4u * t, b[t]);
                     }
@@ -567,19 +675,22 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
                 const uint32_t qrow = sbase + row_base(stage * 2 * p.SP + (qsel ? qy1 : qy0) - 2 * w.pa, pitch);
                 const uint32_t krb = sbase + p.off_k + row_base(w.ring(p, hy + krow), pitch);
                 const uint32_t vrb = sbase + p.off_v + row_base(w.ring(p, hy + vrow), pitch);
-                const uint32_t qa[2] = {qrow + qcol[0], qrow + qcol[1]};
-                const uint32_t ka[2] = {krb + kcol[0], krb + kcol[1]};
-                const uint32_t va[2] = {vrb + vcol[0], vrb + vcol[1]};
-                unsigned char *o[2] = {nullptr, nullptr};
+                uint32_t qa[NT], ka[NT], va[NT];
+                unsigned char *o[NT];
                 const int oy = orow ? qy0 + 1 : qy0;
-                if (oy < H) {
+                unsigned char *orow_ptr = p.out + ((size_t)w.bh * H + oy) * W * kPixB;
 #pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int ox = xq[u] + ocol0;
-                        if (ox < W) o[u] = p.out + (((size_t)w.bh * H + oy) * W + ox) * kPixB;
-                    }
+                for (int u = 0; u < NT; ++u) {
+                    qa[u] = qrow + qcol[u];
+                    ka[u] = krb + kcol[u];
+                    va[u] = vrb + vcol[u];
+                    const int ox = xq[u] + ocol0;
+                    o[u] = (oy < H && ox < W) ? orow_ptr + (size_t)ox * kPixB : nullptr;
                 }
-                tile_pair<T>(qa, ka, va, tb, p.c_log2, o, lane);
+                if (NT == 2 && shared_cols)
+                    tile_run<T, NT, NT == 2>(qa, ka, va, tb, p.c_log2, o, lane);
+                else
+                    tile_run<T, NT, false>(qa, ka, va, tb, p.c_log2, o, lane);
             }
             __syncwarp();
             if (lane == 0) sb_arrive(bar_empty + 8 * stage);
@@ -633,7 +744,7 @@ cudaError_t stream_device(int *sms, int *smem_cap, const void *kern) {
 
 uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
-template <typename T, int NWC>
+template <typename T, int NWC, int NT>
 cudaError_t launch_stream_t(const StreamParams &sp, uint32_t smem, int grid, cudaStream_t st, bool *launched) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
@@ -645,15 +756,15 @@ cudaError_t launch_stream_t(const StreamParams &sp, uint32_t smem, int grid, cud
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, fwd_stream_kernel<T, NWC>, sp);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, fwd_stream_kernel<T, NWC, NT>, sp);
     *launched = true;
     note_kernel("fwd_stream_kernel");
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 // Plan for SP query-row pairs per step; returns the shared-memory bytes.
-uint32_t plan_slide(StreamParams &sp, const Problem &pr, int SP) {
-    sp.MX = (pr.W + 7) / 8;
+uint32_t plan_slide(StreamParams &sp, const Problem &pr, int SP, int span) {
+    sp.MX = (pr.W + span - 1) / span;
     sp.SP = SP;
     sp.NP = (pr.H + 1) / 2;
     const int spi = (sp.NP + sp.SP - 1) / sp.SP;   // steps per image
@@ -672,15 +783,16 @@ uint32_t plan_slide(StreamParams &sp, const Problem &pr, int SP) {
     return sp.off_bar + 16 * NS + 16;
 }
 
-template <typename T, int NWC>
+template <typename T, int NWC, int NT>
 cudaError_t launch_slide(StreamParams &sp, const Problem &pr, cudaStream_t st, bool *launched) {
-    const void *kern = reinterpret_cast<const void *>(&fwd_stream_kernel<T, NWC>);
+    const void *kern = reinterpret_cast<const void *>(&fwd_stream_kernel<T, NWC, NT>);
     int sms = 0, cap = 0;
     cudaError_t e = stream_device(&sms, &cap, kern);
     if (e != cudaSuccess) return e;
-    const int MX = (pr.W + 7) / 8;
+    const int span = kTileCols * NT;   // query columns per consumer warp
+    const int MX = (pr.W + span - 1) / span;
     for (int SP = std::max(1, NWC / MX); SP >= 1; --SP) {
-        const uint32_t smem = plan_slide(sp, pr, SP);
+        const uint32_t smem = plan_slide(sp, pr, SP, span);
         if ((int)smem > cap) continue;
         const int64_t npairs = pr.bh() * sp.NP;
         if (npairs >= INT32_MAX || npairs <= 0) return cudaSuccess;
@@ -697,7 +809,7 @@ cudaError_t launch_slide(StreamParams &sp, const Problem &pr, cudaStream_t st, b
             const int64_t aligned = (sp.NP + c - 1) / c, even = (npairs + sms - 1) / sms;
             if (aligned <= even + 1) grid = (int)(images * c);
         }
-        return launch_stream_t<T, NWC>(sp, smem, grid, st, launched);
+        return launch_stream_t<T, NWC, NT>(sp, smem, grid, st, launched);
     }
     return cudaSuccess;
 }
@@ -714,9 +826,9 @@ cudaError_t launch_stream_impl(const Problem &pr, const void *q, const void *k, 
     sp.H = pr.H; sp.W = pr.W; sp.heads = pr.heads;
     sp.c_log2 = kLog2e / std::sqrt((float)pr.D);
     sp.sqrt_d = std::sqrt((float)pr.D);
-    // 14 consumer warps (SP query-row pairs of MX 8-column spans each) and a
-    // producer warp
-    return launch_slide<T, 14>(sp, pr, st, launched);
+    // NAT_NWC consumer warps (SP query-row pairs of MX column spans each)
+    // and a producer warp
+    return launch_slide<T, NAT_NWC, NAT_NT>(sp, pr, st, launched);
 }
 
 }  // namespace
