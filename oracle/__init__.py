@@ -93,8 +93,14 @@ class Oracle:
         lib.oracle_na2d_av.argtypes = [i] * 7 + [_DP, _DP, _DP, i]
         lib.oracle_na2d_forward.argtypes = [i] * 7 + [_DP, _DP, _DP, _DP, _DP, i]
         lib.oracle_na2d_backward.argtypes = [i] * 7 + [_DP] * 9 + [i]
+        u64, f64 = ctypes.c_ulonglong, ctypes.c_double
+        lib.oracle_na2d_forward_ex.argtypes = [i] * 7 + [_DP] * 6 + [f64, u64, u64]
+        lib.oracle_na2d_backward_ex.argtypes = [i] * 7 + [_DP] * 9 + [f64, u64, u64]
+        lib.oracle_philox4x32_10.argtypes = [ctypes.POINTER(ctypes.c_uint)] * 3
+        lib.oracle_philox4x32_10.restype = None
         for f in ("oracle_axis_window", "oracle_axis_neighbors", "oracle_na2d_qk_rpb",
-                  "oracle_na2d_softmax", "oracle_na2d_av", "oracle_na2d_forward", "oracle_na2d_backward"):
+                  "oracle_na2d_softmax", "oracle_na2d_av", "oracle_na2d_forward", "oracle_na2d_backward",
+                  "oracle_na2d_forward_ex", "oracle_na2d_backward_ex"):
             getattr(lib, f).restype = ctypes.c_int
         self._lib = lib
 
@@ -167,6 +173,63 @@ class Oracle:
                "backward")
         return dq, dk, dv, drpb
 
+    # -- dropout, returned weights --------------------------------------------
+    def philox(self, ctr, key) -> list[int]:
+        """Philox4x32-10 of a 4-word counter and 2-word key (SC 2011 definition)."""
+        c = (ctypes.c_uint * 4)(*ctr)
+        kk = (ctypes.c_uint * 2)(*key)
+        o = (ctypes.c_uint * 4)()
+        self._lib.oracle_philox4x32_10(c, kk, o)
+        return list(o)
+
+    def forward_ex(self, q, k, v, rpb, kernel_size: int, dilation: int, dropout_p: float = 0.0, seed: int = 0,
+                   offset: int = 0, return_attn: bool = False):
+        """Forward with attention dropout (Philox mask) and, optionally, the
+        weights after dropout [B, heads, H, W, k*k]."""
+        q, k, v = _f64(q), _f64(k), _f64(v)
+        rpb = None if rpb is None else _f64(rpb)
+        shp = _shape(q, kernel_size, dilation)
+        out = np.empty(q.shape, dtype=np.float64)
+        attn = np.empty(q.shape[:4] + (kernel_size * kernel_size,), dtype=np.float64) if return_attn else None
+        _check(self._lib.oracle_na2d_forward_ex(*shp, _ptr(q), _ptr(k), _ptr(v), _ptr(rpb), _ptr(out), _ptr(attn),
+                                                float(np.float32(dropout_p)), seed, offset), "forward_ex")
+        return (out, attn) if return_attn else out
+
+    def backward_ex(self, q, k, v, rpb, dout, kernel_size: int, dilation: int, dropout_p: float = 0.0,
+                    seed: int = 0, offset: int = 0):
+        """Gradients of forward_ex with the same dropout mask."""
+        q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+        rpb = None if rpb is None else _f64(rpb)
+        shp = _shape(q, kernel_size, dilation)
+        dq, dk, dv = (np.empty(q.shape, dtype=np.float64) for _ in range(3))
+        nb = 2 * kernel_size - 1
+        drpb = np.empty((q.shape[1], nb, nb), dtype=np.float64)
+        _check(self._lib.oracle_na2d_backward_ex(*shp, _ptr(q), _ptr(k), _ptr(v), _ptr(rpb), _ptr(dout), _ptr(dq),
+                                                 _ptr(dk), _ptr(dv), _ptr(drpb), float(np.float32(dropout_p)), seed,
+                                                 offset), "backward_ex")
+        return dq, dk, dv, drpb
+
+    # -- maps shorter than k * d ------------------------------------------------
+    def forward_padded(self, q, k, v, rpb, kernel_size: int, dilation: int):
+        """The layer's padding (HF DiNAT maybe_pad, gitcode DiNAT article's
+        layer walkthrough): pad the map with zero pixels at the bottom/right
+        up to kernel_size * dilation, attend, crop back to H x W."""
+        H, W = q.shape[2], q.shape[3]
+        pads = ((0, 0), (0, 0), (0, max(0, kernel_size * dilation - H)), (0, max(0, kernel_size * dilation - W)),
+                (0, 0))
+        Q, K, V = (np.pad(_f64(t), pads) for t in (q, k, v))
+        return self.forward(Q, K, V, rpb, kernel_size, dilation)[:, :, :H, :W]
+
+    def backward_padded(self, q, k, v, rpb, dout, kernel_size: int, dilation: int):
+        """Gradients of forward_padded: the padded pixels' outputs are cropped
+        (zero output gradient there) and their input gradients dropped."""
+        H, W = q.shape[2], q.shape[3]
+        pads = ((0, 0), (0, 0), (0, max(0, kernel_size * dilation - H)), (0, max(0, kernel_size * dilation - W)),
+                (0, 0))
+        Q, K, V, G = (np.pad(_f64(t), pads) for t in (q, k, v, dout))
+        dq, dk, dv, drpb = self.backward(Q, K, V, rpb, G, kernel_size, dilation)
+        return dq[:, :, :H, :W], dk[:, :, :H, :W], dv[:, :, :H, :W], drpb
+
     def forward_query(self, q, k, v, rpb, kernel_size: int, dilation: int,
                       b: int, h: int, i: int, j: int) -> np.ndarray:
         """One output row from the definition, with numpy on the window that
@@ -226,3 +289,23 @@ def forward_query(q, k, v, rpb, kernel_size, dilation, b, h, i, j):
 
 def backward(q, k, v, rpb, dout, kernel_size, dilation, nthreads=None):
     return get().backward(q, k, v, rpb, dout, kernel_size, dilation, nthreads)
+
+
+def philox(ctr, key):
+    return get().philox(ctr, key)
+
+
+def forward_ex(q, k, v, rpb, kernel_size, dilation, dropout_p=0.0, seed=0, offset=0, return_attn=False):
+    return get().forward_ex(q, k, v, rpb, kernel_size, dilation, dropout_p, seed, offset, return_attn)
+
+
+def backward_ex(q, k, v, rpb, dout, kernel_size, dilation, dropout_p=0.0, seed=0, offset=0):
+    return get().backward_ex(q, k, v, rpb, dout, kernel_size, dilation, dropout_p, seed, offset)
+
+
+def forward_padded(q, k, v, rpb, kernel_size, dilation):
+    return get().forward_padded(q, k, v, rpb, kernel_size, dilation)
+
+
+def backward_padded(q, k, v, rpb, dout, kernel_size, dilation):
+    return get().backward_padded(q, k, v, rpb, dout, kernel_size, dilation)

@@ -491,3 +491,222 @@ int oracle_na2d_backward(int B, int heads, int H, int W, int D, int k, int d,
     free(jobs);
     return 0;
 }
+
+/* ---------------------------------------------------------------------------
+ * Attention dropout and the returned attention weights.
+ *
+ * The layer applies dropout to the attention weights between the softmax and
+ * natten2dav (gitcode DiNAT article, section "DiNAT 的核心思想"), and with
+ * output_attentions returns those weights ("Dilated Neighborhood Attention
+ * Transformer", HF docs, DinatModel outputs, `attentions`).  Dropout keeps a
+ * weight with probability 1 - p and scales kept weights by 1 / (1 - p).
+ *
+ * The random draw is a counter-based generator so that the GPU and this
+ * oracle draw the same mask: Philox4x32-10 from its publication (Salmon,
+ * Moraes, Dror, Shaw, "Parallel Random Numbers: As Easy as 1, 2, 3", SC 2011):
+ * ten rounds; a round multiplies counter words 0 and 2 by 0xD2511F53 and
+ * 0xCD9E8D57 into 64-bit products and forms (hi(c2*M1) ^ c1 ^ k0, lo(c2*M1),
+ * hi(c0*M0) ^ c3 ^ k1, lo(c0*M0)); the key is bumped by (0x9E3779B9,
+ * 0xBB67AE85) before every round but the first.
+ * Weight e (its linear index in [B, heads, H, W, k*k]) is kept when word
+ * e mod 4 of Philox(counter = (e/4 low 32 bits, e/4 high 32, offset low,
+ * offset high), key = (seed low, seed high)) is >= round(p * 2^32).
+ * ------------------------------------------------------------------------- */
+void oracle_philox4x32_10(const unsigned int ctr[4], const unsigned int key[2], unsigned int out[4])
+{
+    unsigned int c0 = ctr[0], c1 = ctr[1], c2 = ctr[2], c3 = ctr[3];
+    unsigned int k0 = key[0], k1 = key[1];
+    for (int round = 0; round < 10; ++round) {
+        if (round > 0) {
+            k0 += 0x9E3779B9u;
+            k1 += 0xBB67AE85u;
+        }
+        unsigned long long prod0 = (unsigned long long)0xD2511F53u * c0;
+        unsigned long long prod1 = (unsigned long long)0xCD9E8D57u * c2;
+        unsigned int n0 = (unsigned int)(prod1 >> 32) ^ c1 ^ k0;
+        unsigned int n1 = (unsigned int)prod1;
+        unsigned int n2 = (unsigned int)(prod0 >> 32) ^ c3 ^ k1;
+        unsigned int n3 = (unsigned int)prod0;
+        c0 = n0; c1 = n1; c2 = n2; c3 = n3;
+    }
+    out[0] = c0; out[1] = c1; out[2] = c2; out[3] = c3;
+}
+
+static unsigned int drop_threshold(double p)
+{
+    double t = p * 4294967296.0;
+    if (t >= 4294967295.0) return 0xFFFFFFFFu;
+    return (unsigned int)(t + 0.5);
+}
+
+/* dropout factor of weight e: 0 (dropped) or 1 / (1 - p) (kept) */
+static double drop_factor(unsigned long long e, double p, unsigned long long seed, unsigned long long offset)
+{
+    if (p <= 0.0) return 1.0;
+    unsigned long long blk = e >> 2;
+    unsigned int ctr[4] = {(unsigned int)blk, (unsigned int)(blk >> 32), (unsigned int)offset,
+                           (unsigned int)(offset >> 32)};
+    unsigned int key[2] = {(unsigned int)seed, (unsigned int)(seed >> 32)};
+    unsigned int w[4];
+    oracle_philox4x32_10(ctr, key, w);
+    return w[e & 3] >= drop_threshold(p) ? 1.0 / (1.0 - p) : 0.0;
+}
+
+/* Fused definition with dropout and the weights written out: as
+ * forward_slice, then p_n <- factor_n p_n, attn[.., n] = p_n (if attn), and
+ * out = sum_n p_n v_n. */
+static void forward_ex_slice(const oracle_shape *p, int bh, const double *q, const double *kk, const double *v,
+                             const double *rpb, double *out, double *attn, double dp, unsigned long long seed,
+                             unsigned long long offset)
+{
+    const int H = p->H, W = p->W, D = p->D, k = p->k, d = p->d;
+    const int h = bh % p->heads;
+    const int nb = 2 * k - 1;
+    const double scale = 1.0 / sqrt((double)D);
+    const size_t base = (size_t)bh * H * W * D;
+    int *ky = malloc(sizeof(int) * k), *by = malloc(sizeof(int) * k);
+    int *kx = malloc(sizeof(int) * k), *bx = malloc(sizeof(int) * k);
+    double *sc = malloc(sizeof(double) * k * k);
+    for (int i = 0; i < H; ++i) {
+        oracle_axis_neighbors(H, k, d, i, ky, by);
+        for (int j = 0; j < W; ++j) {
+            oracle_axis_neighbors(W, k, d, j, kx, bx);
+            const double *qv = q + base + ((size_t)i * W + j) * D;
+            for (int ty = 0; ty < k; ++ty)
+                for (int tx = 0; tx < k; ++tx) {
+                    const double *kv = kk + base + ((size_t)ky[ty] * W + kx[tx]) * D;
+                    double dot = 0.0;
+                    for (int c = 0; c < D; ++c) dot += qv[c] * kv[c];
+                    double bias = 0.0;
+                    if (rpb) bias = rpb[((size_t)h * nb + by[ty]) * nb + bx[tx]];
+                    sc[ty * k + tx] = dot * scale + bias;
+                }
+            double m = sc[0];
+            for (int t = 1; t < k * k; ++t)
+                if (sc[t] > m) m = sc[t];
+            double sum = 0.0;
+            for (int t = 0; t < k * k; ++t) {
+                sc[t] = exp(sc[t] - m);
+                sum += sc[t];
+            }
+            const unsigned long long row = ((unsigned long long)bh * H + i) * W + j;
+            for (int t = 0; t < k * k; ++t) {
+                sc[t] = sc[t] / sum * drop_factor(row * (unsigned long long)(k * k) + t, dp, seed, offset);
+                if (attn) attn[row * (size_t)(k * k) + t] = sc[t];
+            }
+            double *o = out + base + ((size_t)i * W + j) * D;
+            for (int c = 0; c < D; ++c) o[c] = 0.0;
+            for (int ty = 0; ty < k; ++ty)
+                for (int tx = 0; tx < k; ++tx) {
+                    const double *vv = v + base + ((size_t)ky[ty] * W + kx[tx]) * D;
+                    for (int c = 0; c < D; ++c) o[c] += sc[ty * k + tx] * vv[c];
+                }
+        }
+    }
+    free(ky); free(by); free(kx); free(bx); free(sc);
+}
+
+/* Backward with dropout: out = sum_n f_n p_n v_n with dropout factors f_n.
+ *     dL/dv_n += f_n p_n g,   dL/dp_n = f_n (g . v_n),
+ *     dL/ds_n = p_n (dL/dp_n - sum_m p_m dL/dp_m), then as backward_slice. */
+static void backward_ex_slice(const oracle_shape *p, int bh, const double *q, const double *kk, const double *v,
+                              const double *rpb, const double *dout, double *dq, double *dk, double *dv,
+                              double *drpb_acc, double dp_, unsigned long long seed, unsigned long long offset)
+{
+    const int H = p->H, W = p->W, D = p->D, k = p->k, d = p->d;
+    const int h = bh % p->heads;
+    const int nb = 2 * k - 1;
+    const double scale = 1.0 / sqrt((double)D);
+    const size_t base = (size_t)bh * H * W * D;
+    int *ky = malloc(sizeof(int) * k), *by = malloc(sizeof(int) * k);
+    int *kx = malloc(sizeof(int) * k), *bx = malloc(sizeof(int) * k);
+    double *sc = malloc(sizeof(double) * k * k), *dp = malloc(sizeof(double) * k * k);
+    double *f = malloc(sizeof(double) * k * k);
+    for (size_t e = 0; e < (size_t)H * W * D; ++e) {
+        dq[base + e] = 0.0;
+        dk[base + e] = 0.0;
+        dv[base + e] = 0.0;
+    }
+    for (int i = 0; i < H; ++i) {
+        oracle_axis_neighbors(H, k, d, i, ky, by);
+        for (int j = 0; j < W; ++j) {
+            oracle_axis_neighbors(W, k, d, j, kx, bx);
+            const double *qv = q + base + ((size_t)i * W + j) * D;
+            const double *g = dout + base + ((size_t)i * W + j) * D;
+            for (int ty = 0; ty < k; ++ty)
+                for (int tx = 0; tx < k; ++tx) {
+                    const double *kv = kk + base + ((size_t)ky[ty] * W + kx[tx]) * D;
+                    double dot = 0.0;
+                    for (int c = 0; c < D; ++c) dot += qv[c] * kv[c];
+                    double bias = 0.0;
+                    if (rpb) bias = rpb[((size_t)h * nb + by[ty]) * nb + bx[tx]];
+                    sc[ty * k + tx] = dot * scale + bias;
+                }
+            double m = sc[0];
+            for (int t = 1; t < k * k; ++t)
+                if (sc[t] > m) m = sc[t];
+            double sum = 0.0;
+            for (int t = 0; t < k * k; ++t) {
+                sc[t] = exp(sc[t] - m);
+                sum += sc[t];
+            }
+            const unsigned long long row = ((unsigned long long)bh * H + i) * W + j;
+            for (int t = 0; t < k * k; ++t) {
+                sc[t] /= sum;
+                f[t] = drop_factor(row * (unsigned long long)(k * k) + t, dp_, seed, offset);
+            }
+            double pdp = 0.0;
+            for (int ty = 0; ty < k; ++ty)
+                for (int tx = 0; tx < k; ++tx) {
+                    const double *vv = v + base + ((size_t)ky[ty] * W + kx[tx]) * D;
+                    double dot = 0.0;
+                    for (int c = 0; c < D; ++c) dot += g[c] * vv[c];
+                    dp[ty * k + tx] = f[ty * k + tx] * dot;
+                    pdp += sc[ty * k + tx] * dp[ty * k + tx];
+                }
+            double *dqv = dq + base + ((size_t)i * W + j) * D;
+            for (int ty = 0; ty < k; ++ty)
+                for (int tx = 0; tx < k; ++tx) {
+                    const int n = ty * k + tx;
+                    const size_t key = base + ((size_t)ky[ty] * W + kx[tx]) * D;
+                    const double ds = sc[n] * (dp[n] - pdp);
+                    for (int c = 0; c < D; ++c) {
+                        dv[key + c] += f[n] * sc[n] * g[c];
+                        dqv[c] += ds * kk[key + c] * scale;
+                        dk[key + c] += ds * qv[c] * scale;
+                    }
+                    drpb_acc[((size_t)h * nb + by[ty]) * nb + bx[tx]] += ds;
+                }
+        }
+    }
+    free(ky); free(by); free(kx); free(bx); free(sc); free(dp); free(f);
+}
+
+/* Forward with optional weights output (attn, may be NULL) and dropout
+ * probability dp (0: none); single-threaded per call, slices in order. */
+int oracle_na2d_forward_ex(int B, int heads, int H, int W, int D, int k, int d, const double *q,
+                           const double *kk, const double *v, const double *rpb, double *out, double *attn,
+                           double dp, unsigned long long seed, unsigned long long offset)
+{
+    oracle_shape p = make_shape(B, heads, H, W, D, k, d);
+    if (!shape_ok(&p)) return -1;
+    for (int bh = 0; bh < B * heads; ++bh) forward_ex_slice(&p, bh, q, kk, v, rpb, out, attn, dp, seed, offset);
+    return 0;
+}
+
+int oracle_na2d_backward_ex(int B, int heads, int H, int W, int D, int k, int d, const double *q,
+                            const double *kk, const double *v, const double *rpb, const double *dout, double *dq,
+                            double *dk, double *dv, double *drpb, double dp, unsigned long long seed,
+                            unsigned long long offset)
+{
+    oracle_shape p = make_shape(B, heads, H, W, D, k, d);
+    if (!shape_ok(&p)) return -1;
+    const size_t ntab = (size_t)heads * (2 * k - 1) * (2 * k - 1);
+    double *acc = calloc(ntab ? ntab : 1, sizeof(double));
+    for (int bh = 0; bh < B * heads; ++bh)
+        backward_ex_slice(&p, bh, q, kk, v, rpb, dout, dq, dk, dv, acc, dp, seed, offset);
+    if (drpb)
+        for (size_t e = 0; e < ntab; ++e) drpb[e] = acc[e];
+    free(acc);
+    return 0;
+}

@@ -26,7 +26,19 @@ What fixes each expected value (never the oracle's own formula retyped):
     fp64 when the window covers the image; calculus identities (softmax
     gradients sum to zero, so every head's bias gradient sums to zero; the
     weights sum to one, so the value gradients sum to the output gradients);
-    the dilation decomposition carried over to the gradients.
+    the dilation decomposition carried over to the gradients;
+  * dropout: the generator's published known-answer values
+    (tests/golden/philox4x32_10_kat.txt); p = 0 equals the plain forward; kept
+    weights equal the (pinned) softmax weights / (1 - p) and dropped ones are
+    zero, at the positions an independent Python restatement of the generator
+    selects; the returned weights reproduce the output through the pinned
+    weighted-sum stage; the keep rate is 1 - p within 5 sigma; the backward
+    equals finite differences of the forward with the mask fixed;
+  * maps shorter than k * d (zero padding, then crop): unchanged when no
+    padding is needed; dense attention over the zero-padded map when the
+    padded window covers it; with q = 0 and no bias, the mean of v over the
+    searched window counting padded pixels as zeros; the backward equals
+    finite differences.
 """
 from __future__ import annotations
 
@@ -384,7 +396,155 @@ def pin_backward_dilation_decomposition(orc):
         np.testing.assert_allclose(got[3], drpb_sum, rtol=0, atol=1e-11)
 
 
+# ---------------------------------------------------------------------------
+# Dropout.
+def _philox_py(ctr, key):
+    """Philox4x32-10 restated from its publication (SC 2011), independent of
+    the oracle's C: 10 rounds, multipliers 0xD2511F53 / 0xCD9E8D57, Weyl key
+    increments 0x9E3779B9 / 0xBB67AE85."""
+    c, k = list(ctr), list(key)
+    for r in range(10):
+        if r:
+            k = [(k[0] + 0x9E3779B9) & 0xFFFFFFFF, (k[1] + 0xBB67AE85) & 0xFFFFFFFF]
+        p0, p1 = 0xD2511F53 * c[0], 0xCD9E8D57 * c[2]
+        c = [((p1 >> 32) ^ c[1] ^ k[0]) & 0xFFFFFFFF, p1 & 0xFFFFFFFF, ((p0 >> 32) ^ c[3] ^ k[1]) & 0xFFFFFFFF,
+             p0 & 0xFFFFFFFF]
+    return c
+
+
+def _keep_py(e, p, seed, offset):
+    blk = e >> 2
+    w = _philox_py((blk & 0xFFFFFFFF, blk >> 32, offset & 0xFFFFFFFF, offset >> 32),
+                   (seed & 0xFFFFFFFF, seed >> 32))[e & 3]
+    t = float(np.float32(p)) * 4294967296.0
+    thresh = 0xFFFFFFFF if t >= 4294967295.0 else int(t + 0.5)
+    return w >= thresh
+
+
+def pin_philox_kat(orc):
+    """The oracle's generator reproduces the published known-answer values."""
+    for line in (GOLDEN / "philox4x32_10_kat.txt").read_text().splitlines():
+        if not line.strip() or line.startswith("#"):
+            continue
+        x = [int(t, 16) for t in line.split()]
+        assert orc.philox(x[0:4], x[4:6]) == x[6:10], line
+        assert _philox_py(x[0:4], x[4:6]) == x[6:10], line
+
+
+def pin_dropout(orc):
+    """Dropout between softmax and the weighted sum, and the returned weights."""
+    rng = np.random.default_rng(31)
+    H, W, k, d, D = 9, 10, 3, 2, 4
+    q, kk, v, rpb = _rand(rng, 2, 2, H, W, D, k)
+    base = orc.forward(q, kk, v, rpb, k, d)
+    out0, a0 = orc.forward_ex(q, kk, v, rpb, k, d, 0.0, 7, 0, return_attn=True)
+    np.testing.assert_allclose(out0, base, rtol=0, atol=TOL)
+    soft = orc.softmax(orc.qk_rpb(q, kk, rpb, k, d), k, d, D)
+    np.testing.assert_allclose(a0, soft, rtol=0, atol=TOL)
+    p, seed, offset = 0.3, (5 << 33) + 11, 3
+    out, a = orc.forward_ex(q, kk, v, rpb, k, d, p, seed, offset, return_attn=True)
+    np.testing.assert_allclose(orc.av(a, v, k, d), out, rtol=0, atol=TOL)
+    keep = np.array([_keep_py(e, p, seed, offset) for e in range(a.size)]).reshape(a.shape)
+    scale = 1.0 / (1.0 - float(np.float32(p)))
+    np.testing.assert_allclose(a, np.where(keep, soft * scale, 0.0), rtol=0, atol=TOL)
+    # keep rate over many weights
+    big = np.zeros((1, 1, 60, 60, 1))
+    _, ab = orc.forward_ex(big, big, big, None, 7, 1, 0.25, 123, 0, return_attn=True)
+    frac = float((ab > 0).mean())
+    n = ab.size
+    assert abs(frac - 0.75) < 5 * math.sqrt(0.75 * 0.25 / n), frac
+
+
+def pin_dropout_backward(orc):
+    """With the mask fixed by (seed, offset), the dropout forward is a smooth
+    function of q, k, v, rpb; its gradients equal central differences."""
+    rng = np.random.default_rng(32)
+    B, heads, H, W, D, k, d = 1, 2, 5, 6, 2, 3, 1
+    q, kk, v, rpb = _rand(rng, B, heads, H, W, D, k)
+    dout = rng.standard_normal(q.shape)
+    p, seed = 0.35, 99
+    got = orc.backward_ex(q, kk, v, rpb, dout, k, d, p, seed, 0)
+    eps = 1e-5
+
+    def loss():
+        return float((orc.forward_ex(q, kk, v, rpb, k, d, p, seed, 0) * dout).sum())
+
+    for name, x, grad in (("q", q, got[0]), ("k", kk, got[1]), ("v", v, got[2]), ("rpb", rpb, got[3])):
+        flat, num = x.reshape(-1), np.empty(x.size)
+        for e in range(flat.size):
+            old = flat[e]
+            flat[e] = old + eps
+            up = loss()
+            flat[e] = old - eps
+            dn = loss()
+            flat[e] = old
+            num[e] = (up - dn) / (2 * eps)
+        np.testing.assert_allclose(grad.reshape(-1), num, rtol=1e-6, atol=1e-7, err_msg=f"d{name}")
+    # p = 0: the plain backward
+    for g0, g1 in zip(orc.backward_ex(q, kk, v, rpb, dout, k, d, 0.0, seed, 0),
+                      orc.backward(q, kk, v, rpb, dout, k, d)):
+        np.testing.assert_allclose(g0, g1, rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# Maps shorter than k * d.
+def pin_padding(orc):
+    rng = np.random.default_rng(33)
+    # no padding needed: unchanged
+    q, kk, v, rpb = _rand(rng, 1, 2, 9, 8, 3, 3)
+    np.testing.assert_allclose(orc.forward_padded(q, kk, v, rpb, 3, 2), orc.forward(q, kk, v, rpb, 3, 2),
+                               rtol=0, atol=TOL)
+    # d = 1, H, W < k: every padded window is the whole k x k padded map, so
+    # the real queries see dense attention over it (bias by relative offset)
+    k = 5
+    for (H, W) in [(3, 4), (5, 2), (1, 1)]:
+        q, kk, v, rpb = _rand(rng, 1, 2, H, W, 4, k)
+        pads = ((0, 0), (0, 0), (0, k - H), (0, k - W), (0, 0))
+        Q, K, V = (np.pad(a, pads) for a in (q, kk, v))
+        iy, ix = np.divmod(np.arange(k * k), k)
+        bias = rpb[:, iy[None, :] - iy[:, None] + k - 1, ix[None, :] - ix[:, None] + k - 1][None]
+        want = dense_attention(Q, K, V, bias)[:, :, :H, :W]
+        np.testing.assert_allclose(orc.forward_padded(q, kk, v, rpb, k, 1), want, rtol=0, atol=TOL)
+    # q = 0, no bias: the plain mean over the searched (padded) window
+    H, W, k, d = 4, 7, 3, 2
+    q, kk, v, _ = _rand(rng, 1, 1, H, W, 3, k, with_rpb=False)
+    got = orc.forward_padded(np.zeros_like(q), kk, v, None, k, d)
+    Hp, Wp = max(H, k * d), max(W, k * d)
+    for i in range(H):
+        ky, _ = axis_window_search(Hp, k, d, i)
+        for j in range(W):
+            kx, _ = axis_window_search(Wp, k, d, j)
+            tot = sum(v[0, 0, y, x] for y in ky for x in kx if y < H and x < W)
+            np.testing.assert_allclose(got[0, 0, i, j], tot / (k * k), rtol=0, atol=TOL)
+
+
+def pin_padding_backward(orc):
+    """Gradients of the padded forward equal central differences."""
+    rng = np.random.default_rng(34)
+    H, W, k, d = 3, 5, 3, 2
+    q, kk, v, rpb = _rand(rng, 1, 1, H, W, 2, k)
+    dout = rng.standard_normal(q.shape)
+    got = orc.backward_padded(q, kk, v, rpb, dout, k, d)
+    eps = 1e-5
+
+    def loss():
+        return float((orc.forward_padded(q, kk, v, rpb, k, d) * dout).sum())
+
+    for name, x, grad in (("q", q, got[0]), ("k", kk, got[1]), ("v", v, got[2]), ("rpb", rpb, got[3])):
+        flat, num = x.reshape(-1), np.empty(x.size)
+        for e in range(flat.size):
+            old = flat[e]
+            flat[e] = old + eps
+            up = loss()
+            flat[e] = old - eps
+            dn = loss()
+            flat[e] = old
+            num[e] = (up - dn) / (2 * eps)
+        np.testing.assert_allclose(grad.reshape(-1), num, rtol=1e-6, atol=1e-7, err_msg=f"d{name}")
+
+
 ALL_PINS = [pin_window_keyset, pin_full_attention, pin_brute_force, pin_dilation_decomposition,
             pin_invariants, pin_rpb_orientation, pin_translation, pin_split_stages, pin_stage_table,
             pin_forward_query, pin_backward_finite_differences, pin_backward_dense_autograd,
-            pin_backward_identities, pin_backward_dilation_decomposition]
+            pin_backward_identities, pin_backward_dilation_decomposition, pin_philox_kat, pin_dropout,
+            pin_dropout_backward, pin_padding, pin_padding_backward]

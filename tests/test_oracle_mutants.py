@@ -54,6 +54,14 @@ MUTANTS = {
     "bwd_dv_uses_ds": [("dv[key + c] += sc[n] * g[c];", "dv[key + c] += ds * g[c];")],
     "bwd_drpb_transposed": [("drpb_acc[((size_t)h * nb + by[ty]) * nb + bx[tx]] += ds;",
                              "drpb_acc[((size_t)h * nb + bx[tx]) * nb + by[ty]] += ds;")],
+    # dropout and its generator (indices unchanged)
+    "philox_lo_hi_swapped": [("unsigned int n1 = (unsigned int)prod1;", "unsigned int n1 = (unsigned int)(prod1 >> 32);")],
+    "philox_key_not_bumped": [("            k0 += 0x9E3779B9u;\n", "")],
+    "dropout_not_rescaled": [("? 1.0 / (1.0 - p) : 0.0;", "? 1.0 : 0.0;")],
+    "dropout_keeps_the_dropped": [("return w[e & 3] >= drop_threshold(p)", "return w[e & 3] < drop_threshold(p)")],
+    "dropout_counter_not_grouped": [("unsigned long long blk = e >> 2;", "unsigned long long blk = e;")],
+    "dropout_bwd_dv_unmasked": [("dv[key + c] += f[n] * sc[n] * g[c];", "dv[key + c] += sc[n] * g[c];")],
+    "dropout_bwd_dp_unmasked": [("dp[ty * k + tx] = f[ty * k + tx] * dot;", "dp[ty * k + tx] = dot;")],
     "bwd_drpb_uses_p": [("drpb_acc[((size_t)h * nb + by[ty]) * nb + bx[tx]] += ds;",
                          "drpb_acc[((size_t)h * nb + by[ty]) * nb + bx[tx]] += sc[n];")],
 }
