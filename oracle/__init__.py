@@ -94,8 +94,8 @@ class Oracle:
         lib.oracle_na2d_forward.argtypes = [i] * 7 + [_DP, _DP, _DP, _DP, _DP, i]
         lib.oracle_na2d_backward.argtypes = [i] * 7 + [_DP] * 9 + [i]
         u64, f64 = ctypes.c_ulonglong, ctypes.c_double
-        lib.oracle_na2d_forward_ex.argtypes = [i] * 7 + [_DP] * 6 + [f64, u64, u64]
-        lib.oracle_na2d_backward_ex.argtypes = [i] * 7 + [_DP] * 9 + [f64, u64, u64]
+        lib.oracle_na2d_forward_ex.argtypes = [i] * 7 + [_DP] * 6 + [f64, u64, u64, i, i]
+        lib.oracle_na2d_backward_ex.argtypes = [i] * 7 + [_DP] * 9 + [f64, u64, u64, i, i]
         lib.oracle_philox4x32_10.argtypes = [ctypes.POINTER(ctypes.c_uint)] * 3
         lib.oracle_philox4x32_10.restype = None
         for f in ("oracle_axis_window", "oracle_axis_neighbors", "oracle_na2d_qk_rpb",
@@ -185,29 +185,43 @@ class Oracle:
     def forward_ex(self, q, k, v, rpb, kernel_size: int, dilation: int, dropout_p: float = 0.0, seed: int = 0,
                    offset: int = 0, return_attn: bool = False):
         """Forward with attention dropout (Philox mask) and, optionally, the
-        weights after dropout [B, heads, H, W, k*k]."""
-        q, k, v = _f64(q), _f64(k), _f64(v)
+        weights after dropout [B, heads, H, W, k*k].  Maps shorter than
+        kernel_size * dilation are zero-padded and cropped as in
+        forward_padded; weights are numbered over the real map."""
+        H, W = q.shape[2], q.shape[3]
+        Q, K, V = (self._pad(t, kernel_size, dilation) for t in (q, k, v))
         rpb = None if rpb is None else _f64(rpb)
-        shp = _shape(q, kernel_size, dilation)
-        out = np.empty(q.shape, dtype=np.float64)
+        shp = _shape(Q, kernel_size, dilation)
+        out = np.empty(Q.shape, dtype=np.float64)
         attn = np.empty(q.shape[:4] + (kernel_size * kernel_size,), dtype=np.float64) if return_attn else None
-        _check(self._lib.oracle_na2d_forward_ex(*shp, _ptr(q), _ptr(k), _ptr(v), _ptr(rpb), _ptr(out), _ptr(attn),
-                                                float(np.float32(dropout_p)), seed, offset), "forward_ex")
+        _check(self._lib.oracle_na2d_forward_ex(*shp, _ptr(Q), _ptr(K), _ptr(V), _ptr(rpb), _ptr(out), _ptr(attn),
+                                                float(np.float32(dropout_p)), seed, offset, H, W), "forward_ex")
+        out = np.ascontiguousarray(out[:, :, :H, :W])
         return (out, attn) if return_attn else out
 
     def backward_ex(self, q, k, v, rpb, dout, kernel_size: int, dilation: int, dropout_p: float = 0.0,
                     seed: int = 0, offset: int = 0):
         """Gradients of forward_ex with the same dropout mask."""
-        q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+        H, W = q.shape[2], q.shape[3]
+        Q, K, V, G = (self._pad(t, kernel_size, dilation) for t in (q, k, v, dout))
         rpb = None if rpb is None else _f64(rpb)
-        shp = _shape(q, kernel_size, dilation)
-        dq, dk, dv = (np.empty(q.shape, dtype=np.float64) for _ in range(3))
+        shp = _shape(Q, kernel_size, dilation)
+        dq, dk, dv = (np.empty(Q.shape, dtype=np.float64) for _ in range(3))
         nb = 2 * kernel_size - 1
         drpb = np.empty((q.shape[1], nb, nb), dtype=np.float64)
-        _check(self._lib.oracle_na2d_backward_ex(*shp, _ptr(q), _ptr(k), _ptr(v), _ptr(rpb), _ptr(dout), _ptr(dq),
+        _check(self._lib.oracle_na2d_backward_ex(*shp, _ptr(Q), _ptr(K), _ptr(V), _ptr(rpb), _ptr(G), _ptr(dq),
                                                  _ptr(dk), _ptr(dv), _ptr(drpb), float(np.float32(dropout_p)), seed,
-                                                 offset), "backward_ex")
-        return dq, dk, dv, drpb
+                                                 offset, H, W), "backward_ex")
+        crop = lambda a: np.ascontiguousarray(a[:, :, :H, :W])   # noqa: E731
+        return crop(dq), crop(dk), crop(dv), drpb
+
+    @staticmethod
+    def _pad(t, kernel_size: int, dilation: int):
+        """Zero pixels at the bottom / right up to kernel_size * dilation."""
+        H, W = t.shape[2], t.shape[3]
+        pads = ((0, 0), (0, 0), (0, max(0, kernel_size * dilation - H)), (0, max(0, kernel_size * dilation - W)),
+                (0, 0))
+        return np.ascontiguousarray(np.pad(_f64(t), pads))
 
     # -- maps shorter than k * d ------------------------------------------------
     def forward_padded(self, q, k, v, rpb, kernel_size: int, dilation: int):

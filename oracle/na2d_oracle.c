@@ -557,7 +557,7 @@ static double drop_factor(unsigned long long e, double p, unsigned long long see
  * out = sum_n p_n v_n. */
 static void forward_ex_slice(const oracle_shape *p, int bh, const double *q, const double *kk, const double *v,
                              const double *rpb, double *out, double *attn, double dp, unsigned long long seed,
-                             unsigned long long offset)
+                             unsigned long long offset, int Hr, int Wr)
 {
     const int H = p->H, W = p->W, D = p->D, k = p->k, d = p->d;
     const int h = bh % p->heads;
@@ -589,10 +589,13 @@ static void forward_ex_slice(const oracle_shape *p, int bh, const double *q, con
                 sc[t] = exp(sc[t] - m);
                 sum += sc[t];
             }
-            const unsigned long long row = ((unsigned long long)bh * H + i) * W + j;
+            /* weights are numbered over the real Hr x Wr map (padded queries
+             * are cropped and draw nothing) */
+            const int real = i < Hr && j < Wr;
+            const unsigned long long row = ((unsigned long long)bh * Hr + i) * Wr + j;
             for (int t = 0; t < k * k; ++t) {
-                sc[t] = sc[t] / sum * drop_factor(row * (unsigned long long)(k * k) + t, dp, seed, offset);
-                if (attn) attn[row * (size_t)(k * k) + t] = sc[t];
+                sc[t] = sc[t] / sum * (real ? drop_factor(row * (unsigned long long)(k * k) + t, dp, seed, offset) : 1.0);
+                if (attn && real) attn[row * (size_t)(k * k) + t] = sc[t];
             }
             double *o = out + base + ((size_t)i * W + j) * D;
             for (int c = 0; c < D; ++c) o[c] = 0.0;
@@ -611,7 +614,8 @@ static void forward_ex_slice(const oracle_shape *p, int bh, const double *q, con
  *     dL/ds_n = p_n (dL/dp_n - sum_m p_m dL/dp_m), then as backward_slice. */
 static void backward_ex_slice(const oracle_shape *p, int bh, const double *q, const double *kk, const double *v,
                               const double *rpb, const double *dout, double *dq, double *dk, double *dv,
-                              double *drpb_acc, double dp_, unsigned long long seed, unsigned long long offset)
+                              double *drpb_acc, double dp_, unsigned long long seed, unsigned long long offset,
+                              int Hr, int Wr)
 {
     const int H = p->H, W = p->W, D = p->D, k = p->k, d = p->d;
     const int h = bh % p->heads;
@@ -650,10 +654,11 @@ static void backward_ex_slice(const oracle_shape *p, int bh, const double *q, co
                 sc[t] = exp(sc[t] - m);
                 sum += sc[t];
             }
-            const unsigned long long row = ((unsigned long long)bh * H + i) * W + j;
+            const int real = i < Hr && j < Wr;
+            const unsigned long long row = ((unsigned long long)bh * Hr + i) * Wr + j;
             for (int t = 0; t < k * k; ++t) {
                 sc[t] /= sum;
-                f[t] = drop_factor(row * (unsigned long long)(k * k) + t, dp_, seed, offset);
+                f[t] = real ? drop_factor(row * (unsigned long long)(k * k) + t, dp_, seed, offset) : 1.0;
             }
             double pdp = 0.0;
             for (int ty = 0; ty < k; ++ty)
@@ -683,28 +688,32 @@ static void backward_ex_slice(const oracle_shape *p, int bh, const double *q, co
 }
 
 /* Forward with optional weights output (attn, may be NULL) and dropout
- * probability dp (0: none); single-threaded per call, slices in order. */
+ * probability dp (0: none); single-threaded per call, slices in order.  The
+ * arrays may be a zero-padded map whose real part is the top-left Hr x Wr
+ * (Hr = H, Wr = W without padding): weights are numbered over the real map,
+ * and attn holds [B, heads, Hr, Wr, k*k]. */
 int oracle_na2d_forward_ex(int B, int heads, int H, int W, int D, int k, int d, const double *q,
                            const double *kk, const double *v, const double *rpb, double *out, double *attn,
-                           double dp, unsigned long long seed, unsigned long long offset)
+                           double dp, unsigned long long seed, unsigned long long offset, int Hr, int Wr)
 {
     oracle_shape p = make_shape(B, heads, H, W, D, k, d);
-    if (!shape_ok(&p)) return -1;
-    for (int bh = 0; bh < B * heads; ++bh) forward_ex_slice(&p, bh, q, kk, v, rpb, out, attn, dp, seed, offset);
+    if (!shape_ok(&p) || Hr < 1 || Hr > H || Wr < 1 || Wr > W) return -1;
+    for (int bh = 0; bh < B * heads; ++bh)
+        forward_ex_slice(&p, bh, q, kk, v, rpb, out, attn, dp, seed, offset, Hr, Wr);
     return 0;
 }
 
 int oracle_na2d_backward_ex(int B, int heads, int H, int W, int D, int k, int d, const double *q,
                             const double *kk, const double *v, const double *rpb, const double *dout, double *dq,
                             double *dk, double *dv, double *drpb, double dp, unsigned long long seed,
-                            unsigned long long offset)
+                            unsigned long long offset, int Hr, int Wr)
 {
     oracle_shape p = make_shape(B, heads, H, W, D, k, d);
-    if (!shape_ok(&p)) return -1;
+    if (!shape_ok(&p) || Hr < 1 || Hr > H || Wr < 1 || Wr > W) return -1;
     const size_t ntab = (size_t)heads * (2 * k - 1) * (2 * k - 1);
     double *acc = calloc(ntab ? ntab : 1, sizeof(double));
     for (int bh = 0; bh < B * heads; ++bh)
-        backward_ex_slice(&p, bh, q, kk, v, rpb, dout, dq, dk, dv, acc, dp, seed, offset);
+        backward_ex_slice(&p, bh, q, kk, v, rpb, dout, dq, dk, dv, acc, dp, seed, offset, Hr, Wr);
     if (drpb)
         for (size_t e = 0; e < ntab; ++e) drpb[e] = acc[e];
     free(acc);

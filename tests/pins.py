@@ -484,6 +484,19 @@ def pin_dropout_backward(orc):
     for g0, g1 in zip(orc.backward_ex(q, kk, v, rpb, dout, k, d, 0.0, seed, 0),
                       orc.backward(q, kk, v, rpb, dout, k, d)):
         np.testing.assert_allclose(g0, g1, rtol=0, atol=1e-12)
+    # a map shorter than k * d: without dropout, the padded forward/backward;
+    # with dropout, weights numbered over the real map (the mask of weight
+    # (b, h, i, j, n) does not depend on the padding)
+    H2, W2, k2, d2 = 4, 5, 3, 2
+    q2, k2_, v2, r2 = _rand(rng, 1, 2, H2, W2, 3, k2)
+    g2 = rng.standard_normal(q2.shape)
+    np.testing.assert_allclose(orc.forward_ex(q2, k2_, v2, r2, k2, d2), orc.forward_padded(q2, k2_, v2, r2, k2, d2),
+                               rtol=0, atol=TOL)
+    for a, b in zip(orc.backward_ex(q2, k2_, v2, r2, g2, k2, d2), orc.backward_padded(q2, k2_, v2, r2, g2, k2, d2)):
+        np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+    _, a2 = orc.forward_ex(q2, k2_, v2, r2, k2, d2, 0.4, 17, 2, return_attn=True)
+    keep = np.array([_keep_py(e, 0.4, 17, 2) for e in range(a2.size)]).reshape(a2.shape)
+    assert np.array_equal(a2 > 0, keep)
 
 
 # ---------------------------------------------------------------------------
