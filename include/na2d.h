@@ -42,12 +42,27 @@
  * NA2D_ERR_CUDA (the CUDA error is cleared with cudaGetLastError).  Nothing
  * in the library aborts, traps or prints.
  *
- * Supported set: dtype f32 / f16 / bf16; D = 32; odd k in [1, 13]; d >= 1;
- * H >= k*d and W >= k*d (every dilation group holds at least k positions);
- * B, heads >= 0 (an empty problem returns NA2D_OK without a launch);
- * B*heads*H*W*max(D, k*k) < 2^62; H*W*max(D, k*k) < 2^31; tensor pointers
- * 16-byte aligned (rpb: element aligned).  Arithmetic: fp32 accumulation for
- * every dtype; f16 / bf16 outputs are rounded to nearest even.
+ * Supported set: dtype f32 / f16 / bf16; D in {16, 32, 64, 128}; odd k in
+ * [1, 13]; d >= 1; H, W >= 1; B, heads >= 0 (an empty problem returns NA2D_OK
+ * without a launch); with Hp = max(H, k*d), Wp = max(W, k*d):
+ * B*heads*Hp*Wp*max(D, k*k) < 2^62 and Hp*Wp*max(D, k*k) < 2^31; tensor
+ * pointers 16-byte aligned (rpb: element aligned).  Arithmetic: fp32
+ * accumulation for every dtype; f16 / bf16 outputs are rounded to nearest
+ * even.
+ *
+ * Maps shorter than k*d: the HF DiNAT layer pads its feature map at the
+ * bottom and right up to kernel_size * dilation before attention and crops
+ * afterwards ("maybe_pad"; "Dilated Neighborhood Attention Transformer", HF
+ * docs, DinatModel, and the gitcode DiNAT article's source walkthrough).  At
+ * this boundary the padded pixels are zero vectors of q, k and v: the window
+ * rule runs on the padded size Hp x Wp, a padded key scores its bias alone
+ * and carries a zero value, and only the H x W real queries are computed and
+ * written.  (The layer pads before its q/k/v projection, so its padded
+ * pixels hold the projection biases; a caller that wants exactly that pads
+ * its hidden states itself, which makes H, W >= k*d here.)
+ *
+ * Fast paths: f16 / bf16 with D = 32 and H, W >= k*d run on tensor-core
+ * kernels; every other problem runs on the CUDA-core kernel.
  */
 #ifndef NA2D_H
 #define NA2D_H
@@ -58,6 +73,8 @@
 #define NA2D_API
 #endif
 
+#include <stddef.h>
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -66,11 +83,13 @@ typedef enum {
     NA2D_OK = 0,
     NA2D_ERR_NULL = 1,      /* a required pointer (problem, q, k, v, out, attn) is NULL */
     NA2D_ERR_DTYPE = 2,     /* dtype is not one of na2d_dtype */
-    NA2D_ERR_SHAPE = 3,     /* negative B/heads, H or W < 1, H < k*d or W < k*d,
-                               D other than 32, or a size limit exceeded */
+    NA2D_ERR_SHAPE = 3,     /* negative B/heads, H or W < 1, D not 16/32/64/128, a
+                               size limit exceeded, a workspace too small, or a
+                               dropout probability outside [0, 1) */
     NA2D_ERR_KERNEL = 4,    /* k even, < 1 or > 13 */
     NA2D_ERR_DILATION = 5,  /* d < 1 */
-    NA2D_ERR_ALIGN = 6,     /* q, k, v, out or attn not 16-byte aligned, rpb not element aligned */
+    NA2D_ERR_ALIGN = 6,     /* a tensor not 16-byte aligned (or a stride not a multiple of 16
+                               bytes), rpb not element aligned */
     NA2D_ERR_ALIAS = 7,     /* an output buffer overlaps an input buffer */
     NA2D_ERR_CUDA = 8,      /* a CUDA runtime call or kernel launch failed */
     NA2D_ERR_INTERNAL = 9   /* an internal consistency check failed */
@@ -83,7 +102,7 @@ typedef struct {
     int B;            /* batch */
     int heads;        /* attention heads */
     int H, W;         /* feature map height and width */
-    int D;            /* head dim (32) */
+    int D;            /* head dim: 16, 32, 64 or 128 */
     int k;            /* kernel size: odd, 1..13 */
     int d;            /* dilation: >= 1 */
     na2d_dtype dtype; /* element type of q, k, v, rpb and out */
@@ -156,6 +175,56 @@ NA2D_API na2d_status na2d_backward(const na2d_problem *p, const void *q, const v
 NA2D_API na2d_status na2d_backward_noalloc(const na2d_problem *p, const void *q, const void *k, const void *v,
                                            const void *rpb, const void *dout, void *dq, void *dk, void *dv,
                                            void *drpb, void *stream);
+
+/* A [B, heads, H, W, D] tensor given by element strides, channels contiguous
+ * (element (b, h, y, x, c) at data + b*stride_b + h*stride_h + y*stride_y +
+ * x*stride_x + c).  It covers the channels-last layouts of the model: the
+ * hidden states are (b, h, w, channels) ("Dilated Neighborhood Attention
+ * Transformer", gitcode DiNAT article, "作为骨干网络（Backbone）使用"), and the
+ * fused q/k/v projection output (B, H, W, 3, heads, D) is read in place as
+ * three such views (strides 3*heads*D per pixel, D per head, offsets 0,
+ * heads*D and 2*heads*D).  data is 16-byte aligned and every stride is
+ * non-negative with stride * element size a multiple of 16 bytes
+ * (NA2D_ERR_ALIGN otherwise). */
+typedef struct {
+    void *data;
+    long long stride_b, stride_h, stride_y, stride_x;
+} na2d_tensor;
+
+/* Attention dropout between the softmax and the weighted sum, as in the
+ * layer (gitcode DiNAT article, "DiNAT 的核心思想": the weights pass through
+ * dropout before natten2dav).  Weight number e (its linear index in the
+ * [B, heads, H, W, k*k] weight tensor) is kept when word e % 4 of
+ * Philox4x32-10(counter = (e/4 low 32 bits, e/4 high, offset low, offset
+ * high), key = (seed low, seed high)) is >= round(p * 2^32); a kept weight is
+ * scaled by 1 / (1 - p).  p in [0, 1); 0 disables dropout.  The same seed and
+ * offset in na2d_backward_ex reproduce the mask. */
+typedef struct {
+    float p;
+    unsigned long long seed;
+    unsigned long long offset;
+} na2d_dropout;
+
+/* na2d_forward on strided tensors, optionally also writing the attention
+ * weights (after dropout, as the layer returns them with output_attentions)
+ * to attn [B, heads, H, W, k*k] fp32 (NULL: not written) and applying
+ * dropout (drop NULL or drop->p == 0: none; p outside [0, 1):
+ * NA2D_ERR_SHAPE).  q, k, v, out are views (see na2d_tensor); out must not
+ * overlap itself, an input or attn (NA2D_ERR_ALIAS).  Contiguous tensors
+ * without weights or dropout take the same kernels as na2d_forward; other
+ * calls run on the CUDA-core kernel. */
+NA2D_API na2d_status na2d_forward_ex(const na2d_problem *p, const na2d_tensor *q, const na2d_tensor *k,
+                                     const na2d_tensor *v, const void *rpb, const na2d_tensor *out, float *attn,
+                                     const na2d_dropout *drop, void *stream);
+
+/* na2d_backward on strided tensors with attention dropout (the mask of the
+ * forward call with the same na2d_dropout).  Same workspace rule as
+ * na2d_backward; runs on the CUDA cores. */
+NA2D_API na2d_status na2d_backward_ex(const na2d_problem *p, const na2d_tensor *q, const na2d_tensor *k,
+                                      const na2d_tensor *v, const void *rpb, const na2d_tensor *dout,
+                                      const na2d_tensor *dq, const na2d_tensor *dk, const na2d_tensor *dv,
+                                      void *drpb, const na2d_dropout *drop, void *workspace,
+                                      size_t workspace_bytes, void *stream);
 
 /* Diagnostic.  Kernels that wait on shared-memory barriers for their own
  * tensor copies give up after about a second of device time (a wait that long

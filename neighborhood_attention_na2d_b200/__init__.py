@@ -10,18 +10,27 @@ in the library's sm_100a kernels):
     na2d_forward(q, k, v, rpb, kernel_size, dilation)    -> out   (fused)
     na2d_backward(q, k, v, rpb, dout, kernel_size, dilation) -> (dq, dk, dv, drpb)
     na2d(q, k, v, rpb, kernel_size, dilation)            -> out   (autograd: backward via na2d_backward)
+    na2d_forward_ex(q, k, v, rpb, kernel_size, dilation, return_attn=, dropout_p=, seed=)
+                                                         -> out [, attn]  (strided views, weights, dropout)
+    na2d_backward_ex(q, k, v, rpb, dout, ...)            -> (dq, dk, dv, drpb)  (strided views, dropout)
+    na2d_qkv_packed(qkv, rpb, kernel_size, dilation, heads) -> out (B, H, W, heads*D), read in place
 
-q, k, v are contiguous [B, heads, H, W, D] tensors in float32, float16 or
-bfloat16 on one CUDA device; rpb is [heads, 2k-1, 2k-1] in the same dtype, or
-None.  Calls are asynchronous on the current torch stream.  A non-OK status
-from the library raises ``Na2dError``; there is no CPU fallback.
+q, k, v are [B, heads, H, W, D] tensors (D in 16, 32, 64, 128) in float32,
+float16 or bfloat16 on one CUDA device -- contiguous for the plain calls, any
+strides with contiguous channels for the _ex calls; rpb is [heads, 2k-1, 2k-1]
+in the same dtype, or None.  Maps shorter than k*d are zero-padded at the
+bottom/right and cropped, as the DiNAT layer does.  Calls are asynchronous on
+the current torch stream.  A non-OK status from the library raises
+``Na2dError``; there is no CPU fallback.
 """
 from __future__ import annotations
 
-from ._native import Na2dError, Problem, backward_workspace_size, check, device_faults, lib, status_str  # noqa: F401
+from ._native import (Dropout, Na2dError, Problem, Tensor, backward_workspace_size, check, device_faults, lib,  # noqa: F401
+                      status_str)
 
 __all__ = ["na2d_qk_rpb", "na2d_softmax", "na2d_av", "na2d_forward", "na2d_status_str", "na2d_device_faults",
-           "na2d_last_kernel", "na2d_backward", "na2d", "Na2dError", "make_problem"]
+           "na2d_last_kernel", "na2d_backward", "na2d", "na2d_forward_ex", "na2d_backward_ex", "na2d_qkv_packed",
+           "Na2dError", "make_problem"]
 
 # status codes used for argument errors raised before the library is called
 _ERR_NULL, _ERR_DTYPE, _ERR_SHAPE = 1, 2, 3
@@ -214,18 +223,25 @@ def _autograd_function():
         (both in the library's kernels)."""
 
         @staticmethod
-        def forward(ctx, q, k, v, rpb, kernel_size, dilation):
-            q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+        def forward(ctx, q, k, v, rpb, kernel_size, dilation, dropout_p, seed):
             rpb = None if rpb is None else rpb.contiguous()
             ctx.save_for_backward(q, k, v, rpb)
             ctx.kd = (kernel_size, dilation)
+            ctx.drop = (dropout_p, seed)
+            if dropout_p:
+                return na2d_forward_ex(q, k, v, rpb, kernel_size, dilation, dropout_p=dropout_p, seed=seed)
+            q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
             return na2d_forward(q, k, v, rpb, kernel_size, dilation)
 
         @staticmethod
         def backward(ctx, dout):
             q, k, v, rpb = ctx.saved_tensors
-            dq, dk, dv, drpb = na2d_backward(q, k, v, rpb, dout.contiguous(), *ctx.kd)
-            return dq, dk, dv, drpb, None, None
+            p, seed = ctx.drop
+            if p or not (q.is_contiguous() and k.is_contiguous() and v.is_contiguous()):
+                dq, dk, dv, drpb = na2d_backward_ex(q, k, v, rpb, dout, *ctx.kd, dropout_p=p, seed=seed)
+            else:
+                dq, dk, dv, drpb = na2d_backward(q, k, v, rpb, dout.contiguous(), *ctx.kd)
+            return dq, dk, dv, drpb, None, None, None, None
 
     return _NA2D
 
@@ -233,10 +249,122 @@ def _autograd_function():
 _NA2D = None
 
 
-def na2d(q, k, v, rpb, kernel_size: int, dilation: int = 1):
+def na2d(q, k, v, rpb, kernel_size: int, dilation: int = 1, dropout_p: float = 0.0, seed: int | None = None):
     """Differentiable neighborhood attention (forward and backward in the
-    library's kernels), for training with torch autograd."""
+    library's kernels), for training with torch autograd.  With dropout_p > 0
+    the Philox seed is drawn from torch's CPU generator unless given; the
+    backward reproduces the same mask."""
     global _NA2D
     if _NA2D is None:
         _NA2D = _autograd_function()
-    return _NA2D.apply(q, k, v, rpb, kernel_size, dilation)
+    if dropout_p and seed is None:
+        seed = int(_torch().randint(0, 2 ** 62, (1,)).item())
+    return _NA2D.apply(q, k, v, rpb, kernel_size, dilation, float(dropout_p), int(seed or 0))
+
+
+# ---------------------------------------------------------------------------
+# Strided views, attention weights, dropout.
+def _view(name: str, t, ref_shape, dtype, device) -> Tensor:
+    """An na2d_tensor for a [B, heads, H, W, D] torch tensor with contiguous
+    channels (any other strides); shape, dtype and device are checked here."""
+    if t is None:
+        raise Na2dError(_ERR_NULL, name, f"{name} is required")
+    if tuple(t.shape) != tuple(ref_shape):
+        raise Na2dError(_ERR_SHAPE, name, f"{name} has shape {tuple(t.shape)}, expected {tuple(ref_shape)}")
+    if t.dtype != dtype:
+        raise Na2dError(_ERR_DTYPE, name, f"{name} is {t.dtype}, expected {dtype}")
+    if not t.is_cuda or t.device != device:
+        raise Na2dError(_ERR_NULL, name, f"{name} must be on {device}")
+    if t.stride(4) != 1:
+        raise Na2dError(_ERR_SHAPE, name, f"{name} must have contiguous channels (stride 1 on the last dim)")
+    sb, sh, sy, sx, _ = t.stride()
+    return Tensor(t.data_ptr(), sb, sh, sy, sx)
+
+
+def _dropout(p: float, seed: int, offset: int):
+    if not p:
+        return None
+    return Dropout(float(p), int(seed) & ((1 << 64) - 1), int(offset) & ((1 << 64) - 1))
+
+
+def na2d_forward_ex(q, k, v, rpb, kernel_size: int, dilation: int = 1, out=None, return_attn: bool = False,
+                    dropout_p: float = 0.0, seed: int = 0, offset: int = 0):
+    """Forward on strided tensors (e.g. channels-last views), optionally
+    returning the attention weights [B, heads, H, W, k*k] (fp32, after
+    dropout) and applying attention dropout (Philox, seed/offset)."""
+    import ctypes
+    torch = _torch()
+    _check_qkv(q, kernel_size)
+    p = make_problem(q.shape, kernel_size, dilation, q.dtype)
+    _check_rpb(rpb, q, kernel_size)
+    if out is None:
+        out = torch.empty(q.shape, dtype=q.dtype, device=q.device)
+    views = [_view(n, t, q.shape, q.dtype, q.device) for n, t in (("q", q), ("k", k), ("v", v), ("out", out))]
+    attn = None
+    if return_attn:
+        attn = torch.empty(_attn_shape(q, kernel_size), dtype=torch.float32, device=q.device)
+    dr = _dropout(dropout_p, seed, offset)
+    with torch.cuda.device(q.device):
+        check(lib().na2d_forward_ex(p, *[ctypes.byref(x) for x in views[:3]], _ptr(rpb), ctypes.byref(views[3]),
+                                    None if attn is None else attn.data_ptr(),
+                                    None if dr is None else ctypes.byref(dr), _stream(q)), "na2d_forward_ex")
+    return (out, attn) if return_attn else out
+
+
+def na2d_backward_ex(q, k, v, rpb, dout, kernel_size: int, dilation: int = 1, dq=None, dk=None, dv=None,
+                     drpb=None, dropout_p: float = 0.0, seed: int = 0, offset: int = 0, workspace=None):
+    """Backward on strided tensors with the forward's dropout mask (same
+    dropout_p, seed, offset); returns (dq, dk, dv, drpb)."""
+    import ctypes
+    torch = _torch()
+    _check_qkv(q, kernel_size)
+    p = make_problem(q.shape, kernel_size, dilation, q.dtype)
+    _check_rpb(rpb, q, kernel_size)
+    dq = torch.empty(q.shape, dtype=q.dtype, device=q.device) if dq is None else dq
+    dk = torch.empty(q.shape, dtype=q.dtype, device=q.device) if dk is None else dk
+    dv = torch.empty(q.shape, dtype=q.dtype, device=q.device) if dv is None else dv
+    if rpb is not None and drpb is None:
+        drpb = torch.empty_like(rpb)
+    if drpb is not None:
+        _check_rpb(drpb, q, kernel_size)
+    views = [_view(n, t, q.shape, q.dtype, q.device)
+             for n, t in (("q", q), ("k", k), ("v", v), ("dout", dout), ("dq", dq), ("dk", dk), ("dv", dv))]
+    need = backward_workspace_size(p)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    dr = _dropout(dropout_p, seed, offset)
+    with torch.cuda.device(q.device):
+        check(lib().na2d_backward_ex(p, *[ctypes.byref(x) for x in views[:3]], _ptr(rpb), ctypes.byref(views[3]),
+                                     *[ctypes.byref(x) for x in views[4:]], _ptr(drpb),
+                                     None if dr is None else ctypes.byref(dr), _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(), _stream(q)), "na2d_backward_ex")
+    return dq, dk, dv, drpb
+
+
+def qkv_views(qkv, heads: int):
+    """q, k, v as [B, heads, H, W, D] views of a channels-last fused
+    projection output (B, H, W, 3 * heads * D), ordered (3, heads, D) along
+    the channels.  No data moves."""
+    B, H, W, C = qkv.shape
+    if C % (3 * heads):
+        raise Na2dError(_ERR_SHAPE, "qkv", f"channels {C} are not 3 * heads * D for heads={heads}")
+    D = C // (3 * heads)
+    x = qkv.view(B, H, W, 3, heads, D).permute(3, 0, 4, 1, 2, 5)
+    return x[0], x[1], x[2]
+
+
+def na2d_qkv_packed(qkv, rpb, kernel_size: int, dilation: int, heads: int, out=None):
+    """Neighborhood attention read straight from a channels-last fused q/k/v
+    projection (B, H, W, 3 * heads * D); writes and returns the channels-last
+    output (B, H, W, heads * D) (no permute copies on either side)."""
+    torch = _torch()
+    q, k, v = qkv_views(qkv, heads)
+    B, H, W, C = qkv.shape
+    D = C // (3 * heads)
+    if out is None:
+        out = torch.empty(B, H, W, heads * D, dtype=qkv.dtype, device=qkv.device)
+    if tuple(out.shape) != (B, H, W, heads * D) or not out.is_contiguous():
+        raise Na2dError(_ERR_SHAPE, "out", f"out must be a contiguous ({B}, {H}, {W}, {heads * D}) tensor")
+    ov = out.view(B, H, W, heads, D).permute(0, 3, 1, 2, 4)
+    na2d_forward_ex(q, k, v, rpb, kernel_size, dilation, out=ov)
+    return out

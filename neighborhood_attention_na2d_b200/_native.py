@@ -20,13 +20,24 @@ STATUS_NAMES = {
 # every symbol the header declares
 EXPORTS = ("na2d_qk_rpb", "na2d_softmax", "na2d_av", "na2d_forward", "na2d_device_faults", "na2d_status_str",
            "na2d_version", "na2d_last_kernel", "na2d_backward_workspace_size", "na2d_backward",
-           "na2d_backward_noalloc")
+           "na2d_backward_noalloc", "na2d_forward_ex", "na2d_backward_ex")
 
 
 class Problem(ctypes.Structure):
     """``na2d_problem``: one problem description (scale fixed at 1/sqrt(D))."""
     _fields_ = [("B", ctypes.c_int), ("heads", ctypes.c_int), ("H", ctypes.c_int), ("W", ctypes.c_int),
                 ("D", ctypes.c_int), ("k", ctypes.c_int), ("d", ctypes.c_int), ("dtype", ctypes.c_int)]
+
+
+class Tensor(ctypes.Structure):
+    """``na2d_tensor``: data pointer and element strides (b, head, y, x)."""
+    _fields_ = [("data", ctypes.c_void_p), ("stride_b", ctypes.c_longlong), ("stride_h", ctypes.c_longlong),
+                ("stride_y", ctypes.c_longlong), ("stride_x", ctypes.c_longlong)]
+
+
+class Dropout(ctypes.Structure):
+    """``na2d_dropout``: probability, Philox key and counter offset."""
+    _fields_ = [("p", ctypes.c_float), ("seed", ctypes.c_ulonglong), ("offset", ctypes.c_ulonglong)]
 
 
 class Na2dError(RuntimeError):
@@ -68,6 +79,11 @@ def lib() -> ctypes.CDLL:
         L.na2d_backward.restype = ctypes.c_int
         L.na2d_backward_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.na2d_backward_noalloc.restype = ctypes.c_int
+        TP, DP = ctypes.POINTER(Tensor), ctypes.POINTER(Dropout)
+        L.na2d_forward_ex.argtypes = [P, TP, TP, TP, vp, TP, fp, DP, vp]
+        L.na2d_forward_ex.restype = ctypes.c_int
+        L.na2d_backward_ex.argtypes = [P, TP, TP, TP, vp, TP, TP, TP, TP, vp, DP, vp, ctypes.c_size_t, vp]
+        L.na2d_backward_ex.restype = ctypes.c_int
         L.na2d_last_kernel.argtypes = []
         L.na2d_last_kernel.restype = ctypes.c_char_p
         _lib = L

@@ -2,6 +2,7 @@
 // host-side argument checks, then one launch on the caller's stream.
 #include <cuda_runtime.h>
 
+#include <climits>
 #include <cstdint>
 
 #include "../../include/na2d.h"
@@ -10,7 +11,9 @@
 namespace {
 
 using na2d::DType;
+using na2d::Dropout;
 using na2d::Problem;
+using na2d::View;
 
 constexpr int64_t kMaxTotal = (int64_t)1 << 62;
 constexpr int64_t kMaxPlane = ((int64_t)1 << 31) - 1;
@@ -33,11 +36,13 @@ na2d_status check_problem(const na2d_problem *p, Problem *out, bool *empty) {
     if (p->k < 1 || p->k > 13 || (p->k % 2) == 0) return NA2D_ERR_KERNEL;
     if (p->d < 1) return NA2D_ERR_DILATION;
     if (p->B < 0 || p->heads < 0 || p->H < 1 || p->W < 1) return NA2D_ERR_SHAPE;
-    if (p->D != 32) return NA2D_ERR_SHAPE;
-    // every dilation group must hold at least k positions: floor(L / d) >= k
-    if ((int64_t)p->k * p->d > p->H || (int64_t)p->k * p->d > p->W) return NA2D_ERR_SHAPE;
+    if (p->D != 16 && p->D != 32 && p->D != 64 && p->D != 128) return NA2D_ERR_SHAPE;
+    // maps shorter than k*d are padded (up to k*d), which bounds the padded size
+    if ((int64_t)p->k * p->d > kMaxPlane) return NA2D_ERR_SHAPE;
+    const int64_t Hp = p->H > (int64_t)p->k * p->d ? p->H : (int64_t)p->k * p->d;
+    const int64_t Wp = p->W > (int64_t)p->k * p->d ? p->W : (int64_t)p->k * p->d;
     const int64_t inner = (int64_t)(p->D > p->k * p->k ? p->D : p->k * p->k);
-    const int64_t plane = (int64_t)p->H * p->W * inner;
+    const int64_t plane = Hp * Wp * inner;
     if (plane > kMaxPlane) return NA2D_ERR_SHAPE;
     const int64_t bh = (int64_t)p->B * p->heads;
     if (bh > 0 && bh > kMaxTotal / plane) return NA2D_ERR_SHAPE;
@@ -56,6 +61,74 @@ size_t rpb_bytes(const na2d_problem *p) {
 
 bool rpb_aligned(const na2d_problem *p, const void *rpb) {
     return !rpb || (reinterpret_cast<uintptr_t>(rpb) % elem_size(p->dtype)) == 0;
+}
+
+// A strided tensor argument: 16-byte aligned data, strides (in elements) that
+// keep every pixel row 16-byte aligned, and non-negative.
+na2d_status check_tensor(const na2d_problem *p, const na2d_tensor *t, View *v) {
+    if (!t || !t->data) return NA2D_ERR_NULL;
+    const long long st[4] = {t->stride_b, t->stride_h, t->stride_y, t->stride_x};
+    const size_t e = elem_size(p->dtype);
+    for (long long x : st)
+        if (x < 0 || ((size_t)x * e) % 16 != 0) return NA2D_ERR_ALIGN;
+    if (!aligned16(t->data)) return NA2D_ERR_ALIGN;
+    *v = View{t->data, st[0], st[1], st[2], st[3]};
+    return NA2D_OK;
+}
+
+// [first byte, one past the last byte] a view can touch.
+void view_span(const na2d_problem *p, const View &v, uintptr_t *lo, uintptr_t *hi) {
+    const size_t e = elem_size(p->dtype);
+    const int64_t last = (int64_t)(p->B - 1) * v.sb + (int64_t)(p->heads - 1) * v.sh + (int64_t)(p->H - 1) * v.sy +
+                         (int64_t)(p->W - 1) * v.sx + p->D;
+    *lo = reinterpret_cast<uintptr_t>(v.p);
+    *hi = *lo + (size_t)last * e;
+}
+bool spans_overlap(uintptr_t a0, uintptr_t a1, uintptr_t b0, uintptr_t b1) { return a0 < b1 && b0 < a1; }
+
+// An output view whose pixels do not overlap one another: sorted by stride,
+// each dimension steps past the whole extent of the smaller ones.
+bool view_disjoint(const na2d_problem *p, const View &v) {
+    int64_t st[4] = {v.sb, v.sh, v.sy, v.sx}, ex[4] = {p->B, p->heads, p->H, p->W};
+    for (int i = 0; i < 4; ++i)
+        for (int j = i + 1; j < 4; ++j)
+            if (st[j] < st[i]) {
+                int64_t t = st[i]; st[i] = st[j]; st[j] = t;
+                t = ex[i]; ex[i] = ex[j]; ex[j] = t;
+            }
+    int64_t span = p->D;   // channels are contiguous
+    for (int i = 0; i < 4; ++i) {
+        if (ex[i] <= 1) continue;
+        if (st[i] < span) return false;
+        span = st[i] * (ex[i] - 1) + span;
+    }
+    return true;
+}
+
+// Two views that cannot touch a common element: their address spans are
+// apart, or they have the same strides and interleave block by block (the
+// q / k / v or dq / dk / dv views of one fused channels-last buffer).  The
+// block of a view is its D channels, or the heads * D channels of a pixel when
+// the head stride is D; the views must start at least a block apart and end
+// a block before the next pixel (the smallest stride beyond the block).
+bool views_disjoint(const na2d_problem *p, const View &a, const View &b) {
+    uintptr_t a0, a1, b0, b1;
+    view_span(p, a, &a0, &a1);
+    view_span(p, b, &b0, &b1);
+    if (!spans_overlap(a0, a1, b0, b1)) return true;
+    if (a.sb != b.sb || a.sh != b.sh || a.sy != b.sy || a.sx != b.sx) return false;
+    const int64_t e = (int64_t)elem_size(p->dtype);
+    const int64_t diff = (int64_t)(reinterpret_cast<uintptr_t>(b.p) - reinterpret_cast<uintptr_t>(a.p));
+    if (diff % e) return false;
+    const int64_t delta = diff < 0 ? -diff / e : diff / e;
+    const bool heads_packed = a.sh == p->D && p->heads > 1;
+    const int64_t block = heads_packed ? (int64_t)p->heads * p->D : p->D;
+    int64_t next = INT64_MAX;
+    const int64_t st[4] = {a.sb, heads_packed ? INT64_MAX : a.sh, a.sy, a.sx};
+    const int64_t ex[4] = {p->B, p->heads, p->H, p->W};
+    for (int i = 0; i < 4; ++i)
+        if (ex[i] > 1 && st[i] < next) next = st[i];
+    return delta >= block && delta + block <= next;
 }
 
 // Name of the kernel the calling thread's last forward call launched.
@@ -98,7 +171,52 @@ na2d_status na2d_forward(const na2d_problem *p, const void *q, const void *k, co
         if (e != cudaSuccess || launched) return from_cuda(e);
         return from_cuda(na2d::launch_forward_tc(pr, q, k, v, rpb, out, st));
     }
-    return from_cuda(na2d::launch_forward_simt(pr, q, k, v, rpb, out, st));
+    return from_cuda(na2d::launch_forward_simt(pr, View::contiguous(q, pr), View::contiguous(k, pr),
+                                               View::contiguous(v, pr), rpb, View::contiguous(out, pr), nullptr,
+                                               Dropout{0.f, 0, 0}, st));
+}
+
+na2d_status na2d_forward_ex(const na2d_problem *p, const na2d_tensor *q, const na2d_tensor *k,
+                            const na2d_tensor *v, const void *rpb, const na2d_tensor *out, float *attn,
+                            const na2d_dropout *drop, void *stream) {
+    Problem pr;
+    bool empty = false;
+    na2d_status s = check_problem(p, &pr, &empty);
+    if (s != NA2D_OK) return s;
+    if (empty) return NA2D_OK;
+    View vq, vk, vv, vo;
+    if ((s = check_tensor(p, q, &vq)) != NA2D_OK || (s = check_tensor(p, k, &vk)) != NA2D_OK ||
+        (s = check_tensor(p, v, &vv)) != NA2D_OK || (s = check_tensor(p, out, &vo)) != NA2D_OK)
+        return s;
+    if (!rpb_aligned(p, rpb) || (attn && !aligned16(attn))) return NA2D_ERR_ALIGN;
+    Dropout dr{0.f, 0, 0};
+    if (drop) {
+        if (!(drop->p >= 0.f && drop->p < 1.f)) return NA2D_ERR_SHAPE;
+        dr = Dropout{drop->p, drop->seed, drop->offset};
+    }
+    if (!view_disjoint(p, vo)) return NA2D_ERR_ALIAS;
+    uintptr_t o0, o1, a0, a1;
+    view_span(p, vo, &o0, &o1);
+    const View ins[3] = {vq, vk, vv};
+    for (const View &x : ins)
+        if (!views_disjoint(p, vo, x)) return NA2D_ERR_ALIAS;
+    if (rpb && spans_overlap(o0, o1, reinterpret_cast<uintptr_t>(rpb), reinterpret_cast<uintptr_t>(rpb) + rpb_bytes(p)))
+        return NA2D_ERR_ALIAS;
+    if (attn) {
+        const uintptr_t t0 = reinterpret_cast<uintptr_t>(attn), t1 = t0 + attn_bytes(p);
+        if (spans_overlap(o0, o1, t0, t1)) return NA2D_ERR_ALIAS;
+        for (const View &x : ins) {
+            view_span(p, x, &a0, &a1);
+            if (spans_overlap(t0, t1, a0, a1)) return NA2D_ERR_ALIAS;
+        }
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    t_last_kernel = nullptr;
+    // contiguous tensors without the optional parts take na2d_forward's kernels
+    if (!attn && dr.p == 0.f && vq.is_contiguous(pr) && vk.is_contiguous(pr) && vv.is_contiguous(pr) &&
+        vo.is_contiguous(pr))
+        return na2d_forward(p, q->data, k->data, v->data, rpb, out->data, stream);
+    return from_cuda(na2d::launch_forward_simt(pr, vq, vk, vv, rpb, vo, attn, dr, st));
 }
 
 na2d_status na2d_qk_rpb(const na2d_problem *p, const void *q, const void *k, const void *rpb, float *attn,
@@ -178,6 +296,64 @@ na2d_status na2d_backward(const na2d_problem *p, const void *q, const void *k, c
     t_last_kernel = nullptr;
     return from_cuda(na2d::launch_backward(pr, q, k, v, rpb, dout, dq, dk, dv, drpb, workspace,
                                            static_cast<cudaStream_t>(stream)));
+}
+
+na2d_status na2d_backward_ex(const na2d_problem *p, const na2d_tensor *q, const na2d_tensor *k,
+                             const na2d_tensor *v, const void *rpb, const na2d_tensor *dout, const na2d_tensor *dq,
+                             const na2d_tensor *dk, const na2d_tensor *dv, void *drpb, const na2d_dropout *drop,
+                             void *workspace, size_t workspace_bytes, void *stream) {
+    Problem pr;
+    bool empty = false;
+    na2d_status s = check_problem(p, &pr, &empty);
+    if (s != NA2D_OK) return s;
+    if (empty) return NA2D_OK;
+    View vq, vk, vv, vg, vdq, vdk, vdv;
+    if ((s = check_tensor(p, q, &vq)) != NA2D_OK || (s = check_tensor(p, k, &vk)) != NA2D_OK ||
+        (s = check_tensor(p, v, &vv)) != NA2D_OK || (s = check_tensor(p, dout, &vg)) != NA2D_OK ||
+        (s = check_tensor(p, dq, &vdq)) != NA2D_OK || (s = check_tensor(p, dk, &vdk)) != NA2D_OK ||
+        (s = check_tensor(p, dv, &vdv)) != NA2D_OK)
+        return s;
+    if (!workspace) return NA2D_ERR_NULL;
+    if (!aligned16(workspace) || !rpb_aligned(p, rpb) || !rpb_aligned(p, drpb)) return NA2D_ERR_ALIGN;
+    const size_t need = na2d::backward_workspace_bytes(pr);
+    if (workspace_bytes < need) return NA2D_ERR_SHAPE;
+    Dropout dr{0.f, 0, 0};
+    if (drop) {
+        if (!(drop->p >= 0.f && drop->p < 1.f)) return NA2D_ERR_SHAPE;
+        dr = Dropout{drop->p, drop->seed, drop->offset};
+    }
+    const View outs_v[3] = {vdq, vdk, vdv};
+    const View ins_v[4] = {vq, vk, vv, vg};
+    for (int o = 0; o < 3; ++o) {
+        if (!view_disjoint(p, outs_v[o])) return NA2D_ERR_ALIAS;
+        for (const View &x : ins_v)
+            if (!views_disjoint(p, outs_v[o], x)) return NA2D_ERR_ALIAS;
+        for (int o2 = o + 1; o2 < 3; ++o2)
+            if (!views_disjoint(p, outs_v[o], outs_v[o2])) return NA2D_ERR_ALIAS;
+    }
+    // the workspace and drpb against every tensor and each other
+    uintptr_t lo[2] = {reinterpret_cast<uintptr_t>(workspace), reinterpret_cast<uintptr_t>(drpb)};
+    uintptr_t hi[2] = {lo[0] + need, drpb ? lo[1] + rpb_bytes(p) : lo[1]};
+    for (int o = 0; o < 2; ++o) {
+        if (lo[o] == hi[o]) continue;
+        for (const View &x : ins_v) {
+            uintptr_t a0, a1;
+            view_span(p, x, &a0, &a1);
+            if (spans_overlap(lo[o], hi[o], a0, a1)) return NA2D_ERR_ALIAS;
+        }
+        for (const View &x : outs_v) {
+            uintptr_t a0, a1;
+            view_span(p, x, &a0, &a1);
+            if (spans_overlap(lo[o], hi[o], a0, a1)) return NA2D_ERR_ALIAS;
+        }
+        if (rpb && spans_overlap(lo[o], hi[o], reinterpret_cast<uintptr_t>(rpb),
+                                 reinterpret_cast<uintptr_t>(rpb) + rpb_bytes(p)))
+            return NA2D_ERR_ALIAS;
+    }
+    if (lo[1] != hi[1] && spans_overlap(lo[0], hi[0], lo[1], hi[1])) return NA2D_ERR_ALIAS;
+    t_last_kernel = nullptr;
+    return from_cuda(na2d::launch_backward_views(pr, vq, vk, vv, rpb, vg, vdq, vdk, vdv, drpb, dr, workspace,
+                                                 static_cast<cudaStream_t>(stream)));
 }
 
 na2d_status na2d_backward_noalloc(const na2d_problem *p, const void *q, const void *k, const void *v,

@@ -4,24 +4,28 @@
 // The layer is trained end to end ("Dilated Neighborhood Attention
 // Transformer", gitcode DiNAT article, section "微调示例：加载预训练权重继续训练";
 // the HF tests described under "源码与测试导览" run forward and backward), so
-// its gradients are the chain rule through scores -> softmax -> weighted sum.
-// For a query with scores s_n, weights p_n and output gradient g:
-//     dp_n = g . v_n,   delta = sum_n p_n dp_n,   ds_n = p_n (dp_n - delta),
+// its gradients are the chain rule through scores -> softmax -> (dropout ->)
+// weighted sum.  For a query with scores s_n, weights p_n, dropout factors
+// z_n (0 or 1 / (1 - p_drop); 1 without dropout) and output gradient g:
+//     dP_n = z_n (g . v_n),   delta = sum_n p_n dP_n,   ds_n = p_n (dP_n - delta),
 //     dq  = sum_n ds_n k_n / sqrt(D),   dk_n += ds_n q / sqrt(D),
-//     dv_n += p_n g,    drpb[h, key' - i' + k - 1] += ds_n.
+//     dv_n += z_n p_n g,    drpb[h, key' - i' + k - 1] += ds_n.
 //
-// Three passes on the caller's stream (fp32 arithmetic throughout):
-//  1. bwd_query_kernel, one warp per query: recomputes the scores and the
-//     softmax (lane t holds neighbours t, t + 32, ...), writes dq, and stores
-//     the query's log-sum-exp and delta in the workspace; a block covers
-//     queries of one (batch, head) image and sums its bias gradient in shared
-//     memory before one atomic add per table entry into the workspace's fp32
-//     table.
-//  2. bwd_key_kernel, one warp per key (lane = channel): walks the key's
+// Three passes on the caller's stream (fp32 arithmetic throughout), on
+// tensors given by element strides, any D in {16, 32, 64, 128}, and maps
+// shorter than k*d treated as zero-padded (padded keys have zero q, k and
+// v; padded queries are not outputs, so they carry no gradient):
+//  1. bwd_query_kernel, one warp per real query: recomputes the scores and
+//     the softmax (lane t holds neighbours t, t + 32, ...), writes dq, and
+//     stores the query's log-sum-exp and delta in the workspace; a block
+//     covers queries of one (batch, head) image and sums its bias gradient in
+//     shared memory before one atomic add per table entry into the
+//     workspace's fp32 table.
+//  2. bwd_key_kernel, one warp per real key (lane = channel): walks the key's
 //     inverse neighbourhood (the queries whose clamped window holds it: per
-//     axis a contiguous range of group positions, up to k + k/2 long at the
-//     edges), recomputes p = exp(s - lse) and ds from the stored statistics
-//     and accumulates dk and dv in registers; no atomics.
+//     axis a contiguous range of group positions, up to 2k - 1 long),
+//     recomputes p = exp(s - lse) and ds from the stored statistics and
+//     accumulates dk and dv in registers; no atomics.
 //  3. bwd_rpb_kernel rounds the fp32 bias gradient to the bias dtype.
 // The workspace is [lse, delta] per query (8 bytes per query and head) plus
 // the fp32 table (heads * (2k-1)^2 floats), zeroed by bwd_zero_kernel first.
@@ -37,33 +41,11 @@
 namespace na2d {
 namespace {
 
-constexpr int kD = 32;                    // head dim
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kQPB = 128;                 // queries per block in the query pass
 constexpr int kMaxPerLane = (13 * 13 + 31) / 32;
 constexpr int kMaxTab = 25 * 25;          // (2k-1)^2 for k <= 13
-
-template <typename T> __device__ __forceinline__ void load_row(const T *p, float (&x)[kD]) {
-    constexpr int kPer16 = 16 / sizeof(T);
-    const uint4 *p4 = reinterpret_cast<const uint4 *>(p);
-#pragma unroll
-    for (int c = 0; c < kD / kPer16; ++c) {
-        uint4 u = __ldg(p4 + c);
-        const T *e = reinterpret_cast<const T *>(&u);
-#pragma unroll
-        for (int t = 0; t < kPer16; ++t) x[c * kPer16 + t] = Elem<T>::to_f(e[t]);
-    }
-}
-
-template <typename T> __device__ __forceinline__ float dot_row(const float (&a)[kD], const T *p) {
-    float b[kD];
-    load_row<T>(p, b);
-    float s = 0.f;
-#pragma unroll
-    for (int c = 0; c < kD; ++c) s = fmaf(a[c], b[c], s);
-    return s;
-}
 
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
@@ -76,15 +58,40 @@ __device__ __forceinline__ float warp_max(float x) {
     return x;
 }
 
+// a . row over D channels: a from shared memory (fp32), the row from global
+// memory in 16-byte pieces (the row start is 16-byte aligned).
+template <typename T, int D> __device__ __forceinline__ float dot_s(const float *a, const T *row) {
+    constexpr int kPer16 = 16 / sizeof(T);
+    const uint4 *p4 = reinterpret_cast<const uint4 *>(row);
+    float s = 0.f;
+#pragma unroll
+    for (int c = 0; c < D / kPer16; ++c) {
+        const uint4 u = __ldg(p4 + c);
+        const T *e = reinterpret_cast<const T *>(&u);
+#pragma unroll
+        for (int t = 0; t < kPer16; ++t) s = fmaf(a[c * kPer16 + t], Elem<T>::to_f(e[t]), s);
+    }
+    return s;
+}
+
 struct BwdArgs {
-    const void *q, *k, *v, *rpb, *dout;
-    void *dq, *dk, *dv, *drpb;
+    View q, k, v, g, dq, dk, dv;
+    const void *rpb;
+    void *drpb;
     float *lse, *delta, *tab;    // workspace
-    int heads, H, W, K, d;
-    int64_t nq;                  // B * heads * H * W
+    int heads, H, W, Hp, Wp, K, d;
+    int64_t nq;                  // B * heads * H * W (real queries)
     int qblocks;                 // query-pass blocks per image
     float scale;                 // 1 / sqrt(D)
+    bool dropout;
+    uint32_t drop_thresh;
+    float drop_scale;
+    uint64_t seed, offset;
 };
+
+template <typename T> __device__ __forceinline__ const T *at(const View &x, int64_t b, int h, int y, int xx) {
+    return static_cast<const T *>(x.p) + b * x.sb + h * x.sh + y * x.sy + xx * x.sx;
+}
 
 // ---------------------------------------------------------------------------
 __global__ void bwd_zero_kernel(float *tab, int n) {
@@ -92,30 +99,34 @@ __global__ void bwd_zero_kernel(float *tab, int n) {
 }
 
 // ---------------------------------------------------------------------------
-// Pass 1: block (image bh, chunk) takes queries [chunk * kQPB, +kQPB) of
+// Pass 1: block (image bh, chunk) takes real queries [chunk * kQPB, +kQPB) of
 // image bh, one warp per query at a time.
-template <typename T>
+template <typename T, int D>
 __global__ void __launch_bounds__(kThreads) bwd_query_kernel(const BwdArgs a) {
     __shared__ float bins[kMaxTab];
+    __shared__ float qs[kWarps][D], gs[kWarps][D];
+    constexpr int NC = (D + 31) / 32;
     const int K = a.K, d = a.d, H = a.H, W = a.W, KK = K * K, nb = 2 * K - 1;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t bh = blockIdx.x / a.qblocks;
     const int chunk = (int)(blockIdx.x - bh * a.qblocks);
+    const int64_t b = bh / a.heads;
     const int h = (int)(bh % a.heads);
     for (int i = threadIdx.x; i < nb * nb; i += blockDim.x) bins[i] = 0.f;
     __syncthreads();
-    const T *q = static_cast<const T *>(a.q), *k = static_cast<const T *>(a.k), *v = static_cast<const T *>(a.v);
-    const T *g = static_cast<const T *>(a.dout);
     const T *bias = a.rpb ? static_cast<const T *>(a.rpb) + (size_t)h * nb * nb : nullptr;
-    const size_t plane = (size_t)bh * H * W;
     const int q_end = min(H * W, (chunk + 1) * kQPB);
     for (int qi = chunk * kQPB + warp; qi < q_end; qi += kWarps) {
         const int i = qi / W, j = qi - (qi / W) * W;
-        const int gy = i % d, iy = i / d, sy = window_start(iy, group_len(H, d, gy), K);
-        const int gx = j % d, ix = j / d, sx = window_start(ix, group_len(W, d, gx), K);
-        float qf[kD], gf[kD];
-        load_row<T>(q + (plane + qi) * kD, qf);
-        load_row<T>(g + (plane + qi) * kD, gf);
+        const int gy = i % d, iy = i / d, sy = window_start(iy, group_len(a.Hp, d, gy), K);
+        const int gx = j % d, ix = j / d, sx = window_start(ix, group_len(a.Wp, d, gx), K);
+        const T *qp = at<T>(a.q, b, h, i, j), *gp = at<T>(a.g, b, h, i, j);
+        for (int c = lane; c < D; c += 32) {
+            qs[warp][c] = Elem<T>::to_f(qp[c]);
+            gs[warp][c] = Elem<T>::to_f(gp[c]);
+        }
+        __syncwarp();
+        const int64_t qlin = bh * H * W + qi;
         float s[kMaxPerLane], dp[kMaxPerLane];
         float m = -FLT_MAX;
 #pragma unroll
@@ -125,11 +136,18 @@ __global__ void __launch_bounds__(kThreads) bwd_query_kernel(const BwdArgs a) {
             dp[r] = 0.f;
             if (n < KK) {
                 const int ty = n / K, tx = n - ty * K;
-                const size_t key = plane + (size_t)(gy + d * (sy + ty)) * W + (gx + d * (sx + tx));
-                float sv = dot_row<T>(qf, k + key * kD) * a.scale;
+                const int ky = gy + d * (sy + ty), kx = gx + d * (sx + tx);
+                float dot = 0.f;
+                if (ky < H && kx < W) {
+                    dot = dot_s<T, D>(qs[warp], at<T>(a.k, b, h, ky, kx));
+                    dp[r] = dot_s<T, D>(gs[warp], at<T>(a.v, b, h, ky, kx));
+                }
+                float sv = dot * a.scale;
                 if (bias) sv += Elem<T>::to_f(bias[(sy + ty - iy + K - 1) * nb + (sx + tx - ix + K - 1)]);
                 s[r] = sv;
-                dp[r] = dot_row<T>(gf, v + key * kD);
+                if (a.dropout)
+                    dp[r] = dropout_keep((uint64_t)qlin * KK + n, a.seed, a.offset, a.drop_thresh) ? dp[r] * a.drop_scale
+                                                                                                   : 0.f;
                 m = fmaxf(m, sv);
             }
         }
@@ -159,7 +177,9 @@ __global__ void __launch_bounds__(kThreads) bwd_query_kernel(const BwdArgs a) {
                 atomicAdd(&bins[(sy + ty - iy + K - 1) * nb + (sx + tx - ix + K - 1)], dp[r]);
             }
         }
-        float acc = 0.f;
+        float acc[NC];
+#pragma unroll
+        for (int jj = 0; jj < NC; ++jj) acc[jj] = 0.f;
 #pragma unroll
         for (int r = 0; r < kMaxPerLane; ++r) {
             if (32 * r >= KK) break;
@@ -168,15 +188,24 @@ __global__ void __launch_bounds__(kThreads) bwd_query_kernel(const BwdArgs a) {
                 const int n = 32 * r + tl;
                 const float dsn = __shfl_sync(0xffffffffu, dp[r], tl);
                 const int ty = n / K, tx = n - ty * K;
-                const size_t key = plane + (size_t)(gy + d * (sy + ty)) * W + (gx + d * (sx + tx));
-                acc = fmaf(dsn, Elem<T>::to_f(k[key * kD + lane]), acc);
+                const int ky = gy + d * (sy + ty), kx = gx + d * (sx + tx);
+                if (ky < H && kx < W) {
+                    const T *kp = at<T>(a.k, b, h, ky, kx);
+#pragma unroll
+                    for (int jj = 0; jj < NC; ++jj)
+                        if (lane + 32 * jj < D) acc[jj] = fmaf(dsn, Elem<T>::to_f(kp[lane + 32 * jj]), acc[jj]);
+                }
             }
         }
-        static_cast<T *>(a.dq)[(plane + qi) * kD + lane] = Elem<T>::from_f(acc * a.scale);
+        T *dqp = const_cast<T *>(at<T>(a.dq, b, h, i, j));
+#pragma unroll
+        for (int jj = 0; jj < NC; ++jj)
+            if (lane + 32 * jj < D) dqp[lane + 32 * jj] = Elem<T>::from_f(acc[jj] * a.scale);
         if (lane == 0) {
-            a.lse[plane + qi] = m + __logf(l);
-            a.delta[plane + qi] = delta;
+            a.lse[qlin] = m + __logf(l);
+            a.delta[qlin] = delta;
         }
+        __syncwarp();   // the next query overwrites this warp's staged rows
     }
     __syncthreads();
     for (int i = threadIdx.x; i < nb * nb; i += blockDim.x)
@@ -199,51 +228,82 @@ __device__ __forceinline__ void inverse_range(int jp, int Lg, int K, int *lo, in
     *hi = b;
 }
 
-// Pass 2: one warp per key pixel (b, head, y, x), lane = channel.
-template <typename T>
+// Pass 2: one warp per real key pixel (b, head, y, x), lane = channel(s).
+template <typename T, int D>
 __global__ void __launch_bounds__(kThreads) bwd_key_kernel(const BwdArgs a) {
-    const int K = a.K, d = a.d, H = a.H, W = a.W, nb = 2 * K - 1;
+    constexpr int NC = (D + 31) / 32;
+    const int K = a.K, d = a.d, H = a.H, W = a.W, nb = 2 * K - 1, KK = K * K;
     const int lane = threadIdx.x & 31;
-    const T *q = static_cast<const T *>(a.q), *k = static_cast<const T *>(a.k), *v = static_cast<const T *>(a.v);
-    const T *g = static_cast<const T *>(a.dout);
     const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
     for (int64_t idx = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5; idx < a.nq; idx += nwarps) {
         const int x = (int)(idx % W);
         const int64_t t = idx / W;
         const int y = (int)(t % H);
         const int64_t bh = t / H;
+        const int64_t b = bh / a.heads;
         const int h = (int)(bh % a.heads);
         const T *bias = a.rpb ? static_cast<const T *>(a.rpb) + (size_t)h * nb * nb : nullptr;
-        const size_t plane = (size_t)bh * H * W;
-        const int gy = y % d, jy = y / d, Lgy = group_len(H, d, gy);
-        const int gx = x % d, jx = x / d, Lgx = group_len(W, d, gx);
+        const int gy = y % d, jy = y / d, Lgy = group_len(a.Hp, d, gy);
+        const int gx = x % d, jx = x / d, Lgx = group_len(a.Wp, d, gx);
         int ylo, yhi, xlo, xhi;
         inverse_range(jy, Lgy, K, &ylo, &yhi);
         inverse_range(jx, Lgx, K, &xlo, &xhi);
-        const float kc = Elem<T>::to_f(k[idx * kD + lane]), vc = Elem<T>::to_f(v[idx * kD + lane]);
-        float dk = 0.f, dv = 0.f;
+        const T *kp = at<T>(a.k, b, h, y, x), *vp = at<T>(a.v, b, h, y, x);
+        float kc[NC], vc[NC], dk[NC], dv[NC];
+#pragma unroll
+        for (int jj = 0; jj < NC; ++jj) {
+            const bool on = lane + 32 * jj < D;
+            kc[jj] = on ? Elem<T>::to_f(kp[lane + 32 * jj]) : 0.f;
+            vc[jj] = on ? Elem<T>::to_f(vp[lane + 32 * jj]) : 0.f;
+            dk[jj] = dv[jj] = 0.f;
+        }
         for (int iy = ylo; iy <= yhi; ++iy) {
             const int qy = gy + d * iy;
+            if (qy >= H) break;                   // padded query rows: no gradient
             const int by = jy - iy + K - 1;
+            const int ty = jy - window_start(iy, Lgy, K);
             for (int ix = xlo; ix <= xhi; ++ix) {
-                const size_t qi = plane + (size_t)qy * W + (gx + d * ix);
-                const float qc = Elem<T>::to_f(q[qi * kD + lane]), gc = Elem<T>::to_f(g[qi * kD + lane]);
-                float sdot = qc * kc, pdot = gc * vc;
+                const int qx = gx + d * ix;
+                if (qx >= W) break;
+                const T *qp = at<T>(a.q, b, h, qy, qx), *gp = at<T>(a.g, b, h, qy, qx);
+                float qc[NC], gc[NC], sdot = 0.f, pdot = 0.f;
+#pragma unroll
+                for (int jj = 0; jj < NC; ++jj) {
+                    const bool on = lane + 32 * jj < D;
+                    qc[jj] = on ? Elem<T>::to_f(qp[lane + 32 * jj]) : 0.f;
+                    gc[jj] = on ? Elem<T>::to_f(gp[lane + 32 * jj]) : 0.f;
+                    sdot = fmaf(qc[jj], kc[jj], sdot);
+                    pdot = fmaf(gc[jj], vc[jj], pdot);
+                }
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) {
                     sdot += __shfl_xor_sync(0xffffffffu, sdot, o);
                     pdot += __shfl_xor_sync(0xffffffffu, pdot, o);
                 }
+                const int64_t qlin = bh * H * W + (int64_t)qy * W + qx;
                 float sv = sdot * a.scale;
                 if (bias) sv += Elem<T>::to_f(bias[by * nb + (jx - ix + K - 1)]);
-                const float p = __expf(sv - a.lse[qi]);
-                const float ds = p * (pdot - a.delta[qi]);
-                dv = fmaf(p, gc, dv);
-                dk = fmaf(ds, qc, dk);
+                const float p = __expf(sv - a.lse[qlin]);
+                float z = 1.f;
+                if (a.dropout) {
+                    const int n = ty * K + (jx - window_start(ix, Lgx, K));
+                    z = dropout_keep((uint64_t)qlin * KK + n, a.seed, a.offset, a.drop_thresh) ? a.drop_scale : 0.f;
+                }
+                const float ds = p * (z * pdot - a.delta[qlin]);
+#pragma unroll
+                for (int jj = 0; jj < NC; ++jj) {
+                    dv[jj] = fmaf(p * z, gc[jj], dv[jj]);
+                    dk[jj] = fmaf(ds, qc[jj], dk[jj]);
+                }
             }
         }
-        static_cast<T *>(a.dk)[idx * kD + lane] = Elem<T>::from_f(dk * a.scale);
-        static_cast<T *>(a.dv)[idx * kD + lane] = Elem<T>::from_f(dv);
+        T *dkp = const_cast<T *>(at<T>(a.dk, b, h, y, x)), *dvp = const_cast<T *>(at<T>(a.dv, b, h, y, x));
+#pragma unroll
+        for (int jj = 0; jj < NC; ++jj)
+            if (lane + 32 * jj < D) {
+                dkp[lane + 32 * jj] = Elem<T>::from_f(dk[jj] * a.scale);
+                dvp[lane + 32 * jj] = Elem<T>::from_f(dv[jj]);
+            }
     }
 }
 
@@ -259,14 +319,23 @@ int grid_for(int64_t threads) {
     return (int)(g < 1 ? 1 : (g > cap ? cap : g));
 }
 
-template <typename T> cudaError_t launch_bwd_t(const BwdArgs &a, int64_t bh, cudaStream_t st) {
+template <typename T, int D> cudaError_t launch_bwd_t(const BwdArgs &a, int64_t bh, cudaStream_t st) {
     const int ntab = a.heads * (2 * a.K - 1) * (2 * a.K - 1);
     bwd_zero_kernel<<<grid_for(ntab), kThreads, 0, st>>>(a.tab, ntab);
-    bwd_query_kernel<T><<<(unsigned)(bh * a.qblocks), kThreads, 0, st>>>(a);
-    bwd_key_kernel<T><<<grid_for(a.nq * 32), kThreads, 0, st>>>(a);
+    bwd_query_kernel<T, D><<<(unsigned)(bh * a.qblocks), kThreads, 0, st>>>(a);
+    bwd_key_kernel<T, D><<<grid_for(a.nq * 32), kThreads, 0, st>>>(a);
     if (a.drpb) bwd_rpb_kernel<T><<<grid_for(ntab), kThreads, 0, st>>>(a.tab, static_cast<T *>(a.drpb), ntab);
     note_kernel("bwd_query_kernel+bwd_key_kernel");
     return cudaGetLastError();
+}
+
+template <typename T> cudaError_t launch_bwd_d(const BwdArgs &a, int D, int64_t bh, cudaStream_t st) {
+    switch (D) {
+    case 16: return launch_bwd_t<T, 16>(a, bh, st);
+    case 32: return launch_bwd_t<T, 32>(a, bh, st);
+    case 64: return launch_bwd_t<T, 64>(a, bh, st);
+    default: return launch_bwd_t<T, 128>(a, bh, st);
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -294,28 +363,41 @@ size_t backward_workspace_bytes(const Problem &p) {
     return (2 * nq + ntab) * sizeof(float);
 }
 
-cudaError_t launch_backward(const Problem &p, const void *q, const void *k, const void *v, const void *rpb,
-                            const void *dout, void *dq, void *dk, void *dv, void *drpb, void *workspace,
-                            cudaStream_t st) {
+cudaError_t launch_backward_views(const Problem &p, const View &q, const View &k, const View &v, const void *rpb,
+                                  const View &dout, const View &dq, const View &dk, const View &dv, void *drpb,
+                                  const Dropout &drop, void *workspace, cudaStream_t st) {
     BwdArgs a;
-    a.q = q; a.k = k; a.v = v; a.rpb = rpb; a.dout = dout;
-    a.dq = dq; a.dk = dk; a.dv = dv; a.drpb = drpb;
+    a.q = q; a.k = k; a.v = v; a.g = dout; a.dq = dq; a.dk = dk; a.dv = dv;
+    a.rpb = rpb; a.drpb = drpb;
     a.nq = p.bh() * p.H * p.W;
     float *ws = static_cast<float *>(workspace);
     a.lse = ws;
     a.delta = ws + a.nq;
     a.tab = ws + 2 * a.nq;
-    a.heads = p.heads; a.H = p.H; a.W = p.W; a.K = p.k; a.d = p.d;
+    a.heads = p.heads; a.H = p.H; a.W = p.W; a.Hp = p.Hp(); a.Wp = p.Wp(); a.K = p.k; a.d = p.d;
     a.qblocks = (p.H * p.W + kQPB - 1) / kQPB;
     a.scale = 1.0f / sqrtf((float)p.D);
+    a.dropout = drop.p > 0.f;
+    const double th = (double)drop.p * 4294967296.0;
+    a.drop_thresh = th >= 4294967295.0 ? 0xFFFFFFFFu : (uint32_t)(th + 0.5);
+    a.drop_scale = a.dropout ? 1.0f / (1.0f - drop.p) : 1.0f;
+    a.seed = drop.seed;
+    a.offset = drop.offset;
     if (p.bh() * a.qblocks >= INT32_MAX) return cudaErrorInvalidConfiguration;
     switch (p.dtype) {
-    case DType::F32: return launch_bwd_t<float>(a, p.bh(), st);
-    case DType::F16: return launch_bwd_t<__half>(a, p.bh(), st);
-    default: return launch_bwd_t<__nv_bfloat16>(a, p.bh(), st);
+    case DType::F32: return launch_bwd_d<float>(a, p.D, p.bh(), st);
+    case DType::F16: return launch_bwd_d<__half>(a, p.D, p.bh(), st);
+    default: return launch_bwd_d<__nv_bfloat16>(a, p.D, p.bh(), st);
     }
 }
 
+cudaError_t launch_backward(const Problem &p, const void *q, const void *k, const void *v, const void *rpb,
+                            const void *dout, void *dq, void *dk, void *dv, void *drpb, void *workspace,
+                            cudaStream_t st) {
+    return launch_backward_views(p, View::contiguous(q, p), View::contiguous(k, p), View::contiguous(v, p), rpb,
+                                 View::contiguous(dout, p), View::contiguous(dq, p), View::contiguous(dk, p),
+                                 View::contiguous(dv, p), drpb, Dropout{0.f, 0, 0}, workspace, st);
+}
 
 size_t noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
 

@@ -118,4 +118,38 @@ __device__ __forceinline__ float ex2(float x) {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
+// ---------------------------------------------------------------------------
+// Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As
+// Easy as 1, 2, 3", SC 2011): a counter-based generator, 10 rounds of the
+// 4x32 round function with the published multipliers and Weyl key
+// increments.  Attention dropout draws one 32-bit word per attention weight.
+// ---------------------------------------------------------------------------
+__host__ __device__ __forceinline__ void philox4x32_10(uint32_t (&c)[4], uint32_t k0, uint32_t k1) {
+    for (int r = 0; r < 10; ++r) {
+        if (r) {
+            k0 += 0x9E3779B9u;
+            k1 += 0xBB67AE85u;
+        }
+        const uint64_t p0 = (uint64_t)0xD2511F53u * c[0], p1 = (uint64_t)0xCD9E8D57u * c[2];
+        const uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
+        const uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
+        const uint32_t n0 = hi1 ^ c[1] ^ k0, n2 = hi0 ^ c[3] ^ k1;
+        c[0] = n0;
+        c[1] = lo1;
+        c[2] = n2;
+        c[3] = lo0;
+    }
+}
+
+// Dropout decision for attention weight number e (the weight's linear index
+// in the [B, heads, H, W, k*k] tensor): word e % 4 of Philox(counter =
+// (e / 4 low, e / 4 high, offset low, offset high), key = seed), as a
+// fraction u = word / 2^32; the weight is kept when u >= p.
+__host__ __device__ __forceinline__ bool dropout_keep(uint64_t e, uint64_t seed, uint64_t offset, uint32_t thresh) {
+    const uint64_t blk = e >> 2;
+    uint32_t c[4] = {(uint32_t)blk, (uint32_t)(blk >> 32), (uint32_t)offset, (uint32_t)(offset >> 32)};
+    philox4x32_10(c, (uint32_t)seed, (uint32_t)(seed >> 32));
+    return c[e & 3] >= thresh;
+}
+
 }  // namespace na2d

@@ -13,15 +13,41 @@ struct Problem {
     int B, heads, H, W, D, k, d;
     DType dtype;
     int64_t bh() const { return (int64_t)B * heads; }
+    // padded map (maps shorter than k*d are padded with zero pixels at the
+    // bottom / right and the output cropped)
+    int Hp() const { return H > k * d ? H : k * d; }
+    int Wp() const { return W > k * d ? W : k * d; }
+};
+
+// A [B, heads, H, W, D] tensor given by element strides; channels contiguous.
+struct View {
+    const void *p;
+    int64_t sb, sh, sy, sx;
+    static View contiguous(const void *ptr, const Problem &pr) {
+        const int64_t sx = pr.D, sy = (int64_t)pr.W * sx, sh = (int64_t)pr.H * sy, sb = (int64_t)pr.heads * sh;
+        return View{ptr, sb, sh, sy, sx};
+    }
+    bool is_contiguous(const Problem &pr) const {
+        const View c = contiguous(p, pr);
+        return sb == c.sb && sh == c.sh && sy == c.sy && sx == c.sx;
+    }
+};
+
+// Attention dropout: probability p (0: none), Philox key and counter offset.
+struct Dropout {
+    float p;
+    uint64_t seed, offset;
 };
 
 // Fused forward on the tensor cores (f16 / bf16, D = 32, k in 3..13).
 cudaError_t launch_forward_tc(const Problem &p, const void *q, const void *k, const void *v,
                               const void *rpb, void *out, cudaStream_t stream);
 
-// Fused forward on the CUDA cores (any dtype, D = 32, any odd k <= 13).
-cudaError_t launch_forward_simt(const Problem &p, const void *q, const void *k, const void *v,
-                                const void *rpb, void *out, cudaStream_t stream);
+// Fused forward on the CUDA cores: any dtype, D in {16, 32, 64, 128}, any
+// odd k <= 13, strided views, padded short maps; optionally writes the
+// (dropped-out) attention weights to attn and applies dropout.
+cudaError_t launch_forward_simt(const Problem &p, const View &q, const View &k, const View &v, const void *rpb,
+                                const View &out, float *attn, const Dropout &drop, cudaStream_t stream);
 
 // Split path.
 cudaError_t launch_qk_rpb(const Problem &p, const void *q, const void *k, const void *rpb, float *attn,
@@ -35,6 +61,10 @@ size_t backward_workspace_bytes(const Problem &p);
 cudaError_t launch_backward(const Problem &p, const void *q, const void *k, const void *v, const void *rpb,
                             const void *dout, void *dq, void *dk, void *dv, void *drpb, void *workspace,
                             cudaStream_t stream);
+// The same on strided views, with attention dropout.
+cudaError_t launch_backward_views(const Problem &p, const View &q, const View &k, const View &v, const void *rpb,
+                                  const View &dout, const View &dq, const View &dk, const View &dv, void *drpb,
+                                  const Dropout &drop, void *workspace, cudaStream_t stream);
 
 // The backward with the library's built-in scratch array instead of a
 // caller workspace (no allocation); problems whose workspace exceeds

@@ -1016,7 +1016,9 @@ bool encode_group_map(CUtensorMap *map, const void *base, DType dt, int64_t bh, 
 }
 
 bool tc_supported(const Problem &p) {
-    return (p.dtype == DType::F16 || p.dtype == DType::BF16) && p.D == 32 && p.k >= 3 && p.k <= 13 && (p.k & 1);
+    // every dilation group at least k long (no padded map)
+    return (p.dtype == DType::F16 || p.dtype == DType::BF16) && p.D == 32 && p.k >= 3 && p.k <= 13 && (p.k & 1) &&
+           (int64_t)p.k * p.d <= p.H && (int64_t)p.k * p.d <= p.W;
 }
 
 cudaError_t launch_forward_tc(const Problem &p, const void *q, const void *k, const void *v, const void *rpb,

@@ -25,9 +25,8 @@ FAKE2 = 0x200000
 BAD_PROBLEMS = [
     (dict(k=6), 4), (dict(k=0), 4), (dict(k=15), 4), (dict(k=-3), 4),
     (dict(d=0), 5), (dict(d=-1), 5),
-    (dict(H=13, d=2), 3), (dict(W=13, d=2), 3), (dict(H=6), 3), (dict(W=6), 3),
-    (dict(H=0), 3), (dict(B=-1), 3), (dict(heads=-2), 3),
-    (dict(D=64), 3), (dict(D=16), 3),
+    (dict(H=0), 3), (dict(W=0), 3), (dict(B=-1), 3), (dict(heads=-2), 3),
+    (dict(D=48), 3), (dict(D=256), 3), (dict(D=8), 3),
     (dict(dtype=7), 2),
     (dict(H=1 << 20, W=1 << 20, k=1), 3),  # plane too large
 ]
@@ -80,6 +79,33 @@ def _host_checks() -> dict:
     r["bwd_alias_ws"] = _native.backward_ptr(p, F[0], F[1], F[2], None, F[7], F[3], F[4], F[5], None, F[7], ws)
     r["bwd_bad_k"] = _native.backward_ptr(prob(k=4), F[0], F[1], F[2], None, F[7], F[3], F[4], F[5], None, F[6], ws)
     r["bwd_empty"] = _native.backward_ptr(prob(B=0), 0, 0, 0, None, 0, 0, 0, 0, None, 0, 0)
+    # forward_ex: strided views, weights, dropout
+    import ctypes
+    def T(ptr, sb=2 * 14 * 14 * 32, sh=14 * 14 * 32, sy=14 * 32, sx=32):
+        return _native.Tensor(ptr, sb, sh, sy, sx)
+    def fx(q, k, v, out, attn=None, drop=None, pp=None):
+        return L.na2d_forward_ex(ctypes.byref(pp or p), ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), None,
+                                 ctypes.byref(out), attn, None if drop is None else ctypes.byref(drop), None)
+    r["fx_null"] = fx(T(0), T(F[1]), T(F[2]), T(F[3]))
+    r["fx_stride_align"] = fx(T(F[0], sx=36), T(F[1]), T(F[2]), T(F[3]))
+    r["fx_neg_stride"] = fx(T(F[0], sy=-448), T(F[1]), T(F[2]), T(F[3]))
+    r["fx_out_self_overlap"] = fx(T(F[0]), T(F[1]), T(F[2]), T(F[3], sx=16))
+    r["fx_out_on_input"] = fx(T(F[0]), T(F[1]), T(F[2]), T(F[0]))
+    r["fx_attn_on_input"] = fx(T(F[0]), T(F[1]), T(F[2]), T(F[3]), attn=F[1])
+    r["fx_drop_p"] = fx(T(F[0]), T(F[1]), T(F[2]), T(F[3]), drop=_native.Dropout(1.0, 1, 0))
+    r["fx_drop_neg"] = fx(T(F[0]), T(F[1]), T(F[2]), T(F[3]), drop=_native.Dropout(-0.1, 1, 0))
+    r["fx_empty"] = fx(T(0), T(0), T(0), T(0), pp=prob(B=0))
+    # one fused channels-last buffer: q, k, v views 2 * 32 elements apart per
+    # head block, the output interleaved with them in a fourth slot is refused
+    # only when it lands on an input block
+    P3 = dict(sb=14 * 14 * 4 * 64, sh=32, sy=14 * 4 * 64, sx=4 * 64)
+    base = F[0]
+    r["fx_fused_ok"] = L.na2d_forward_ex(ctypes.byref(p), ctypes.byref(T(base, **P3)),
+                                         ctypes.byref(T(base + 128, **P3)), ctypes.byref(T(base + 256, **P3)), None,
+                                         ctypes.byref(T(base + 384, **P3)), None, None, None)
+    r["fx_fused_clash"] = L.na2d_forward_ex(ctypes.byref(p), ctypes.byref(T(base, **P3)),
+                                            ctypes.byref(T(base + 128, **P3)), ctypes.byref(T(base + 256, **P3)),
+                                            None, ctypes.byref(T(base + 192, **P3)), None, None, None)
     return r
 
 
@@ -92,6 +118,13 @@ def host_results():
     out = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=300)
     assert out.returncode == 0, out.stderr
     return json.loads(out.stdout.strip().splitlines()[-1])
+
+
+def test_fused_views_pass_the_host_checks(host_results):
+    """Interleaved q / k / v / out views of one fused buffer pass every host
+    check; with no device the call then fails only at the launch
+    (NA2D_ERR_CUDA), never with an argument error."""
+    assert host_results["fx_fused_ok"] == 8
 
 
 def test_backward_workspace_size(host_results):
@@ -138,6 +171,8 @@ def test_forward_rejects_bad_problems(host_results, i):
     ("empty_B", 0), ("empty_heads", 0), ("empty_qk", 0), ("empty_softmax", 0), ("empty_av", 0), ("faults_null", 1),
     ("bwd_null_dout", 1), ("bwd_null_ws", 1), ("bwd_small_ws", 3), ("bwd_align", 6), ("bwd_alias_in", 7),
     ("bwd_alias_out", 7), ("bwd_alias_ws", 7), ("bwd_bad_k", 4), ("bwd_empty", 0),
+    ("fx_null", 1), ("fx_stride_align", 6), ("fx_neg_stride", 6), ("fx_out_self_overlap", 7), ("fx_out_on_input", 7),
+    ("fx_attn_on_input", 7), ("fx_drop_p", 3), ("fx_drop_neg", 3), ("fx_empty", 0), ("fx_fused_clash", 7),
 ])
 def test_host_checks(host_results, case, status):
     assert host_results[case] == status
