@@ -434,6 +434,12 @@ def run_ours(args, world, rank, local):
             del s2
         torch.cuda.empty_cache()
 
+    # ---- the other calls of the library on NAT-Tiny stage-1-sized inputs (1 GPU)
+    ext = {}
+    if world == 1 and not args.no_per_workload:
+        ext = time_extensions(dev, l2, args.warmup)
+        torch.cuda.empty_cache()
+
     # ---- end to end through the public API: pinned host -> device, forward, device -> host
     e2e = run_e2e(args, wl, dev, rank, world, pg)
 
@@ -451,6 +457,8 @@ def run_ours(args, world, rank, local):
     }
     if per_wl:
         line["per_workload"] = per_wl
+    if ext:
+        line["extensions"] = ext
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
     if pg:
@@ -458,6 +466,135 @@ def run_ours(args, world, rank, local):
         pg.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def time_calls(fn, n_sets, warmup, dev, min_seconds=0.2):
+    """Median time of one call of fn(i) (i rotates over n_sets input sets),
+    replayed from a CUDA graph of 20 calls, CUDA events on the stream."""
+    import torch
+    stream = torch.cuda.Stream(dev)
+    stream.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(stream):
+        for i in range(max(warmup, 3)):
+            fn(i)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(20):
+                fn(i)
+        g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        runs, total = [], 0.0
+        while len(runs) < 5 or total < min_seconds * 1e3:
+            a.record(stream)
+            g.replay()
+            b.record(stream)
+            b.synchronize()
+            ms = a.elapsed_time(b)
+            runs.append(ms / 20)
+            total += ms
+    torch.cuda.synchronize()
+    del g
+    return statistics.median(runs)
+
+
+def time_extensions(dev, l2, warmup):
+    """Times the library's other calls at the NAT-Tiny stage-1 size (B=32,
+    heads=2, 56x56, D=32, k=7, d=1; fp16 unless noted), rotating input sets
+    beyond 3x L2: the backward; the forward read in place from a channels-last
+    fused q/k/v buffer; the forward returning the attention weights with
+    dropout p=0.1; a D=64 forward (heads=1 so the bytes match); a map
+    shorter than k*d (DiNAT stage-4-sized 7x7 with dilation 2, padded to
+    14x14, B=128 heads=16 bf16).  HBM fraction against the measured copy
+    bandwidth, on the bytes each call must move."""
+    import torch
+    import neighborhood_attention_na2d_b200 as na
+    from neighborhood_attention_na2d_b200.inputs import Shape
+
+    peak, _ = hbm_peak()
+    out = {}
+    nat = Shape(32, 2, 56, 56, 32, 7, 1, "f16", 1)
+    qh = nat.queries_heads
+    tensor = qh * 64                                          # one [B,heads,H,W,32] fp16 tensor
+
+    def sets(shape, n_extra=0):
+        R = max(2, math.ceil(3 * l2 / (4 * shape.queries_heads * shape.D * 2)))
+        res = []
+        for r in range(R):
+            q, k, v, rpb = (t.to(dev) for t in make_inputs(shape, shape.seed + 1000 * r))
+            res.append([q, k, v, rpb] + [torch.randn_like(q) for _ in range(n_extra)])
+        return res
+
+    def record(name, shape, ms, moved, kernel, note):
+        out[name] = {"ms_per_call": ms, "value": shape.queries_heads / (ms / 1e3), "unit": UNIT,
+                     "achieved_gbs": moved / (ms / 1e3) / 1e9, "frac": moved / (ms / 1e3) / 1e9 / peak,
+                     "bytes_per_call": moved, "kernel": kernel, "shape": shape.describe(), "note": note}
+
+    # backward
+    S = sets(nat, 1)
+    ws = torch.empty(na.backward_workspace_size(na.make_problem(S[0][0].shape, 7, 1, S[0][0].dtype)),
+                     dtype=torch.uint8, device=dev)
+    grads = [torch.empty_like(S[0][0]) for _ in range(3)] + [torch.empty_like(S[0][3])]
+
+    def bwd(i):
+        q, k, v, rpb, g = S[i % len(S)]
+        na.na2d_backward(q, k, v, rpb, g, 7, 1, *grads, workspace=ws)
+    ms = time_calls(bwd, len(S), warmup, dev)
+    record("backward", nat, ms, 7 * tensor + 2 * 8 * qh, na.na2d_last_kernel(),
+           "reads q, k, v, dout; writes dq, dk, dv; 8 bytes per query of statistics written and read")
+    del S, ws, grads
+
+    # channels-last fused q/k/v, read in place
+    R = max(2, math.ceil(3 * l2 / (4 * tensor)))
+    bufs = [(torch.randn(32, 56, 56, 3 * 2 * 32, device=dev).half(), torch.empty(32, 56, 56, 64, device=dev).half())
+            for _ in range(R)]
+    rpb = (torch.randn(2, 13, 13, device=dev) * 0.02).half()
+
+    def qkv(i):
+        x, o = bufs[i % R]
+        na.na2d_qkv_packed(x, rpb, 7, 1, 2, out=o)
+    ms = time_calls(qkv, R, warmup, dev)
+    record("fused_qkv_channels_last", nat, ms, 4 * tensor, na.na2d_last_kernel(),
+           "q, k, v strided views of one (B, H, W, 3*heads*D) buffer, output (B, H, W, heads*D)")
+    del bufs
+
+    # weights out + dropout
+    S = sets(nat)
+    outs = torch.empty_like(S[0][0])
+
+    def wdrop(i):
+        q, k, v, rpb = S[i % len(S)]
+        na.na2d_forward_ex(q, k, v, rpb, 7, 1, out=outs, return_attn=True, dropout_p=0.1, seed=i)
+    ms = time_calls(wdrop, len(S), warmup, dev)
+    record("weights_and_dropout", nat, ms, 4 * tensor + qh * 49 * 4, na.na2d_last_kernel(),
+           "attention dropout p=0.1 (Philox mask) and the fp32 weights [B, heads, H, W, 49] written")
+    del S, outs
+
+    # D = 64
+    d64 = Shape(32, 1, 56, 56, 64, 7, 1, "f16", 5)
+    S = sets(d64)
+    o64 = torch.empty_like(S[0][0])
+
+    def f64(i):
+        q, k, v, rpb = S[i % len(S)]
+        na.na2d_forward(q, k, v, rpb, 7, 1, out=o64)
+    ms = time_calls(f64, len(S), warmup, dev)
+    record("head_dim_64", d64, ms, 4 * d64.queries_heads * 128, na.na2d_last_kernel(), "D = 64")
+    del S, o64
+
+    # padded short map
+    pad = Shape(128, 16, 7, 7, 32, 7, 2, "bf16", 6)
+    S = sets(pad)
+    op = torch.empty_like(S[0][0])
+
+    def fpad(i):
+        q, k, v, rpb = S[i % len(S)]
+        na.na2d_forward(q, k, v, rpb, 7, 2, out=op)
+    ms = time_calls(fpad, len(S), warmup, dev)
+    record("padded_short_map", pad, ms, 4 * pad.queries_heads * 64, na.na2d_last_kernel(),
+           "7x7 map with k=7, d=2: zero-padded to 14x14 and cropped")
+    return out
 
 
 # workloads timed beside the headline in a 1-GPU run (the second stage-1

@@ -248,6 +248,18 @@ NA2D_API int na2d_version(void);
  * the tests to record which kernel each problem shape reaches. */
 NA2D_API const char *na2d_last_kernel(void);
 
+/* Test hook for the error path of the bounded waits.  The streaming kernel
+ * (the k = 7 sliding-window forward) waits for its copies with a limit; when
+ * a wait runs out the kernel counts the event (see na2d_device_faults), stops
+ * issuing and computing, waits for its copies already in flight (always with
+ * the full limit, so nothing lands in released shared memory), and returns;
+ * the outputs of that call are then unspecified.  This call shortens the
+ * data waits' limit to sm_clocks for the calls that follow on any thread
+ * (0 restores the default, about 2^31 clocks).  A limit of a few hundred
+ * clocks makes a wait run out on purpose without any device fault; tests use
+ * it to run the error path. */
+NA2D_API void na2d_debug_set_wait_limit(long long sm_clocks);
+
 #ifdef __cplusplus
 }
 #endif

@@ -167,7 +167,8 @@ na2d_status na2d_forward(const na2d_problem *p, const void *q, const void *k, co
         bool launched = false;
         cudaError_t e = na2d::launch_forward_umma(pr, q, k, v, rpb, out, st, &launched);
         if (e != cudaSuccess || launched) return from_cuda(e);
-        e = na2d::launch_forward_stream(pr, q, k, v, rpb, out, st, &launched);
+        e = na2d::launch_forward_stream(pr, View::contiguous(q, pr), View::contiguous(k, pr), View::contiguous(v, pr),
+                                        rpb, View::contiguous(out, pr), st, &launched);
         if (e != cudaSuccess || launched) return from_cuda(e);
         return from_cuda(na2d::launch_forward_tc(pr, q, k, v, rpb, out, st));
     }
@@ -216,6 +217,13 @@ na2d_status na2d_forward_ex(const na2d_problem *p, const na2d_tensor *q, const n
     if (!attn && dr.p == 0.f && vq.is_contiguous(pr) && vk.is_contiguous(pr) && vv.is_contiguous(pr) &&
         vo.is_contiguous(pr))
         return na2d_forward(p, q->data, k->data, v->data, rpb, out->data, stream);
+    // strided views without the optional parts: the tensor-core kernels that
+    // read rows with strides
+    if (!attn && dr.p == 0.f && na2d::tc_supported(pr)) {
+        bool launched = false;
+        cudaError_t e = na2d::launch_forward_stream(pr, vq, vk, vv, rpb, vo, st, &launched);
+        if (e != cudaSuccess || launched) return from_cuda(e);
+    }
     return from_cuda(na2d::launch_forward_simt(pr, vq, vk, vv, rpb, vo, attn, dr, st));
 }
 
@@ -416,5 +424,7 @@ const char *na2d_status_str(na2d_status s) {
 int na2d_version(void) { return 200; }
 
 const char *na2d_last_kernel(void) { return t_last_kernel; }
+
+void na2d_debug_set_wait_limit(long long sm_clocks) { na2d::set_stream_wait_limit(sm_clocks); }
 
 }  // extern "C"

@@ -21,11 +21,12 @@
 //     covers queries of one (batch, head) image and sums its bias gradient in
 //     shared memory before one atomic add per table entry into the
 //     workspace's fp32 table.
-//  2. bwd_key_kernel, one warp per real key (lane = channel): walks the key's
-//     inverse neighbourhood (the queries whose clamped window holds it: per
-//     axis a contiguous range of group positions, up to 2k - 1 long),
-//     recomputes p = exp(s - lse) and ds from the stored statistics and
-//     accumulates dk and dv in registers; no atomics.
+//  2. bwd_key_kernel, one warp per real key: walks the key's inverse
+//     neighbourhood (the queries whose clamped window holds it: per axis a
+//     contiguous range of group positions, up to 2k - 1 long) 8 queries at a
+//     time (4 lanes per query, a quarter of the channels each), recomputes
+//     p = exp(s - lse) and ds from the stored statistics and accumulates dk
+//     and dv in registers; no atomics.
 //  3. bwd_rpb_kernel rounds the fp32 bias gradient to the bias dtype.
 // The workspace is [lse, delta] per query (8 bytes per query and head) plus
 // the fp32 table (heads * (2k-1)^2 floats), zeroed by bwd_zero_kernel first.
@@ -228,12 +229,18 @@ __device__ __forceinline__ void inverse_range(int jp, int Lg, int K, int *lo, in
     *hi = b;
 }
 
-// Pass 2: one warp per real key pixel (b, head, y, x), lane = channel(s).
+// Pass 2: one warp per real key pixel (b, head, y, x).  The key's inverse
+// neighbourhood (up to (2k - 1)^2 queries) is walked 8 queries at a time:
+// lanes 4s .. 4s + 3 take query slot s, each lane a quarter of the channels
+// (D / 4), so a query's dot products need two shuffle rounds.  Each lane
+// accumulates its quarter of dk and dv for its slot's queries; the 8 slots
+// are summed at the end (three shuffle rounds) and slot 0 writes.
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads) bwd_key_kernel(const BwdArgs a) {
-    constexpr int NC = (D + 31) / 32;
+    constexpr int QC = D / 4;                      // channels per lane
     const int K = a.K, d = a.d, H = a.H, W = a.W, nb = 2 * K - 1, KK = K * K;
-    const int lane = threadIdx.x & 31;
+    const int lane = threadIdx.x & 31, slot = lane >> 2, quarter = lane & 3;
+    const int c0 = quarter * QC;
     const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
     for (int64_t idx = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5; idx < a.nq; idx += nwarps) {
         const int x = (int)(idx % W);
@@ -248,62 +255,68 @@ __global__ void __launch_bounds__(kThreads) bwd_key_kernel(const BwdArgs a) {
         int ylo, yhi, xlo, xhi;
         inverse_range(jy, Lgy, K, &ylo, &yhi);
         inverse_range(jx, Lgx, K, &xlo, &xhi);
-        const T *kp = at<T>(a.k, b, h, y, x), *vp = at<T>(a.v, b, h, y, x);
-        float kc[NC], vc[NC], dk[NC], dv[NC];
+        // real queries only: the padded rows / columns come last in each range
+        yhi = min(yhi, (H - 1 - gy) / d);
+        xhi = min(xhi, (W - 1 - gx) / d);
+        const int nx = xhi - xlo + 1, cnt = (yhi - ylo + 1) * nx;
+        const T *kp = at<T>(a.k, b, h, y, x) + c0, *vp = at<T>(a.v, b, h, y, x) + c0;
+        float kc[QC], vc[QC], dk[QC], dv[QC];
 #pragma unroll
-        for (int jj = 0; jj < NC; ++jj) {
-            const bool on = lane + 32 * jj < D;
-            kc[jj] = on ? Elem<T>::to_f(kp[lane + 32 * jj]) : 0.f;
-            vc[jj] = on ? Elem<T>::to_f(vp[lane + 32 * jj]) : 0.f;
-            dk[jj] = dv[jj] = 0.f;
+        for (int c = 0; c < QC; ++c) {
+            kc[c] = Elem<T>::to_f(kp[c]);
+            vc[c] = Elem<T>::to_f(vp[c]);
+            dk[c] = dv[c] = 0.f;
         }
-        for (int iy = ylo; iy <= yhi; ++iy) {
-            const int qy = gy + d * iy;
-            if (qy >= H) break;                   // padded query rows: no gradient
-            const int by = jy - iy + K - 1;
-            const int ty = jy - window_start(iy, Lgy, K);
-            for (int ix = xlo; ix <= xhi; ++ix) {
-                const int qx = gx + d * ix;
-                if (qx >= W) break;
-                const T *qp = at<T>(a.q, b, h, qy, qx), *gp = at<T>(a.g, b, h, qy, qx);
-                float qc[NC], gc[NC], sdot = 0.f, pdot = 0.f;
+        for (int t0 = 0; t0 < cnt; t0 += 8) {
+            const int tq = t0 + slot;
+            const bool on = tq < cnt;
+            const int iy = ylo + (on ? tq / nx : 0), ix = xlo + (on ? tq % nx : 0);
+            const int qy = gy + d * iy, qx = gx + d * ix;
+            const T *qp = at<T>(a.q, b, h, qy, qx) + c0, *gp = at<T>(a.g, b, h, qy, qx) + c0;
+            float qc[QC], gc[QC], sdot = 0.f, pdot = 0.f;
 #pragma unroll
-                for (int jj = 0; jj < NC; ++jj) {
-                    const bool on = lane + 32 * jj < D;
-                    qc[jj] = on ? Elem<T>::to_f(qp[lane + 32 * jj]) : 0.f;
-                    gc[jj] = on ? Elem<T>::to_f(gp[lane + 32 * jj]) : 0.f;
-                    sdot = fmaf(qc[jj], kc[jj], sdot);
-                    pdot = fmaf(gc[jj], vc[jj], pdot);
-                }
+            for (int c = 0; c < QC; ++c) {
+                qc[c] = Elem<T>::to_f(qp[c]);
+                gc[c] = Elem<T>::to_f(gp[c]);
+                sdot = fmaf(qc[c], kc[c], sdot);
+                pdot = fmaf(gc[c], vc[c], pdot);
+            }
+            sdot += __shfl_xor_sync(0xffffffffu, sdot, 1);
+            pdot += __shfl_xor_sync(0xffffffffu, pdot, 1);
+            sdot += __shfl_xor_sync(0xffffffffu, sdot, 2);
+            pdot += __shfl_xor_sync(0xffffffffu, pdot, 2);
+            const int64_t qlin = bh * H * W + (int64_t)qy * W + qx;
+            float sv = sdot * a.scale;
+            if (bias) sv += Elem<T>::to_f(bias[(jy - iy + K - 1) * nb + (jx - ix + K - 1)]);
+            const float p = on ? __expf(sv - a.lse[qlin]) : 0.f;
+            float z = 1.f;
+            if (a.dropout && on) {
+                const int n = (jy - window_start(iy, Lgy, K)) * K + (jx - window_start(ix, Lgx, K));
+                z = dropout_keep((uint64_t)qlin * KK + n, a.seed, a.offset, a.drop_thresh) ? a.drop_scale : 0.f;
+            }
+            const float ds = on ? p * (z * pdot - a.delta[qlin]) : 0.f;
+            const float pz = p * z;
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    sdot += __shfl_xor_sync(0xffffffffu, sdot, o);
-                    pdot += __shfl_xor_sync(0xffffffffu, pdot, o);
-                }
-                const int64_t qlin = bh * H * W + (int64_t)qy * W + qx;
-                float sv = sdot * a.scale;
-                if (bias) sv += Elem<T>::to_f(bias[by * nb + (jx - ix + K - 1)]);
-                const float p = __expf(sv - a.lse[qlin]);
-                float z = 1.f;
-                if (a.dropout) {
-                    const int n = ty * K + (jx - window_start(ix, Lgx, K));
-                    z = dropout_keep((uint64_t)qlin * KK + n, a.seed, a.offset, a.drop_thresh) ? a.drop_scale : 0.f;
-                }
-                const float ds = p * (z * pdot - a.delta[qlin]);
-#pragma unroll
-                for (int jj = 0; jj < NC; ++jj) {
-                    dv[jj] = fmaf(p * z, gc[jj], dv[jj]);
-                    dk[jj] = fmaf(ds, qc[jj], dk[jj]);
-                }
+            for (int c = 0; c < QC; ++c) {
+                dv[c] = fmaf(pz, gc[c], dv[c]);
+                dk[c] = fmaf(ds, qc[c], dk[c]);
             }
         }
-        T *dkp = const_cast<T *>(at<T>(a.dk, b, h, y, x)), *dvp = const_cast<T *>(at<T>(a.dv, b, h, y, x));
 #pragma unroll
-        for (int jj = 0; jj < NC; ++jj)
-            if (lane + 32 * jj < D) {
-                dkp[lane + 32 * jj] = Elem<T>::from_f(dk[jj] * a.scale);
-                dvp[lane + 32 * jj] = Elem<T>::from_f(dv[jj]);
+        for (int o = 4; o < 32; o <<= 1)
+#pragma unroll
+            for (int c = 0; c < QC; ++c) {
+                dk[c] += __shfl_xor_sync(0xffffffffu, dk[c], o);
+                dv[c] += __shfl_xor_sync(0xffffffffu, dv[c], o);
             }
+        if (slot == 0) {
+            T *dkp = const_cast<T *>(at<T>(a.dk, b, h, y, x)) + c0, *dvp = const_cast<T *>(at<T>(a.dv, b, h, y, x)) + c0;
+#pragma unroll
+            for (int c = 0; c < QC; ++c) {
+                dkp[c] = Elem<T>::from_f(dk[c] * a.scale);
+                dvp[c] = Elem<T>::from_f(dv[c]);
+            }
+        }
     }
 }
 

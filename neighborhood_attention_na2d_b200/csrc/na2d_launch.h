@@ -106,8 +106,12 @@ cudaError_t read_umma_faults(unsigned int *count, cudaStream_t stream);
 // *launched when it took the problem; otherwise the caller uses
 // launch_forward_tc.
 bool stream_supported(const Problem &p);
-cudaError_t launch_forward_stream(const Problem &p, const void *q, const void *k, const void *v,
-                                  const void *rpb, void *out, cudaStream_t stream, bool *launched);
+// q, k, v are views with one shared set of strides; out any view.
+cudaError_t launch_forward_stream(const Problem &p, const View &q, const View &k, const View &v, const void *rpb,
+                                  const View &out, cudaStream_t stream, bool *launched);
+// Test hook: the streaming kernel's data waits give up after `clocks` SM
+// clocks (0: the default, about a second).
+void set_stream_wait_limit(long long clocks);
 // As read_device_faults, for the streaming kernel's counter.
 cudaError_t read_stream_faults(unsigned int *count, cudaStream_t stream);
 

@@ -45,6 +45,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <map>
 #include <mutex>
@@ -78,6 +79,14 @@ struct StreamParams {
     unsigned char *out;
     const void *rpb;
     int H, W, heads;
+    // byte strides (batch, head, row, pixel) of q, k, v (one set: the three
+    // views of one tensor or three contiguous tensors) and of out
+    int64_t in_sb, in_sh, in_sy, in_sx;
+    int64_t out_sb, out_sh, out_sy, out_sx;
+    int rows_contiguous;   // 1: an image row of q / k / v is one run of W * 64 bytes
+    // limit of the data waits in SM clocks (kWaitLimit unless a test shortens
+    // it); the final waits for copies in flight always use kWaitLimit
+    long long wait_limit;
     int nsteps;      // query-row pairs (split over the CTAs)
     int MX, SP, NP, NR;
     float c_log2;    // log2(e) / sqrt(D)
@@ -100,17 +109,41 @@ __device__ __forceinline__ bool sb_try(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Bounded wait for the phase with the given parity: gives up after about 2^31
-// SM clocks (about a second) and returns false.
-__device__ __forceinline__ bool sb_wait(uint32_t bar, uint32_t parity) {
+// Bounded wait for the phase with the given parity: gives up after `limit`
+// SM clocks (by default 2^31, about a second) and returns false.
+constexpr long long kWaitLimit = 1LL << 31;
+// Non-blocking test of the phase (no suspend).
+__device__ __forceinline__ bool sb_test(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ bool sb_wait(uint32_t bar, uint32_t parity, long long limit = kWaitLimit) {
+    if (limit < kWaitLimit) {
+        // a shortened limit (tests of the error path): poll without the
+        // suspend hint, which could outlast the limit
+        const long long t0 = clock64();
+        while (!sb_test(bar, parity))
+            if (clock64() - t0 > limit) return false;
+        return true;
+    }
     if (sb_try(bar, parity)) return true;
     const long long t0 = clock64();
     while (!sb_try(bar, parity))
-        if (clock64() - t0 > (1LL << 31)) return false;
+        if (clock64() - t0 > limit) return false;
     return true;
 }
 __device__ __forceinline__ void sb_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
+}
+// Arrives on the barrier once all of this thread's earlier cp.async copies
+// have landed (the arrival is counted in the barrier's initial count).
+__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(bar) : "memory");
 }
 
 // ---- programmatic dependent launch ------------------------------------------
@@ -241,6 +274,7 @@ struct SlideWalk {
     int pa, pe;       // the step's first pair and one past its last
     int ge;           // end of the CTA's range (global pair index)
     int h;            // head of image bh
+    int b;            // batch of image bh
     int ring_lo;      // ring row of lo()
     __device__ __forceinline__ int lo(const StreamParams &p) const { return pair_halo(pa, p.H); }
     __device__ __forceinline__ int hi(const StreamParams &p) const { return pair_halo(pe - 1, p.H) + 7; }
@@ -253,8 +287,11 @@ struct SlideWalk {
         pa = gb - bh * p.NP;
         pe = step_end(p);
         h = bh % p.heads;
+        b = bh / p.heads;
         ring_lo = 0;
     }
+    // byte offset of image (b, h) for the given batch / head strides
+    __device__ __forceinline__ int64_t image(int64_t sb, int64_t sh) const { return (int64_t)b * sb + (int64_t)h * sh; }
     __device__ __forceinline__ static int wrap(int x, int NR) { return x >= NR ? x - NR : x; }
     __device__ __forceinline__ int ring(const StreamParams &p, int row) const {
         return wrap(ring_lo + row - lo(p), p.NR);
@@ -265,7 +302,10 @@ struct SlideWalk {
         const int hi_ring = wrap(ring_lo + old_hi - old_lo, p.NR);
         if (pe == p.NP) {
             ++bh;
-            if (++h == p.heads) h = 0;
+            if (++h == p.heads) {
+                h = 0;
+                ++b;
+            }
             pa = 0;
             pe = step_end(p);
             ring_lo = wrap(hi_ring + 1, p.NR);
@@ -504,7 +544,9 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
 
     if (threadIdx.x == NWC * 32) {
         for (int i = 0; i < NS; ++i) {
-            sb_init(bar_full + 8 * i, 1);     // one expect_tx arrival per step
+            // bulk copies: one expect_tx arrival per step; strided rows: one
+            // cp.async arrival per producer lane
+            sb_init(bar_full + 8 * i, p.rows_contiguous ? 1 : 32);
             sb_init(bar_empty + 8 * i, NWC);
         }
         *abort_flag = 0;
@@ -512,7 +554,53 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
     }
     __syncthreads();
 
-    if (warp == NWC) {
+    if (warp == NWC && !p.rows_contiguous) {
+        // =================== producer, strided rows ===================
+        // the warp copies each new row's pixels as 16-byte pieces (cp.async),
+        // every lane arriving on the stage's full barrier once its copies of
+        // the step have landed
+        grid_dep_wait();
+        SlideWalk w;
+        w.init(p, s_begin, s_end);
+        for (int i = 0; i < nst; ++i) {
+            const int stage = i % NS;
+            const int first = i ? w.next(p) : w.lo(p);
+            const bool ok = i >= NS ? sb_wait(bar_empty + 8 * stage, (uint32_t)(((i / NS) - 1) & 1), p.wait_limit)
+                                    : (i == 0 || sb_wait(bar_full + 8 * (i - 1), 0u, p.wait_limit));
+            if (!ok) {
+                if (lane == 0) {
+                    atomicAdd(&g_stream_timeouts, 1u);
+                    *abort_flag = 1;
+                }
+                break;
+            }
+            if (*abort_flag) break;
+            const int hi = w.hi(p);
+            const int y0 = 2 * w.pa, y1 = min(2 * w.pe, p.H);
+            const int64_t img = w.image(p.in_sb, p.in_sh);
+            const int pieces = p.W * 4;
+            for (int row = first; row <= hi; ++row) {
+                const uint32_t o = row_base(w.ring(p, row), pitch);
+                const int64_t src = img + (int64_t)row * p.in_sy;
+                for (int e = lane; e < pieces; e += 32) {
+                    const int64_t so = src + (int64_t)(e >> 2) * p.in_sx + 16 * (e & 3);
+                    const uint32_t d = o + (uint32_t)(e >> 2) * kPixB + 16u * (uint32_t)(e & 3);
+                    cp_async_16(sbase + p.off_k + d, p.k + so);
+                    cp_async_16(sbase + p.off_v + d, p.v + so);
+                }
+            }
+            for (int y = y0; y < y1; ++y) {
+                const uint32_t o = row_base(stage * 2 * p.SP + (y - y0), pitch);
+                const int64_t src = img + (int64_t)y * p.in_sy;
+                for (int e = lane; e < pieces; e += 32)
+                    cp_async_16(sbase + o + (uint32_t)(e >> 2) * kPixB + 16u * (uint32_t)(e & 3),
+                                p.q + src + (int64_t)(e >> 2) * p.in_sx + 16 * (e & 3));
+            }
+            cp_async_arrive(bar_full + 8 * stage);
+        }
+        // every copy lands before the CTA's shared memory is released
+        cp_async_wait<0>();
+    } else if (warp == NWC) {
         // =================== producer ===================
         // one thread issues one bulk copy per image row: the step's new K and
         // V rows into the ring, its query rows into the stage
@@ -529,8 +617,8 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
                 // previous step's rows have landed, so that the first step's
                 // rows do not queue behind the next steps'; later, a step
                 // waits for its stage to be released
-                const bool ok = i >= NS ? sb_wait(bar_empty + 8 * stage, (uint32_t)(((i / NS) - 1) & 1))
-                                        : (i == 0 || sb_wait(bar_full + 8 * (i - 1), 0u));
+                const bool ok = i >= NS ? sb_wait(bar_empty + 8 * stage, (uint32_t)(((i / NS) - 1) & 1), p.wait_limit)
+                                        : (i == 0 || sb_wait(bar_full + 8 * (i - 1), 0u, p.wait_limit));
                 if (!ok) {
                     atomicAdd(&g_stream_timeouts, 1u);
                     *abort_flag = 1;
@@ -540,16 +628,17 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
                 const int hi = w.hi(p);
                 const int y0 = 2 * w.pa, y1 = min(2 * w.pe, p.H);
                 const uint32_t bar = bar_full + 8 * stage;
+                const int64_t img = w.image(p.in_sb, p.in_sh);
                 sb_expect_tx(bar, (uint32_t)(2 * (hi - first + 1) + (y1 - y0)) * rowbytes);
                 for (int row = first; row <= hi; ++row) {
                     const uint32_t o = row_base(w.ring(p, row), pitch);
-                    const size_t src = ((size_t)w.bh * p.H + row) * rowbytes;
+                    const int64_t src = img + (int64_t)row * p.in_sy;
                     bulk_g2s(sbase + p.off_k + o, p.k + src, rowbytes, bar);
                     bulk_g2s(sbase + p.off_v + o, p.v + src, rowbytes, bar);
                 }
                 for (int y = y0; y < y1; ++y)
-                    bulk_g2s(sbase + row_base(stage * 2 * p.SP + (y - y0), pitch),
-                             p.q + ((size_t)w.bh * p.H + y) * rowbytes, rowbytes, bar);
+                    bulk_g2s(sbase + row_base(stage * 2 * p.SP + (y - y0), pitch), p.q + img + (int64_t)y * p.in_sy,
+                             rowbytes, bar);
                 ++issued;
             }
             // copies still in flight must land before the CTA's shared
@@ -663,7 +752,7 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
                     tmem_st_wait();
                 }
             }
-            if (!sb_wait(bar_full + 8 * stage, (uint32_t)((i / NS) & 1))) {
+            if (!sb_wait(bar_full + 8 * stage, (uint32_t)((i / NS) & 1), p.wait_limit)) {
                 if (lane == 0) {
                     atomicAdd(&g_stream_timeouts, 1u);
                     *abort_flag = 1;
@@ -678,14 +767,14 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
                 uint32_t qa[NT], ka[NT], va[NT];
                 unsigned char *o[NT];
                 const int oy = orow ? qy0 + 1 : qy0;
-                unsigned char *orow_ptr = p.out + ((size_t)w.bh * H + oy) * W * kPixB;
+                unsigned char *orow_ptr = p.out + w.image(p.out_sb, p.out_sh) + (int64_t)oy * p.out_sy;
 #pragma unroll
                 for (int u = 0; u < NT; ++u) {
                     qa[u] = qrow + qcol[u];
                     ka[u] = krb + kcol[u];
                     va[u] = vrb + vcol[u];
                     const int ox = xq[u] + ocol0;
-                    o[u] = (oy < H && ox < W) ? orow_ptr + (size_t)ox * kPixB : nullptr;
+                    o[u] = (oy < H && ox < W) ? orow_ptr + (int64_t)ox * p.out_sx : nullptr;
                 }
                 if (NT == 2 && shared_cols)
                     tile_run<T, NT, NT == 2>(qa, ka, va, tb, p.c_log2, o, lane);
@@ -743,6 +832,12 @@ cudaError_t stream_device(int *sms, int *smem_cap, const void *kern) {
 }
 
 uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
+
+std::atomic<long long> &wait_limit_store() {
+    static std::atomic<long long> v{0};
+    return v;
+}
+long long stream_wait_limit() { return wait_limit_store().load(); }
 
 template <typename T, int NWC, int NT>
 cudaError_t launch_stream_t(const StreamParams &sp, uint32_t smem, int grid, cudaStream_t st, bool *launched) {
@@ -815,14 +910,20 @@ cudaError_t launch_slide(StreamParams &sp, const Problem &pr, cudaStream_t st, b
 }
 
 template <typename T>
-cudaError_t launch_stream_impl(const Problem &pr, const void *q, const void *k, const void *v, const void *rpb,
-                               void *out, cudaStream_t st, bool *launched) {
+cudaError_t launch_stream_impl(const Problem &pr, const View &q, const View &k, const View &v, const void *rpb,
+                               const View &out, cudaStream_t st, bool *launched) {
     StreamParams sp{};
-    sp.q = static_cast<const unsigned char *>(q);
-    sp.k = static_cast<const unsigned char *>(k);
-    sp.v = static_cast<const unsigned char *>(v);
-    sp.out = static_cast<unsigned char *>(out);
+    sp.q = static_cast<const unsigned char *>(q.p);
+    sp.k = static_cast<const unsigned char *>(k.p);
+    sp.v = static_cast<const unsigned char *>(v.p);
+    sp.out = static_cast<unsigned char *>(const_cast<void *>(out.p));
     sp.rpb = rpb;
+    const int64_t e = 2;   // f16 / bf16
+    sp.in_sb = q.sb * e; sp.in_sh = q.sh * e; sp.in_sy = q.sy * e; sp.in_sx = q.sx * e;
+    sp.out_sb = out.sb * e; sp.out_sh = out.sh * e; sp.out_sy = out.sy * e; sp.out_sx = out.sx * e;
+    sp.rows_contiguous = (q.sx == 32 && q.sy == (int64_t)32 * pr.W) ? 1 : 0;
+    const long long lim = stream_wait_limit();
+    sp.wait_limit = lim > 0 ? lim : kWaitLimit;
     sp.H = pr.H; sp.W = pr.W; sp.heads = pr.heads;
     sp.c_log2 = kLog2e / std::sqrt((float)pr.D);
     sp.sqrt_d = std::sqrt((float)pr.D);
@@ -833,19 +934,28 @@ cudaError_t launch_stream_impl(const Problem &pr, const void *q, const void *k, 
 
 }  // namespace
 
+bool stream_views_supported(const Problem &p, const View &q, const View &k, const View &v) {
+    // q, k and v share one set of strides (three contiguous tensors, or the
+    // three views of one fused tensor)
+    return q.sb == k.sb && q.sh == k.sh && q.sy == k.sy && q.sx == k.sx && q.sb == v.sb && q.sh == v.sh &&
+           q.sy == v.sy && q.sx == v.sx;
+}
+
 bool stream_supported(const Problem &p) {
     if (p.dtype != DType::F16 && p.dtype != DType::BF16) return false;
     if (p.k != KW || p.D != 32 || p.heads > 64) return false;
     return p.d == 1 && p.W >= 14 && p.W <= 64 && p.H >= 8;          // sliding rows
 }
 
-cudaError_t launch_forward_stream(const Problem &p, const void *q, const void *k, const void *v, const void *rpb,
-                                  void *out, cudaStream_t st, bool *launched) {
+cudaError_t launch_forward_stream(const Problem &p, const View &q, const View &k, const View &v, const void *rpb,
+                                  const View &out, cudaStream_t st, bool *launched) {
     *launched = false;
-    if (!stream_supported(p)) return cudaSuccess;
+    if (!stream_supported(p) || !stream_views_supported(p, q, k, v)) return cudaSuccess;
     if (p.dtype == DType::F16) return launch_stream_impl<__half>(p, q, k, v, rpb, out, st, launched);
     return launch_stream_impl<__nv_bfloat16>(p, q, k, v, rpb, out, st, launched);
 }
+
+void set_stream_wait_limit(long long clocks) { wait_limit_store().store(clocks > 0 ? clocks : 0); }
 
 cudaError_t read_stream_faults(unsigned int *count, cudaStream_t st) {
     unsigned int zero = 0;

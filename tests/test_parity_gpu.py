@@ -296,6 +296,32 @@ def test_chained_calls_same_stream(shape, graph):
         prev = got
 
 
+def test_bounded_wait_error_path_runs_out_and_recovers():
+    """The error path of the bounded waits, run on purpose without any fault:
+    with the streaming kernel's data-wait limit cut to 200 SM clocks, the
+    first copies (about a microsecond away) cannot land in time; the kernel
+    must count the event, drain its copies in flight and return.  The count
+    is then non-zero, and with the default limit restored the next call is
+    correct and counts nothing."""
+    from neighborhood_attention_na2d_b200 import _native
+    shape = Shape(4, 2, 56, 56, 32, 7, 1, "f16", 1701)
+    q, k, v, rpb = make_inputs(shape)
+    qd, kd, vd, rd = (t.cuda() for t in (q, k, v, rpb))
+    assert na.na2d_device_faults() == 0
+    try:
+        _native.lib().na2d_debug_set_wait_limit(200)
+        na.na2d_forward(qd, kd, vd, rd, 7, 1)
+        assert na.na2d_last_kernel() == "fwd_stream_kernel"
+        assert na.na2d_device_faults() > 0
+    finally:
+        _native.lib().na2d_debug_set_wait_limit(0)
+    out = na.na2d_forward(qd, kd, vd, rd, 7, 1)
+    torch.cuda.synchronize()
+    assert na.na2d_device_faults() == 0
+    want = oracle.forward(f64(q), f64(k), f64(v), f64(rpb), 7, 1)
+    assert max_err(out.double().cpu().numpy(), want) <= TOL["f16"]
+
+
 def test_no_device_wait_timed_out():
     """Runs after the parity tests above (same module): no kernel gave up on a
     bounded wait."""
