@@ -50,6 +50,7 @@
 #include <map>
 #include <mutex>
 #include <set>
+#include <type_traits>
 
 #include "na2d_device.cuh"
 #include "na2d_launch.h"
@@ -66,6 +67,7 @@ constexpr int kTabHead = 13 * kTabPitch;
 constexpr int kTileCols = 4;          // query columns of a tile
 constexpr int kHaloCols = kTileCols + KW - 1;   // 10 key columns per tile
 constexpr int kKG = kHaloCols / 2;    // 5 key groups of 16 keys (8 rows x 2 columns)
+constexpr int kMargin = KW / 2;       // zero pixels left of every shared-memory row
 #ifndef NAT_NWC
 #define NAT_NWC 14                    // consumer warps
 #define NAT_NT 2                      // 4-column tiles per consumer warp and step
@@ -89,6 +91,7 @@ struct StreamParams {
     long long wait_limit;
     int nsteps;      // query-row pairs (split over the CTAs)
     int MX, SP, NP, NR;
+    uint32_t pitch;  // bytes per shared-memory row: kMargin zero pixels, W pixels, zero pixels up to MX*span + 3
     float c_log2;    // log2(e) / sqrt(D)
     float sqrt_d;    // sqrt(D)
     uint32_t off_k, off_v, off_tab, off_bar;   // byte offsets in dynamic shared memory (Q at 0)
@@ -195,6 +198,24 @@ __device__ __forceinline__ void tmem_ld4(uint32_t taddr, float (&v)[4]) {
                  : "memory");
 }
 
+// ldmatrix (x4, and x4.trans) at a compile-time byte offset from a base
+// address: the offset goes into the instruction, so a tile's 20-odd
+// fragment loads share one address register.
+template <int OFF> __device__ __forceinline__ void ldsm_x4_at(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4+%5];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr), "n"(OFF));
+}
+template <int OFF> __device__ __forceinline__ void ldsm_x4_t_at(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4+%5];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr), "n"(OFF));
+}
+// 4-byte global store at a compile-time byte offset from a pointer.
+template <int OFF> __device__ __forceinline__ void st_b32_at(unsigned char *ptr, uint32_t v) {
+    asm volatile("st.global.b32 [%0+%1], %2;\n" ::"l"(ptr), "n"(OFF), "r"(v) : "memory");
+}
+
 // Transposes an 8 x 8 matrix of 16-bit elements held one row-pair per lane
 // (the mma / ldmatrix fragment layout) across the warp.
 __device__ __forceinline__ uint32_t movm_t(uint32_t x) {
@@ -257,9 +278,6 @@ __device__ __forceinline__ int win_start(int y, int L) { return clampi(y - KW / 
 // hold both rows' clamped windows.
 __device__ __forceinline__ int pair_halo(int pair, int H) { return min(win_start(2 * pair, H), H - 8); }
 
-// Halo start of the 4-column tile at x0: the first of 10 consecutive key
-// columns that hold its queries' clamped windows.
-__device__ __forceinline__ int tile_halo(int x0, int W) { return clampi(x0 - KW / 2, 0, W - kHaloCols); }
 
 // The CTA's steps in order, with the K / V ring bookkeeping.  A CTA owns a
 // contiguous range of query-row pairs in (image, pair) order (global pair
@@ -339,11 +357,34 @@ __device__ __forceinline__ void sb_expect_tx(uint32_t bar, uint32_t bytes) {
 }
 
 // Skewed row layout: row r of a buffer starts at r * pitch + 16 * (r & 3)
-// bytes (pitch = (W + 1) * 64); pixels and their four 16-byte chunks are
-// stored in order, so a whole image row lands with one bulk copy.  Any 4
-// consecutive rows x 2 adjacent pixels of one chunk index fall in 8 distinct
-// bank groups.
+// bytes; image column x is pixel kMargin + x of the row (pixels and their
+// four 16-byte chunks in order), so a whole image row lands with one bulk
+// copy.  The kMargin pixels on the left and the pixels right of the image
+// (up to column MX * span + kMargin - 1) are zeros, written once: every tile's
+// 10-column halo starts at x0 - kMargin without clamping, and halo columns
+// outside the image read zero keys and values (their scores are masked by
+// the bias).  Any 4 consecutive rows x 2 adjacent pixels of one chunk index
+// fall in 8 distinct bank groups.  The skew makes a row overrun its pitch by
+// up to 48 bytes, into the next row's left margin (zeros both ways); each
+// buffer keeps 64 bytes of slack after its last row.
 __device__ __forceinline__ uint32_t row_base(int r, uint32_t pitch) { return (uint32_t)r * pitch + 16u * (r & 3); }
+
+// Fragment loads of key group G (compile time): K k-steps 0 / 1, V channels
+// 0-15 / 16-31.
+template <int G> __device__ __forceinline__ void ld_k(uint32_t (&k0)[4], uint32_t (&k1)[4], uint32_t base) {
+    ldsm_x4_at<128 * G>(k0, base);
+    ldsm_x4_at<128 * G + 32>(k1, base);
+}
+template <int G> __device__ __forceinline__ void ld_v(uint32_t (&v0)[4], uint32_t (&v1)[4], uint32_t base) {
+    ldsm_x4_t_at<128 * G>(v0, base);
+    ldsm_x4_t_at<128 * G + 32>(v1, base);
+}
+template <int G, int N, typename F> __device__ __forceinline__ void static_for(F &&f) {
+    if constexpr (G < N) {
+        f(std::integral_constant<int, G>{});
+        static_for<G + 1, N>(f);
+    }
+}
 
 // One P.V k-step of a tile: O^T += V^T P^T (channels 0-15 and 16-31) and the
 // row sums l += 1^T P^T; `first` starts the accumulators at zero.
@@ -398,31 +439,30 @@ __device__ __forceinline__ void tile_run(const uint32_t (&qa)[NT], const uint32_
     tmem_ld_wait();
     // ---- S^T = K Q^T + bias (C-init)
     if constexpr (SHARED) {
-#pragma unroll
-        for (int gi = 0; gi < NG; ++gi) {
+        static_for<0, NG>([&](auto G) {
+            constexpr int gi = decltype(G)::value;
             uint32_t k0[4], k1[4];
-            ldsm_x4(k0, ka[0] + 128u * gi);
-            ldsm_x4(k1, ka[0] + 128u * gi + 32u);
-            if (gi < kKG) {
+            ld_k<gi>(k0, k1, ka[0]);
+            if constexpr (gi < kKG) {
                 Mma<T>::run(s[0][gi], k0, qb[0][0], qb[0][1]);
                 Mma<T>::run(s[0][gi], k1, qb[0][2], qb[0][3]);
             }
-            if (gi >= 2) {
+            if constexpr (gi >= 2) {
                 Mma<T>::run(s[1][gi - 2], k0, qb[1][0], qb[1][1]);
                 Mma<T>::run(s[1][gi - 2], k1, qb[1][2], qb[1][3]);
             }
-        }
+        });
     } else {
-#pragma unroll
-        for (int t = 0; t < kKG; ++t)
+        static_for<0, kKG>([&](auto G) {
+            constexpr int t = decltype(G)::value;
 #pragma unroll
             for (int u = 0; u < NT; ++u) {
                 uint32_t k0[4], k1[4];
-                ldsm_x4(k0, ka[u] + 128u * t);
-                ldsm_x4(k1, ka[u] + 128u * t + 32u);
+                ld_k<t>(k0, k1, ka[u]);
                 Mma<T>::run(s[u][t], k0, qb[u][0], qb[u][1]);
                 Mma<T>::run(s[u][t], k1, qb[u][2], qb[u][3]);
             }
+        });
     }
     // ---- row max of queries 2c (m[u][0]) and 2c + 1 (m[u][1]): registers, then
     // the 8 lanes that hold the other keys of the same queries
@@ -462,28 +502,22 @@ __device__ __forceinline__ void tile_run(const uint32_t (&qa)[NT], const uint32_
     constexpr uint32_t ONE = OnesBits<T>::v;
     const uint32_t ones[4] = {ONE, ONE, ONE, ONE};
     float o[NT][2][4], l[NT][4];
-#pragma unroll
-    for (int gi = 0; gi < NG; ++gi) {
+    static_for<0, NG>([&](auto G) {
+        constexpr int gi = decltype(G)::value;
         if constexpr (SHARED) {
             uint32_t v0[4], v1[4];
-            ldsm_x4_t(v0, va[0] + 128u * gi);
-            ldsm_x4_t(v1, va[0] + 128u * gi + 32u);
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int t = gi - 2 * u;
-                if (t < 0 || t >= kKG) continue;
-                pv_step<T>(o[u], l[u], v0, v1, bp[u][t], ones, t == 0);
-            }
+            ld_v<gi>(v0, v1, va[0]);
+            if constexpr (gi < kKG) pv_step<T>(o[0], l[0], v0, v1, bp[0][gi], ones, gi == 0);
+            if constexpr (gi >= 2) pv_step<T>(o[NT - 1], l[NT - 1], v0, v1, bp[NT - 1][gi - 2], ones, gi == 2);
         } else {
 #pragma unroll
             for (int u = 0; u < NT; ++u) {
                 uint32_t v0[4], v1[4];
-                ldsm_x4_t(v0, va[u] + 128u * gi);
-                ldsm_x4_t(v1, va[u] + 128u * gi + 32u);
+                ld_v<gi>(v0, v1, va[u]);
                 pv_step<T>(o[u], l[u], v0, v1, bp[u][gi], ones, gi == 0);
             }
         }
-    }
+    });
     // ---- normalise, transpose back (query lane / 4, channels 2c, 2c + 1 of
     // each 8-channel chunk) and store 4 bytes per chunk
     const uint32_t cofs = 4u * (uint32_t)(lane & 3);
@@ -502,8 +536,11 @@ __device__ __forceinline__ void tile_run(const uint32_t (&qa)[NT], const uint32_
             y[2 * h + 1] = movm_t(Elem<T>::pack2(a2, a3));
         }
         if (out[u]) {
-#pragma unroll
-            for (int j = 0; j < 4; ++j) *reinterpret_cast<uint32_t *>(out[u] + 16 * j + cofs) = y[j];
+            unsigned char *op = out[u] + cofs;
+            st_b32_at<0>(op, y[0]);
+            st_b32_at<16>(op, y[1]);
+            st_b32_at<32>(op, y[2]);
+            st_b32_at<48>(op, y[3]);
         }
     }
 }
@@ -540,7 +577,8 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + p.off_bar + 16 * NS + 4);
     // bias table, with 64 bytes of padding on either side for unclamped column reads
     float *tab = reinterpret_cast<float *>(smem + p.off_tab + 64);
-    const uint32_t pitch = (uint32_t)(p.W + 1) * kPixB;   // row pitch in bytes
+    const uint32_t pitch = p.pitch;                        // row pitch in bytes
+    constexpr uint32_t kLead = kMargin * kPixB;            // image column 0 within a row
 
     if (threadIdx.x == NWC * 32) {
         for (int i = 0; i < NS; ++i) {
@@ -580,7 +618,7 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
             const int64_t img = w.image(p.in_sb, p.in_sh);
             const int pieces = p.W * 4;
             for (int row = first; row <= hi; ++row) {
-                const uint32_t o = row_base(w.ring(p, row), pitch);
+                const uint32_t o = row_base(w.ring(p, row), pitch) + kLead;
                 const int64_t src = img + (int64_t)row * p.in_sy;
                 for (int e = lane; e < pieces; e += 32) {
                     const int64_t so = src + (int64_t)(e >> 2) * p.in_sx + 16 * (e & 3);
@@ -590,7 +628,7 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
                 }
             }
             for (int y = y0; y < y1; ++y) {
-                const uint32_t o = row_base(stage * 2 * p.SP + (y - y0), pitch);
+                const uint32_t o = row_base(stage * 2 * p.SP + (y - y0), pitch) + kLead;
                 const int64_t src = img + (int64_t)y * p.in_sy;
                 for (int e = lane; e < pieces; e += 32)
                     cp_async_16(sbase + o + (uint32_t)(e >> 2) * kPixB + 16u * (uint32_t)(e & 3),
@@ -631,14 +669,14 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
                 const int64_t img = w.image(p.in_sb, p.in_sh);
                 sb_expect_tx(bar, (uint32_t)(2 * (hi - first + 1) + (y1 - y0)) * rowbytes);
                 for (int row = first; row <= hi; ++row) {
-                    const uint32_t o = row_base(w.ring(p, row), pitch);
+                    const uint32_t o = row_base(w.ring(p, row), pitch) + kLead;
                     const int64_t src = img + (int64_t)row * p.in_sy;
                     bulk_g2s(sbase + p.off_k + o, p.k + src, rowbytes, bar);
                     bulk_g2s(sbase + p.off_v + o, p.v + src, rowbytes, bar);
                 }
                 for (int y = y0; y < y1; ++y)
-                    bulk_g2s(sbase + row_base(stage * 2 * p.SP + (y - y0), pitch), p.q + img + (int64_t)y * p.in_sy,
-                             rowbytes, bar);
+                    bulk_g2s(sbase + row_base(stage * 2 * p.SP + (y - y0), pitch) + kLead,
+                             p.q + img + (int64_t)y * p.in_sy, rowbytes, bar);
                 ++issued;
             }
             // copies still in flight must land before the CTA's shared
@@ -657,6 +695,18 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
                 float v = 0.f;
                 if (rpb && b < 13) v = Elem<T>::to_f(rpb[(h * 13 + a) * 13 + b]) * p.sqrt_d;
                 tab[i] = v;
+            }
+            // zero the margins of every ring row of K and V (the copies write
+            // only the image columns)
+            {
+                const int lead16 = kMargin * 4, row16 = (int)(pitch / 16), tail16 = row16 - lead16 - 4 * p.W;
+                const int per_row = lead16 + tail16;
+                for (int i = threadIdx.x; i < 2 * p.NR * per_row; i += NWC * 32) {
+                    const int r = (i / per_row) % p.NR, t = i % per_row;
+                    const uint32_t off = (i / per_row >= p.NR ? p.off_v : p.off_k) + row_base(r, pitch) +
+                                         16u * (uint32_t)(t < lead16 ? t : t + 4 * p.W);
+                    *reinterpret_cast<uint4 *>(smem + off) = make_uint4(0, 0, 0, 0);
+                }
             }
             if (warp == 0) tmem_alloc(smem_u32(tmem_slot));
             tmem_fence_before();
@@ -682,16 +732,19 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
 #pragma unroll
         for (int u = 0; u < NT; ++u) {
             xq[u] = x0 + kTileCols * u;
-            const int hx = tile_halo(xq[u], W);
-            qcol[u] = (uint32_t)min(xq[u] + (lane & 3), W - 1) * kPixB + 16u * (uint32_t)(lane >> 3);
-            kcol[u] = (uint32_t)(hx + (mk & 1)) * kPixB + 16u * (uint32_t)(lane >> 4);
-            vcol[u] = (uint32_t)(hx + (mv & 1)) * kPixB + 16u * (uint32_t)((lane >> 3) & 1);
+            // halo columns hx .. hx + 9: x0 - 3 .. x0 + 6, except for a last
+            // tile that starts within 3 columns of the right edge, whose
+            // queries all share the window W - 7 .. W - 1
+            const int hx = min(xq[u] - kMargin, W - KW);
+            qcol[u] = (uint32_t)(min(xq[u] + (lane & 3), W - 1) + kMargin) * kPixB + 16u * (uint32_t)(lane >> 3);
+            kcol[u] = (uint32_t)(hx + kMargin + (mk & 1)) * kPixB + 16u * (uint32_t)(lane >> 4);
+            vcol[u] = (uint32_t)(hx + kMargin + (mv & 1)) * kPixB + 16u * (uint32_t)((lane >> 3) & 1);
             xin[u] = 0;
 #pragma unroll
             for (int jlo = 0; jlo < 2; ++jlo) {
                 const int qx = min(xq[u] + 2 * (c & 1) + jlo, W - 1), sx = win_start(qx, W);
                 // kx - qx + 6 for key column kx = hx + 2t + (g & 1): within
-                // [-3, 15], inside the padded table
+                // [0, 12]
                 cb[u][jlo] = hx + (g & 1) - qx + 6;
 #pragma unroll
                 for (int t = 0; t < kKG; ++t) {
@@ -700,9 +753,10 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
                 }
             }
         }
-        // the two tiles' halos are 4 columns apart (away from the image's
-        // left and right edges): their key groups can be shared
-        const bool shared_cols = NT == 2 && tile_halo(xq[NT - 1], W) == tile_halo(xq[0], W) + kTileCols;
+        // the two tiles' halos are 4 columns apart (all but a warp that holds
+        // a last tile starting within 3 columns of the right edge): their key
+        // groups can be shared
+        const bool shared_cols = NT == 2 && min(xq[NT - 1] - kMargin, W - KW) == xq[0] - kMargin + kTileCols;
         const int qsel = (lane >> 2) & 1;
         // output pixel of this lane's epilogue query (lane / 4): tile row g / 4, column g % 4
         const int orow = g >> 2, ocol0 = g & 3;
@@ -762,8 +816,10 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
             if (*abort_flag) break;
             if (work) {
                 const uint32_t qrow = sbase + row_base(stage * 2 * p.SP + (qsel ? qy1 : qy0) - 2 * w.pa, pitch);
-                const uint32_t krb = sbase + p.off_k + row_base(w.ring(p, hy + krow), pitch);
-                const uint32_t vrb = sbase + p.off_v + row_base(w.ring(p, hy + vrow), pitch);
+                // ring rows of this lane's K and V fragment rows
+                const int rb = w.ring_lo - w.lo(p) + hy;
+                const uint32_t krb = sbase + p.off_k + row_base(SlideWalk::wrap(rb + krow, p.NR), pitch);
+                const uint32_t vrb = sbase + p.off_v + row_base(SlideWalk::wrap(rb + vrow, p.NR), pitch);
                 uint32_t qa[NT], ka[NT], va[NT];
                 unsigned char *o[NT];
                 const int oy = orow ? qy0 + 1 : qy0;
@@ -858,19 +914,21 @@ cudaError_t launch_stream_t(const StreamParams &sp, uint32_t smem, int grid, cud
 }
 
 // Plan for SP query-row pairs per step; returns the shared-memory bytes.
-uint32_t plan_slide(StreamParams &sp, const Problem &pr, int SP, int span) {
+// `aligned`: every CTA's range lies inside one image.
+uint32_t plan_slide(StreamParams &sp, const Problem &pr, int SP, int span, bool aligned) {
     sp.MX = (pr.W + span - 1) / span;
     sp.SP = SP;
     sp.NP = (pr.H + 1) / 2;
     const int spi = (sp.NP + sp.SP - 1) / sp.SP;   // steps per image
     // K / V rows needed by NS consecutive steps: 2*SP per step plus a 6-row
-    // halo for every image those steps touch
-    const int images = std::min(NS, (NS - 2) / spi + 2);
+    // halo for every image those steps touch (one when no CTA crosses images)
+    const int images = aligned ? 1 : std::min(NS, (NS - 2) / spi + 2);
     sp.NR = (int)align_up((uint32_t)(2 * sp.SP * NS + 6 * images), 4);
-    // skewed rows: pitch (W + 1) * 64 bytes (see row_base)
-    const uint32_t pitch = (uint32_t)(pr.W + 1) * kPixB;
-    const uint32_t qbytes = (uint32_t)(NS * 2 * sp.SP) * pitch;
-    const uint32_t ring = (uint32_t)sp.NR * pitch;
+    // rows: kMargin zero pixels, the image, zero pixels up to column
+    // MX * span + kMargin - 1 (the last tile's halo); see row_base
+    sp.pitch = (uint32_t)(sp.MX * span + 2 * kMargin) * kPixB;
+    const uint32_t qbytes = (uint32_t)(NS * 2 * sp.SP) * sp.pitch + 64;
+    const uint32_t ring = (uint32_t)sp.NR * sp.pitch + 64;
     sp.off_k = align_up(qbytes, 128);
     sp.off_v = sp.off_k + align_up(ring, 128);
     sp.off_tab = sp.off_v + align_up(ring, 128);
@@ -886,24 +944,31 @@ cudaError_t launch_slide(StreamParams &sp, const Problem &pr, cudaStream_t st, b
     if (e != cudaSuccess) return e;
     const int span = kTileCols * NT;   // query columns per consumer warp
     const int MX = (pr.W + span - 1) / span;
-    for (int SP = std::max(1, NWC / MX); SP >= 1; --SP) {
-        const uint32_t smem = plan_slide(sp, pr, SP, span);
-        if ((int)smem > cap) continue;
-        const int64_t npairs = pr.bh() * sp.NP;
-        if (npairs >= INT32_MAX || npairs <= 0) return cudaSuccess;
-        sp.nsteps = (int)npairs;
-        // CTAs: one per SM with an even split of the pairs, or, when the
-        // images fit on the SMs, a whole number c of CTAs per image, so that
-        // every CTA's range lies inside one image (no second halo and no
-        // second clamped image top, which cost about a step).  The aligned
-        // split is taken while it gives a CTA at most one pair more.
-        const int64_t images = pr.bh();
-        int grid = (int)std::min<int64_t>(npairs, sms);
-        if (images <= sms) {
-            const int64_t c = std::min<int64_t>(sms / images, sp.NP);
-            const int64_t aligned = (sp.NP + c - 1) / c, even = (npairs + sms - 1) / sms;
-            if (aligned <= even + 1) grid = (int)(images * c);
+    sp.NP = (pr.H + 1) / 2;
+    const int64_t npairs = pr.bh() * sp.NP;
+    if (npairs >= INT32_MAX || npairs <= 0) return cudaSuccess;
+    sp.nsteps = (int)npairs;
+    // CTAs: one per SM with an even split of the pairs, or, when the images
+    // fit on the SMs, a whole number c of CTAs per image, so that every CTA's
+    // range lies inside one image (no second halo and no second clamped image
+    // top, which cost about a step).  The aligned split is taken while it
+    // gives a CTA at most one pair more.
+    const int64_t images = pr.bh();
+    int grid = (int)std::min<int64_t>(npairs, sms);
+    bool aligned = false;
+    if (images <= sms) {
+        const int64_t c = std::min<int64_t>(sms / images, sp.NP);
+        const int64_t per = (sp.NP + c - 1) / c, even = (npairs + sms - 1) / sms;
+        if (per <= even + 1) {
+            // per pairs per CTA when they divide an image's pairs (the ranges
+            // then stay inside one image), else an even split over images * c
+            aligned = sp.NP % per == 0;
+            grid = (int)(images * (aligned ? sp.NP / per : c));
         }
+    }
+    for (int SP = std::max(1, NWC / MX); SP >= 1; --SP) {
+        const uint32_t smem = plan_slide(sp, pr, SP, span, aligned);
+        if ((int)smem > cap) continue;
         return launch_stream_t<T, NWC, NT>(sp, smem, grid, st, launched);
     }
     return cudaSuccess;

@@ -298,13 +298,14 @@ def test_chained_calls_same_stream(shape, graph):
 
 def test_bounded_wait_error_path_runs_out_and_recovers():
     """The error path of the bounded waits, run on purpose without any fault:
-    with the streaming kernel's data-wait limit cut to 200 SM clocks, the
-    first copies (about a microsecond away) cannot land in time; the kernel
-    must count the event, drain its copies in flight and return.  The count
-    is then non-zero, and with the default limit restored the next call is
-    correct and counts nothing."""
+    with the streaming kernel's wait limit cut to 200 SM clocks, a CTA with
+    several steps cannot see its stages released in time (the consumers need
+    microseconds for their first step, the producer reaches the wait for the
+    fourth stage at once); the kernel must count the event, drain its copies
+    in flight and return.  The count is then non-zero, and with the default
+    limit restored the next call is correct and counts nothing."""
     from neighborhood_attention_na2d_b200 import _native
-    shape = Shape(4, 2, 56, 56, 32, 7, 1, "f16", 1701)
+    shape = Shape(32, 2, 56, 56, 32, 7, 1, "f16", 1701)   # 14 query-row pairs (7 steps) per CTA
     q, k, v, rpb = make_inputs(shape)
     qd, kd, vd, rd = (t.cuda() for t in (q, k, v, rpb))
     assert na.na2d_device_faults() == 0
