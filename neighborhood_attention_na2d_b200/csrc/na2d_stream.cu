@@ -761,52 +761,73 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
         // output pixel of this lane's epilogue query (lane / 4): tile row g / 4, column g % 4
         const int orow = g >> 2, ocol0 = g & 3;
         int bias_key = -1;
+        // Geometry of one step for this warp, worked out one step early: right
+        // after the previous step's tiles, while their last products and
+        // stores drain.
+        struct Geo {
+            int pair, h, key;
+            bool work;
+            uint32_t qrow, krb, vrb;
+            unsigned char *orow;   // output row of this lane's epilogue query, or null
+        };
+        auto geo_of = [&](const SlideWalk &w, int stage, Geo &e) {
+            e.pair = w.pa + pw;
+            e.work = active && e.pair < w.pe;
+            e.h = w.h;
+            const int qy0 = 2 * e.pair, qy1 = min(qy0 + 1, H - 1);
+            const int hy = pair_halo(e.pair, H);
+            e.key = ((w.h * 8 + (qy0 - hy)) * 2 + (qy1 - qy0)) * 4 + (win_start(qy0, H) - hy) * 2 +
+                    (win_start(qy1, H) - hy);
+            e.qrow = sbase + row_base(stage * 2 * p.SP + (qsel ? qy1 : qy0) - 2 * w.pa, pitch);
+            // ring rows of this lane's K and V fragment rows
+            const int rb = w.ring_lo - w.lo(p) + hy;
+            e.krb = sbase + p.off_k + row_base(SlideWalk::wrap(rb + krow, p.NR), pitch);
+            e.vrb = sbase + p.off_v + row_base(SlideWalk::wrap(rb + vrow, p.NR), pitch);
+            const int oy = orow ? qy0 + 1 : qy0;
+            e.orow = (e.work && oy < H) ? p.out + w.image(p.out_sb, p.out_sh) + (int64_t)oy * p.out_sy : nullptr;
+        };
         SlideWalk w;
         w.init(p, s_begin, s_end);
+        Geo cur;
+        geo_of(w, 0, cur);
+        int stage = 0;
+        uint32_t parity = 0;
         for (int i = 0; i < nst; ++i) {
-            const int stage = i % NS;
-            if (i) w.next(p);
-            const int pair = w.pa + pw;
-            const bool work = active && pair < w.pe;
-            const int qy0 = 2 * pair, qy1 = min(qy0 + 1, H - 1);
-            const int hy = pair_halo(pair, H);
-            if (work) {
-                const int sy0 = win_start(qy0, H), sy1 = win_start(qy1, H);
+            if (cur.work && cur.key != bias_key) {
                 // bias: rewritten when the head or the row geometry changes,
                 // before the wait for the step's rows (it needs none of them),
                 // so that it overlaps the copies
-                const int key = ((w.h * 8 + (qy0 - hy)) * 2 + (qy1 - qy0)) * 4 + (sy0 - hy) * 2 + (sy1 - hy);
-                if (key != bias_key) {
-                    bias_key = key;
-                    // this lane's queries 2c, 2c + 1 share tile row c / 2; its
-                    // keys lie on halo rows g / 2 (j < 2) and 4 + g / 2 (j >= 2)
-                    const int qy = (c >> 1) ? qy1 : qy0, sy = (c >> 1) ? sy1 : sy0;
-                    const float *rows[2];
-                    bool yin[2];
+                bias_key = cur.key;
+                const int qy0 = 2 * cur.pair, qy1 = min(qy0 + 1, H - 1);
+                const int hy = pair_halo(cur.pair, H);
+                // this lane's queries 2c, 2c + 1 share tile row c / 2; its
+                // keys lie on halo rows g / 2 (j < 2) and 4 + g / 2 (j >= 2)
+                const int qy = (c >> 1) ? qy1 : qy0, sy = win_start(qy, H);
+                const float *rows[2];
+                bool yin[2];
 #pragma unroll
-                    for (int jh = 0; jh < 2; ++jh) {
-                        const int ky = hy + 4 * jh + (g >> 1);
-                        yin[jh] = (unsigned)(ky - sy) < (unsigned)KW;
-                        rows[jh] = tab + w.h * kTabHead + clampi(ky - qy + 6, 0, 12) * kTabPitch;
-                    }
-#pragma unroll
-                    for (int u = 0; u < NT; ++u) {
-                        float b[kKG][4];
-#pragma unroll
-                        for (int t = 0; t < kKG; ++t)
-#pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                const float v = rows[j >> 1][cb[u][j & 1] + 2 * t];
-                                const bool in = yin[j >> 1] && ((xin[u] >> (2 * t + (j & 1))) & 1u);
-                                b[t][j] = in ? v : kMaskC;
-                            }
-#pragma unroll
-                        for (int t = 0; t < kKG; ++t) tmem_st4(tb + 32u * u + 4u * t, b[t]);
-                    }
-                    tmem_st_wait();
+                for (int jh = 0; jh < 2; ++jh) {
+                    const int ky = hy + 4 * jh + (g >> 1);
+                    yin[jh] = (unsigned)(ky - sy) < (unsigned)KW;
+                    rows[jh] = tab + cur.h * kTabHead + clampi(ky - qy + 6, 0, 12) * kTabPitch;
                 }
+#pragma unroll
+                for (int u = 0; u < NT; ++u) {
+                    float b[kKG][4];
+#pragma unroll
+                    for (int t = 0; t < kKG; ++t)
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const float v = rows[j >> 1][cb[u][j & 1] + 2 * t];
+                            const bool in = yin[j >> 1] && ((xin[u] >> (2 * t + (j & 1))) & 1u);
+                            b[t][j] = in ? v : kMaskC;
+                        }
+#pragma unroll
+                    for (int t = 0; t < kKG; ++t) tmem_st4(tb + 32u * u + 4u * t, b[t]);
+                }
+                tmem_st_wait();
             }
-            if (!sb_wait(bar_full + 8 * stage, (uint32_t)((i / NS) & 1), p.wait_limit)) {
+            if (!sb_wait(bar_full + 8 * stage, parity, p.wait_limit)) {
                 if (lane == 0) {
                     atomicAdd(&g_stream_timeouts, 1u);
                     *abort_flag = 1;
@@ -814,23 +835,16 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
                 break;
             }
             if (*abort_flag) break;
-            if (work) {
-                const uint32_t qrow = sbase + row_base(stage * 2 * p.SP + (qsel ? qy1 : qy0) - 2 * w.pa, pitch);
-                // ring rows of this lane's K and V fragment rows
-                const int rb = w.ring_lo - w.lo(p) + hy;
-                const uint32_t krb = sbase + p.off_k + row_base(SlideWalk::wrap(rb + krow, p.NR), pitch);
-                const uint32_t vrb = sbase + p.off_v + row_base(SlideWalk::wrap(rb + vrow, p.NR), pitch);
+            if (cur.work) {
                 uint32_t qa[NT], ka[NT], va[NT];
                 unsigned char *o[NT];
-                const int oy = orow ? qy0 + 1 : qy0;
-                unsigned char *orow_ptr = p.out + w.image(p.out_sb, p.out_sh) + (int64_t)oy * p.out_sy;
 #pragma unroll
                 for (int u = 0; u < NT; ++u) {
-                    qa[u] = qrow + qcol[u];
-                    ka[u] = krb + kcol[u];
-                    va[u] = vrb + vcol[u];
+                    qa[u] = cur.qrow + qcol[u];
+                    ka[u] = cur.krb + kcol[u];
+                    va[u] = cur.vrb + vcol[u];
                     const int ox = xq[u] + ocol0;
-                    o[u] = (oy < H && ox < W) ? orow_ptr + (int64_t)ox * p.out_sx : nullptr;
+                    o[u] = (cur.orow && ox < W) ? cur.orow + (int64_t)ox * p.out_sx : nullptr;
                 }
                 if (NT == 2 && shared_cols)
                     tile_run<T, NT, NT == 2>(qa, ka, va, tb, p.c_log2, o, lane);
@@ -839,6 +853,13 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
             }
             __syncwarp();
             if (lane == 0) sb_arrive(bar_empty + 8 * stage);
+            const int nstage = stage + 1 == NS ? 0 : stage + 1;
+            parity ^= nstage == 0 ? 1u : 0u;
+            stage = nstage;
+            if (i + 1 < nst) {
+                w.next(p);
+                geo_of(w, stage, cur);
+            }
         }
     }
     // ---- epilogue: TMEM released by the warp that took it, after every warp
