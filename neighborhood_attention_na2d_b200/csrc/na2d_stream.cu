@@ -565,8 +565,11 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
     extern __shared__ __align__(1024) unsigned char smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // this CTA's range of query-row pairs (the CTAs' loads differ by at most one pair)
-    const int s_begin = (int)((int64_t)p.nsteps * blockIdx.x / gridDim.x);
-    const int s_end = (int)((int64_t)p.nsteps * (blockIdx.x + 1) / gridDim.x);
+    // CTA b takes pairs [b * base + min(b, rem), ...): base = nsteps / grid,
+    // the first rem = nsteps % grid CTAs one more
+    const int base = p.nsteps / (int)gridDim.x, rem = p.nsteps - base * (int)gridDim.x;
+    const int bx = (int)blockIdx.x;
+    const int s_begin = bx * base + min(bx, rem), s_end = s_begin + base + (bx < rem ? 1 : 0);
     grid_dep_launch();
     if (s_begin >= s_end) return;
     const int nst = slide_steps(p, s_begin, s_end);
@@ -686,28 +689,29 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
         }
     } else {
         // =================== consumers ===================
-        // prologue (overlaps the first copies): bias table, tensor memory
+        // prologue (overlaps the first copies): bias table, zero margins,
+        // tensor memory.  Each thread's first table entry is requested before
+        // the zeroing, whose stores then cover the load's latency.
         {
             grid_dep_wait();   // first global read: the bias table
             const T *rpb = reinterpret_cast<const T *>(p.rpb);
-            for (int i = threadIdx.x; i < p.heads * kTabHead; i += NWC * 32) {
+            auto tab_entry = [&](int i) {
                 const int h = i / kTabHead, a = (i / kTabPitch) % 13, b = i % kTabPitch;
-                float v = 0.f;
-                if (rpb && b < 13) v = Elem<T>::to_f(rpb[(h * 13 + a) * 13 + b]) * p.sqrt_d;
-                tab[i] = v;
-            }
+                return (rpb && b < 13) ? Elem<T>::to_f(rpb[(h * 13 + a) * 13 + b]) * p.sqrt_d : 0.f;
+            };
+            const int ntab = p.heads * kTabHead;
+            const float first = (int)threadIdx.x < ntab ? tab_entry(threadIdx.x) : 0.f;
             // zero the margins of every ring row of K and V (the copies write
-            // only the image columns)
-            {
-                const int lead16 = kMargin * 4, row16 = (int)(pitch / 16), tail16 = row16 - lead16 - 4 * p.W;
-                const int per_row = lead16 + tail16;
-                for (int i = threadIdx.x; i < 2 * p.NR * per_row; i += NWC * 32) {
-                    const int r = (i / per_row) % p.NR, t = i % per_row;
-                    const uint32_t off = (i / per_row >= p.NR ? p.off_v : p.off_k) + row_base(r, pitch) +
-                                         16u * (uint32_t)(t < lead16 ? t : t + 4 * p.W);
-                    *reinterpret_cast<uint4 *>(smem + off) = make_uint4(0, 0, 0, 0);
-                }
+            // only the image columns): one warp per row
+            const int lead16 = kMargin * 4, tail0 = lead16 + 4 * p.W, per_row = lead16 + (int)(pitch / 16) - tail0;
+            for (int r = warp; r < 2 * p.NR; r += NWC) {
+                const uint32_t rowoff = r < p.NR ? p.off_k + row_base(r, pitch) : p.off_v + row_base(r - p.NR, pitch);
+                for (int t = lane; t < per_row; t += 32)
+                    *reinterpret_cast<uint4 *>(smem + rowoff + 16u * (uint32_t)(t < lead16 ? t : t - lead16 + tail0)) =
+                        make_uint4(0, 0, 0, 0);
             }
+            if ((int)threadIdx.x < ntab) tab[threadIdx.x] = first;
+            for (int i = threadIdx.x + NWC * 32; i < ntab; i += NWC * 32) tab[i] = tab_entry(i);
             if (warp == 0) tmem_alloc(smem_u32(tmem_slot));
             tmem_fence_before();
             consumers_sync(NWC * 32);
@@ -857,8 +861,25 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
             parity ^= nstage == 0 ? 1u : 0u;
             stage = nstage;
             if (i + 1 < nst) {
-                w.next(p);
-                geo_of(w, stage, cur);
+                const int npe = w.pe + p.SP;
+                if (w.pe - w.pa == p.SP && w.pa >= 2 && npe <= min(p.NP, w.ge - w.bh * p.NP) && 2 * npe <= H - 3) {
+                    // this step and the next are full and interior (every
+                    // pair's halo starts 3 rows above it, unclamped): the
+                    // rows, the ring and the output advance by 2 SP rows and
+                    // the bias key stays
+                    w.pa = w.pe;
+                    w.pe = npe;
+                    w.ring_lo = SlideWalk::wrap(w.ring_lo + 2 * p.SP, p.NR);
+                    cur.pair += p.SP;
+                    cur.qrow = sbase + row_base(stage * 2 * p.SP + 2 * pw + qsel, pitch);
+                    const int rb = w.ring_lo + 2 * pw;
+                    cur.krb = sbase + p.off_k + row_base(SlideWalk::wrap(rb + krow, p.NR), pitch);
+                    cur.vrb = sbase + p.off_v + row_base(SlideWalk::wrap(rb + vrow, p.NR), pitch);
+                    if (cur.orow) cur.orow += (int64_t)(2 * p.SP) * p.out_sy;
+                } else {
+                    w.next(p);
+                    geo_of(w, stage, cur);
+                }
             }
         }
     }
