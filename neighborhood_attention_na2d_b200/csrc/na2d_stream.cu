@@ -39,9 +39,13 @@
 // output tile is transposed back with movmatrix and stored.
 //
 // Shared-memory layout of the rows (Q, K, V; 64 bytes per pixel, four 16-byte
-// chunks): row r of a buffer starts at r * (W + 1) * 64 + 16 * (r & 3); any 4
+// chunks): row r of a buffer starts at r * pitch + 16 * (r & 3), with image
+// column x at pixel 3 + x and zero pixels on both sides (see row_base); any 4
 // consecutive rows x 2 adjacent pixels of one chunk index fall in 8 distinct
-// bank groups, which is the access pattern of every K and V fragment.
+// bank groups, which is the access pattern of every K and V fragment.  With
+// the zero margins every tile's halo starts 3 columns left of the tile, so the
+// two tiles of a warp always share their key groups (except at a ragged right
+// edge).
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -838,7 +842,8 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
                 }
                 break;
             }
-            if (*abort_flag) break;
+            // no per-step abort check: a producer that gave up never completes
+            // this step's barrier, so the wait above runs out and ends the warp
             if (cur.work) {
                 uint32_t qa[NT], ka[NT], va[NT];
                 unsigned char *o[NT];
