@@ -95,7 +95,7 @@ struct StreamParams {
     long long wait_limit;
     int nsteps;      // query-row pairs (split over the CTAs)
     int MX, SP, NP, NR;
-    uint32_t pitch;  // bytes per shared-memory row: kMargin zero pixels, W pixels, zero pixels up to MX*span + 3
+    uint32_t pitch;  // bytes per shared-memory row: kMargin zero pixels, W pixels, kMargin zero pixels
     float c_log2;    // log2(e) / sqrt(D)
     float sqrt_d;    // sqrt(D)
     uint32_t off_k, off_v, off_tab, off_bar;   // byte offsets in dynamic shared memory (Q at 0)
@@ -363,11 +363,10 @@ __device__ __forceinline__ void sb_expect_tx(uint32_t bar, uint32_t bytes) {
 // Skewed row layout: row r of a buffer starts at r * pitch + 16 * (r & 3)
 // bytes; image column x is pixel kMargin + x of the row (pixels and their
 // four 16-byte chunks in order), so a whole image row lands with one bulk
-// copy.  The kMargin pixels on the left and the pixels right of the image
-// (up to column MX * span + kMargin - 1) are zeros, written once: every tile's
-// 10-column halo starts at x0 - kMargin without clamping, and halo columns
-// outside the image read zero keys and values (their scores are masked by
-// the bias).  Any 4 consecutive rows x 2 adjacent pixels of one chunk index
+// copy.  The kMargin pixels on either side of the image are zeros, written
+// once: every tile's 10-column halo starts at x0 - kMargin (clamped only for
+// a last tile within 3 columns of the right edge), and halo columns outside
+// the image read zero keys and values (their scores are masked by the bias).  Any 4 consecutive rows x 2 adjacent pixels of one chunk index
 // fall in 8 distinct bank groups.  The skew makes a row overrun its pitch by
 // up to 48 bytes, into the next row's left margin (zeros both ways); each
 // buffer keeps 64 bytes of slack after its last row.
@@ -971,9 +970,10 @@ uint32_t plan_slide(StreamParams &sp, const Problem &pr, int SP, int span, bool 
     // halo for every image those steps touch (one when no CTA crosses images)
     const int images = aligned ? 1 : std::min(NS, (NS - 2) / spi + 2);
     sp.NR = (int)align_up((uint32_t)(2 * sp.SP * NS + 6 * images), 4);
-    // rows: kMargin zero pixels, the image, zero pixels up to column
-    // MX * span + kMargin - 1 (the last tile's halo); see row_base
-    sp.pitch = (uint32_t)(sp.MX * span + 2 * kMargin) * kPixB;
+    // rows: kMargin zero pixels, the image, kMargin zero pixels.  A tile's
+    // halo starts at min(x0 - 3, W - 7) >= -3 and spans 10 columns, so every
+    // halo column lies in [-3, W + 2]; see row_base
+    sp.pitch = (uint32_t)(pr.W + 2 * kMargin) * kPixB;
     const uint32_t qbytes = (uint32_t)(NS * 2 * sp.SP) * sp.pitch + 64;
     const uint32_t ring = (uint32_t)sp.NR * sp.pitch + 64;
     sp.off_k = align_up(qbytes, 128);
