@@ -121,6 +121,9 @@ __global__ void __launch_bounds__(kThreads) bwd_query_kernel(const BwdArgs a) {
         const int i = qi / W, j = qi - (qi / W) * W;
         const int gy = i % d, iy = i / d, sy = window_start(iy, group_len(a.Hp, d, gy), K);
         const int gx = j % d, ix = j / d, sx = window_start(ix, group_len(a.Wp, d, gx), K);
+        // neighbour rows ty < nty and columns tx < ntx lie on the real map
+        // (the rest are zero padding): gy + d (sy + ty) < H
+        const int nty = min(K, (H - 1 - gy) / d - sy + 1), ntx = min(K, (W - 1 - gx) / d - sx + 1);
         const T *qp = at<T>(a.q, b, h, i, j), *gp = at<T>(a.g, b, h, i, j);
         for (int c = lane; c < D; c += 32) {
             qs[warp][c] = Elem<T>::to_f(qp[c]);
@@ -129,17 +132,20 @@ __global__ void __launch_bounds__(kThreads) bwd_query_kernel(const BwdArgs a) {
         __syncwarp();
         const int64_t qlin = bh * H * W + qi;
         float s[kMaxPerLane], dp[kMaxPerLane];
+        int tys[kMaxPerLane], txs[kMaxPerLane];
         float m = -FLT_MAX;
 #pragma unroll
         for (int r = 0; r < kMaxPerLane; ++r) {
             const int n = lane + 32 * r;
             s[r] = -FLT_MAX;
             dp[r] = 0.f;
+            tys[r] = n / K;
+            txs[r] = n - tys[r] * K;
             if (n < KK) {
-                const int ty = n / K, tx = n - ty * K;
+                const int ty = tys[r], tx = txs[r];
                 const int ky = gy + d * (sy + ty), kx = gx + d * (sx + tx);
                 float dot = 0.f;
-                if (ky < H && kx < W) {
+                if (ty < nty && tx < ntx) {
                     dot = dot_s<T, D>(qs[warp], at<T>(a.k, b, h, ky, kx));
                     dp[r] = dot_s<T, D>(gs[warp], at<T>(a.v, b, h, ky, kx));
                 }
@@ -173,28 +179,33 @@ __global__ void __launch_bounds__(kThreads) bwd_query_kernel(const BwdArgs a) {
         for (int r = 0; r < kMaxPerLane; ++r) {
             const int n = lane + 32 * r;
             dp[r] = s[r] * (dp[r] - delta);      // ds_n
-            if (n < KK) {
-                const int ty = n / K, tx = n - ty * K;
-                atomicAdd(&bins[(sy + ty - iy + K - 1) * nb + (sx + tx - ix + K - 1)], dp[r]);
-            }
+            if (n < KK) atomicAdd(&bins[(sy + tys[r] - iy + K - 1) * nb + (sx + txs[r] - ix + K - 1)], dp[r]);
         }
+        // dq = sum_n ds_n k_n, lane = channel: the neighbours in order, each
+        // ds from its lane; the key pointer steps along the window
         float acc[NC];
 #pragma unroll
         for (int jj = 0; jj < NC; ++jj) acc[jj] = 0.f;
+        const int64_t stx = (int64_t)d * a.k.sx, sty = (int64_t)d * a.k.sy;
+        const T *krow = at<T>(a.k, b, h, gy + d * sy, gx + d * sx) + lane, *kp = krow;
+        int ty = 0, tx = 0;
 #pragma unroll
         for (int r = 0; r < kMaxPerLane; ++r) {
             if (32 * r >= KK) break;
             const int cnt = min(32, KK - 32 * r);
             for (int tl = 0; tl < cnt; ++tl) {
-                const int n = 32 * r + tl;
                 const float dsn = __shfl_sync(0xffffffffu, dp[r], tl);
-                const int ty = n / K, tx = n - ty * K;
-                const int ky = gy + d * (sy + ty), kx = gx + d * (sx + tx);
-                if (ky < H && kx < W) {
-                    const T *kp = at<T>(a.k, b, h, ky, kx);
+                if (ty < nty && tx < ntx) {
 #pragma unroll
                     for (int jj = 0; jj < NC; ++jj)
-                        if (lane + 32 * jj < D) acc[jj] = fmaf(dsn, Elem<T>::to_f(kp[lane + 32 * jj]), acc[jj]);
+                        if (lane + 32 * jj < D) acc[jj] = fmaf(dsn, Elem<T>::to_f(kp[32 * jj]), acc[jj]);
+                }
+                kp += stx;
+                if (++tx == K) {
+                    tx = 0;
+                    ++ty;
+                    krow += sty;
+                    kp = krow;
                 }
             }
         }
@@ -216,17 +227,13 @@ __global__ void __launch_bounds__(kThreads) bwd_query_kernel(const BwdArgs a) {
 // ---------------------------------------------------------------------------
 // The group positions of the queries whose clamped window holds key position
 // jp (group coordinates, group length Lg): a contiguous range [lo, hi].
+// With window starts s(ip) = clamp(ip - K/2, 0, Lg - K) (non-decreasing):
+// hi is the last ip with s(ip) <= jp, i.e. Lg - 1 once jp reaches the last
+// start Lg - K, else jp + K/2; lo is the first ip with s(ip) + K > jp, i.e. 0
+// while jp < K, else jp - K/2.
 __device__ __forceinline__ void inverse_range(int jp, int Lg, int K, int *lo, int *hi) {
-    int a = INT32_MAX, b = -1;
-    for (int ip = max(0, jp - K + 1); ip <= min(Lg - 1, jp + K - 1); ++ip) {
-        const int s = window_start(ip, Lg, K);
-        if (s <= jp && jp < s + K) {
-            a = min(a, ip);
-            b = ip;
-        }
-    }
-    *lo = a;
-    *hi = b;
+    *hi = jp >= Lg - K ? Lg - 1 : jp + K / 2;
+    *lo = jp < K ? 0 : jp - K / 2;
 }
 
 // Pass 2: one warp per real key pixel (b, head, y, x).  The key's inverse
@@ -267,12 +274,22 @@ __global__ void __launch_bounds__(kThreads) bwd_key_kernel(const BwdArgs a) {
             vc[c] = Elem<T>::to_f(vp[c]);
             dk[c] = dv[c] = 0.f;
         }
-        for (int t0 = 0; t0 < cnt; t0 += 8) {
-            const int tq = t0 + slot;
-            const bool on = tq < cnt;
-            const int iy = ylo + (on ? tq / nx : 0), ix = xlo + (on ? tq % nx : 0);
-            const int qy = gy + d * iy, qx = gx + d * ix;
+        // slot s takes queries s, s + 8, ... of the range in row-major order;
+        // two rounds are in flight at a time
+        int iy = ylo, ix = xlo + slot;
+        while (ix > xhi) {
+            ix -= nx;
+            ++iy;
+        }
+        auto round = [&](bool on, int ry, int rx) {
+            if (!on) {   // a slot past the range reads the first query, and adds nothing
+                ry = ylo;
+                rx = xlo;
+            }
+            const int qy = gy + d * ry, qx = gx + d * rx;
             const T *qp = at<T>(a.q, b, h, qy, qx) + c0, *gp = at<T>(a.g, b, h, qy, qx) + c0;
+            const int64_t qlin = bh * H * W + (int64_t)qy * W + qx;
+            const float lse = a.lse[qlin], dlt = a.delta[qlin];
             float qc[QC], gc[QC], sdot = 0.f, pdot = 0.f;
 #pragma unroll
             for (int c = 0; c < QC; ++c) {
@@ -285,22 +302,36 @@ __global__ void __launch_bounds__(kThreads) bwd_key_kernel(const BwdArgs a) {
             pdot += __shfl_xor_sync(0xffffffffu, pdot, 1);
             sdot += __shfl_xor_sync(0xffffffffu, sdot, 2);
             pdot += __shfl_xor_sync(0xffffffffu, pdot, 2);
-            const int64_t qlin = bh * H * W + (int64_t)qy * W + qx;
             float sv = sdot * a.scale;
-            if (bias) sv += Elem<T>::to_f(bias[(jy - iy + K - 1) * nb + (jx - ix + K - 1)]);
-            const float p = on ? __expf(sv - a.lse[qlin]) : 0.f;
+            if (bias) sv += Elem<T>::to_f(bias[(jy - ry + K - 1) * nb + (jx - rx + K - 1)]);
+            const float p = on ? __expf(sv - lse) : 0.f;
             float z = 1.f;
             if (a.dropout && on) {
-                const int n = (jy - window_start(iy, Lgy, K)) * K + (jx - window_start(ix, Lgx, K));
+                const int n = (jy - window_start(ry, Lgy, K)) * K + (jx - window_start(rx, Lgx, K));
                 z = dropout_keep((uint64_t)qlin * KK + n, a.seed, a.offset, a.drop_thresh) ? a.drop_scale : 0.f;
             }
-            const float ds = on ? p * (z * pdot - a.delta[qlin]) : 0.f;
+            const float ds = on ? p * (z * pdot - dlt) : 0.f;
             const float pz = p * z;
 #pragma unroll
             for (int c = 0; c < QC; ++c) {
                 dv[c] = fmaf(pz, gc[c], dv[c]);
                 dk[c] = fmaf(ds, qc[c], dk[c]);
             }
+        };
+        auto advance = [&]() {
+            ix += 8;
+            while (ix > xhi) {
+                ix -= nx;
+                ++iy;
+            }
+        };
+        for (int t0 = 0; t0 < cnt; t0 += 16) {
+            const int y0 = iy, x0 = ix;
+            advance();
+            const int y1 = iy, x1 = ix;
+            advance();
+            round(t0 + slot < cnt, y0, x0);
+            if (t0 + 8 < cnt) round(t0 + 8 + slot < cnt, y1, x1);
         }
 #pragma unroll
         for (int o = 4; o < 32; o <<= 1)
