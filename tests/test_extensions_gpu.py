@@ -202,3 +202,36 @@ def test_forward_ex_contiguous_takes_the_fast_kernels():
     q, k, v, rpb = (t.cuda() for t in make_inputs(shape))
     na.na2d_forward_ex(q, k, v, rpb, 7, 1)
     assert na.na2d_last_kernel() == "fwd_stream_kernel"
+
+
+# ---------------------------------------------------------------------------
+STRIDED = ["fused_qkv", "channels_last", "padded_rows"]
+
+
+@pytest.mark.parametrize("layout", STRIDED)
+def test_stream_kernel_strided_rows(layout):
+    """The k = 7 sliding-window kernel on q, k, v views whose rows are not
+    contiguous: the three views of a fused (B, H, W, 3 heads D) buffer,
+    channels-last (B, H, W, heads D) tensors, and [B, heads, H, W, D] slices
+    of tensors with two spare pixels per row.  The producer warp copies such
+    rows as 16-byte pieces; the output equals the oracle."""
+    B, heads, H, W, D, k, d = 2, 2, 14, 20, 32, 7, 1
+    shape = Shape(B, heads, H, W, D, k, d, "f16", 1500)
+    q, kk, v, rpb = make_inputs(shape)
+    if layout == "fused_qkv":
+        qkv = torch.cat([t.permute(0, 2, 3, 1, 4).reshape(B, H, W, heads * D) for t in (q, kk, v)], dim=-1).cuda()
+        qd, kd, vd = na.qkv_views(qkv, heads)
+    elif layout == "channels_last":
+        qd, kd, vd = (t.permute(0, 2, 3, 1, 4).contiguous().cuda().permute(0, 3, 1, 2, 4) for t in (q, kk, v))
+    else:
+        def padded(t):
+            big = torch.zeros(B, heads, H, W + 2, D, dtype=t.dtype)
+            big[:, :, :, :W] = t
+            return big.cuda()[:, :, :, :W]
+        qd, kd, vd = (padded(t) for t in (q, kk, v))
+    out = torch.full((B, heads, H, W, D), float("nan"), dtype=q.dtype, device="cuda")
+    na.na2d_forward_ex(qd, kd, vd, rpb.cuda(), k, d, out=out)
+    torch.cuda.synchronize()
+    assert na.na2d_last_kernel() == "fwd_stream_kernel"
+    want = oracle.forward(f64(q), f64(kk), f64(v), f64(rpb), k, d)
+    assert max_err(f64(out), want) <= TOL["f16"]
