@@ -32,10 +32,10 @@
 // unit j and then the epilogue of its unit j - 2, so it never waits for a
 // P.V that was just issued, and one warpgroup's softmax overlaps the other's
 // MMAs and epilogue.  Warp 8, lane 0 issues the TMA copies into a ring of
-// NSTG stages; warp 9, lane 0 issues the MMAs (each unit's P.V before the
-// Q K^T two units ahead, so a P.V never waits for a copy) and signals
-// completion with tcgen05.commit on mbarriers; warp 9 owns the TMEM
-// allocation.  Every wait is bounded: one that runs out counts the event,
+// NSTG stages; warps 9 and 10, lane 0, issue the MMAs of the even and the
+// odd units (each unit's P.V before the Q K^T two units ahead, so a P.V
+// never waits for a copy) and signal completion with tcgen05.commit on
+// mbarriers; warp 9 owns the TMEM allocation.  Every wait is bounded: one that runs out counts the event,
 // raises the block's abort flag, and the block winds down (its MMAs and
 // copies in flight are waited for before TMEM and shared memory are
 // released).
@@ -64,8 +64,8 @@ constexpr uint32_t kStage = 3 * kTile;   // Q, K, V tiles of a unit
 constexpr int kTabPitch = 16;            // floats per bias-table row (13 used)
 constexpr int kTabHead = 13 * kTabPitch;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kThreads = 320;            // 8 softmax warps, producer warp, MMA warp
-constexpr int kWarpTma = 8, kWarpMma = 9;
+constexpr int kThreads = 352;            // 8 softmax warps, producer warp, two MMA warps
+constexpr int kWarpTma = 8, kWarpMma = 9;   // MMA warps 9 (even units) and 10 (odd units)
 
 __device__ unsigned int g_umma_timeouts;
 
@@ -256,9 +256,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_umma_kernel(const __grid_cons
     const uint32_t bar_s = bar_empty + 8 * NSTG;        // [2] S ready (commit)
     const uint32_t bar_p = bar_s + 16;                  // [2] P written (4 warps)
     const uint32_t bar_o = bar_p + 16;                  // [4] O ready (commit)
-    const uint32_t bar_drain = bar_o + 32;              // all MMAs done (commit)
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + p.off_bar + 16 * NSTG + 72);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + p.off_bar + 16 * NSTG + 76);
+    const uint32_t bar_drain = bar_o + 32;              // [2] all MMAs of an MMA warp done (commit)
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + p.off_bar + 16 * NSTG + 80);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + p.off_bar + 16 * NSTG + 84);
 
     // One unit's copies into stage j % NSTG: Q, K, V of groups 2u and 2u + 1;
     // a unit without a second group loads the first one twice (finite
@@ -301,6 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_umma_kernel(const __grid_cons
             }
             for (int i = 0; i < 4; ++i) mb_init(bar_o + 8 * i, 1);
             mb_init(bar_drain, 1);
+            mb_init(bar_drain + 8, 1);
             *abort_flag = 0;
             asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
             grid_dep_wait();   // before the first copy
@@ -348,11 +349,17 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_umma_kernel(const __grid_cons
             for (int j = max(0, issued - NSTG); j < issued; ++j)
                 mb_wait(bar_full + 8 * (j % NSTG), (uint32_t)((j / NSTG) & 1));
         }
-    } else if (warp == kWarpMma) {
-        // =================== MMA issuer ===================
-        // Order: S_0, S_1, then per unit j: O_j = P_j V_j, S_{j+2} = Q K^T.
-        // S_{j+2} reuses S / P buffer j & 1 after the P.V that reads P_j
-        // (tcgen05.mma of one thread execute in issue order).
+    } else if (warp == kWarpMma || warp == kWarpMma + 1) {
+        // =================== MMA issuers ===================
+        // Warp kWarpMma + e issues the MMAs of the units j with j % 2 = e,
+        // whose S / P buffer is e and whose softmax is warpgroup e's: all
+        // ordering a unit needs stays within one issuing thread, and the two
+        // threads' MMAs overlap (one thread's issue, not the tensor core,
+        // bounds these small products).  Order per thread: S_e, then per
+        // unit j: O_j = P_j V_j, S_{j+2} = Q K^T; S_{j+2} reuses buffer e
+        // after the P.V that reads P_j (tcgen05.mma of one thread execute in
+        // issue order).
+        const int e = warp - kWarpMma;
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_f16<T>(128, 0);
             constexpr uint32_t idesc_pv = idesc_f16<T>(32, 1);
@@ -370,8 +377,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_umma_kernel(const __grid_cons
                 umma_commit(bar_s + 8 * (j & 1));
                 return true;
             };
-            bool ok = issue_qk(0) && (nst < 2 || issue_qk(1));
-            for (int j = 0; ok && j < nst; ++j) {
+            bool ok = e >= nst || issue_qk(e);
+            for (int j = e; ok && j < nst; j += 2) {
                 const int b = j & 1, s = j % NSTG;
                 if (!mb_wait(bar_p + 8 * b, (uint32_t)((j >> 1) & 1)) || *abort_flag) {
                     ok = false;
@@ -394,9 +401,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_umma_kernel(const __grid_cons
                 atomicAdd(&g_umma_timeouts, 1u);
                 *abort_flag = 1;
             }
-            // every MMA issued has completed before TMEM is released
-            umma_commit(bar_drain);
-            mb_wait(bar_drain, 0);
+            // every MMA this thread issued has completed before TMEM is released
+            umma_commit(bar_drain + 8 * e);
+            mb_wait(bar_drain + 8 * e, 0);
         }
     } else {
         // =================== softmax warpgroups ===================
@@ -596,7 +603,7 @@ cudaError_t launch_umma_t(const Problem &pr, const void *q, const void *k, const
     up.off_bar = align_up(up.off_tab + (uint32_t)(pr.heads * kTabHead * 4), 16);
     // + 1024 bytes for aligning the base; at least 116 KB so that two blocks
     // never share an SM (each takes all 512 TMEM columns)
-    const uint32_t smem = std::max<uint32_t>(up.off_bar + 16 * NSTG + 80 + 1024, 116u * 1024u);
+    const uint32_t smem = std::max<uint32_t>(up.off_bar + 16 * NSTG + 88 + 1024, 116u * 1024u);
     if ((int)smem > cap) return cudaSuccess;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)std::min(up.NU, sms));
