@@ -106,6 +106,9 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(const FwdArgs a) {
         for (int c = lane; c < D; c += 32) qsh[warp][c] = Elem<T>::to_f(qp[c]);
         __syncwarp();
         const Win wy = axis_win(i, a.Hp, K, d), wx = axis_win(j, a.Wp, K, d);
+        // neighbour rows ty < nty and columns tx < ntx lie on the real map
+        // (the rest are zero padding): wy.g + d (wy.s + ty) < H
+        const int nty = min(K, (a.H - 1 - wy.g) / d - wy.s + 1), ntx = min(K, (a.W - 1 - wx.g) / d - wx.s + 1);
         const T *kb = static_cast<const T *>(a.k.p) + b * a.k.sb + h * a.k.sh;
         const T *vb = static_cast<const T *>(a.v.p) + b * a.v.sb + h * a.v.sh;
         const T *bias = a.rpb ? static_cast<const T *>(a.rpb) + (size_t)h * nb * nb : nullptr;
@@ -119,7 +122,7 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(const FwdArgs a) {
                 const int ty = n / K, tx = n - ty * K;
                 const int ky = wy.g + d * (wy.s + ty), kx = wx.g + d * (wx.s + tx);
                 float dot = 0.f;
-                if (ky < a.H && kx < a.W) dot = dot_q<T, D>(qsh[warp], kb + ky * a.k.sy + kx * a.k.sx);
+                if (ty < nty && tx < ntx) dot = dot_q<T, D>(qsh[warp], kb + ky * a.k.sy + kx * a.k.sx);
                 float sv = dot * a.scale;
                 if (bias) sv += Elem<T>::to_f(bias[(wy.s + ty - wy.ip + K - 1) * nb + (wx.s + tx - wx.ip + K - 1)]);
                 sc[r] = sv;
@@ -148,20 +151,29 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(const FwdArgs a) {
         float acc[NC];
 #pragma unroll
         for (int jj = 0; jj < NC; ++jj) acc[jj] = 0.f;
+        // lane = channel: the neighbours in order, each weight from its lane;
+        // the value pointer steps along the window
+        const int64_t stx = (int64_t)d * a.v.sx, sty = (int64_t)d * a.v.sy;
+        const T *vrow = vb + (int64_t)(wy.g + d * wy.s) * a.v.sy + (int64_t)(wx.g + d * wx.s) * a.v.sx + lane;
+        const T *vp = vrow;
+        int ty = 0, tx = 0;
 #pragma unroll
         for (int r = 0; r < kMaxPerLane; ++r) {
             if (32 * r >= KK) break;
             const int cnt = min(32, KK - 32 * r);
             for (int tl = 0; tl < cnt; ++tl) {
-                const int n = 32 * r + tl;
                 const float pn = __shfl_sync(0xffffffffu, sc[r], tl);
-                const int ty = n / K, tx = n - ty * K;
-                const int ky = wy.g + d * (wy.s + ty), kx = wx.g + d * (wx.s + tx);
-                if (pn != 0.f && ky < a.H && kx < a.W) {
-                    const T *vp = vb + ky * a.v.sy + kx * a.v.sx;
+                if (pn != 0.f && ty < nty && tx < ntx) {
 #pragma unroll
                     for (int jj = 0; jj < NC; ++jj)
-                        if (lane + 32 * jj < D) acc[jj] = fmaf(pn, Elem<T>::to_f(vp[lane + 32 * jj]), acc[jj]);
+                        if (lane + 32 * jj < D) acc[jj] = fmaf(pn, Elem<T>::to_f(vp[32 * jj]), acc[jj]);
+                }
+                vp += stx;
+                if (++tx == K) {
+                    tx = 0;
+                    ++ty;
+                    vrow += sty;
+                    vp = vrow;
                 }
             }
         }
