@@ -250,12 +250,9 @@ __global__ void __launch_bounds__(kThreads) bwd_key_kernel(const BwdArgs a) {
     const int c0 = quarter * QC;
     const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
     for (int64_t idx = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5; idx < a.nq; idx += nwarps) {
-        const int x = (int)(idx % W);
-        const int64_t t = idx / W;
-        const int y = (int)(t % H);
-        const int64_t bh = t / H;
-        const int64_t b = bh / a.heads;
-        const int h = (int)(bh % a.heads);
+        int x, y, h;
+        int64_t bh, b;
+        split_pixel(idx, W, H, a.heads, x, y, bh, b, h);
         const T *bias = a.rpb ? static_cast<const T *>(a.rpb) + (size_t)h * nb * nb : nullptr;
         const int gy = y % d, jy = y / d, Lgy = group_len(a.Hp, d, gy);
         const int gx = x % d, jx = x / d, Lgx = group_len(a.Wp, d, gx);

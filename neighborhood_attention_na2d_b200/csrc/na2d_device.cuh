@@ -24,6 +24,27 @@ __host__ __device__ __forceinline__ int window_start(int ip, int Lg, int k) {
     return s > Lg - k ? Lg - k : s;
 }
 
+// Pixel (b, h, y, x) of linear index idx = ((b * heads + h) * H + y) * W + x,
+// with bh = b * heads + h; 32-bit divisions while the index fits in 31 bits.
+__device__ __forceinline__ void split_pixel(int64_t idx, int W, int H, int heads, int &x, int &y, int64_t &bh,
+                                            int64_t &b, int &h) {
+    if (idx < 0x7fffffff) {
+        const int i = (int)idx, t = i / W, bhi = t / H;
+        x = i - t * W;
+        y = t - bhi * H;
+        b = bhi / heads;
+        h = bhi - (int)b * heads;
+        bh = bhi;
+    } else {
+        const int64_t t = idx / W;
+        x = (int)(idx - t * W);
+        bh = t / H;
+        y = (int)(t - bh * H);
+        b = bh / heads;
+        h = (int)(bh - b * heads);
+    }
+}
+
 // ---------------------------------------------------------------------------
 // Element types.
 // ---------------------------------------------------------------------------

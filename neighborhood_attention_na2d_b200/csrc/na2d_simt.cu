@@ -96,12 +96,9 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(const FwdArgs a) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t nwarps = (int64_t)gridDim.x * kWarps;
     for (int64_t idx = blockIdx.x * (int64_t)kWarps + warp; idx < a.nq; idx += nwarps) {
-        const int j = (int)(idx % a.W);
-        const int64_t t = idx / a.W;
-        const int i = (int)(t % a.H);
-        const int64_t bh = t / a.H;
-        const int64_t b = bh / a.heads;
-        const int h = (int)(bh % a.heads);
+        int j, i, h;
+        int64_t bh, b;
+        split_pixel(idx, a.W, a.H, a.heads, j, i, bh, b, h);
         const T *qp = static_cast<const T *>(a.q.p) + b * a.q.sb + h * a.q.sh + i * a.q.sy + j * a.q.sx;
         for (int c = lane; c < D; c += 32) qsh[warp][c] = Elem<T>::to_f(qp[c]);
         __syncwarp();
