@@ -95,6 +95,9 @@ struct StreamParams {
     long long wait_limit;
     int nsteps;      // query-row pairs (split over the CTAs)
     int MX, SP, NP, NR;
+    // column bands (maps wider than 64): nb bands of whole 8-column warp
+    // spans, band k of band_oct + (k < band_extra) spans; 1 band otherwise
+    int nb, band_oct, band_extra;
     uint32_t pitch;  // bytes per shared-memory row: kMargin zero pixels, W pixels, kMargin zero pixels
     float c_log2;    // log2(e) / sqrt(D)
     float sqrt_d;    // sqrt(D)
@@ -292,11 +295,12 @@ __device__ __forceinline__ int pair_halo(int pair, int H) { return min(win_start
 // consumers run the same walk.  Only the image, the step's pairs and the ring
 // row of the step's first key row are kept; the rest is recomputed.
 struct SlideWalk {
-    int bh;           // image
+    int bh;           // image (a column band of one (batch, head) map when nb > 1)
     int pa, pe;       // the step's first pair and one past its last
     int ge;           // end of the CTA's range (global pair index)
     int h;            // head of image bh
     int b;            // batch of image bh
+    int band;         // column band of image bh
     int ring_lo;      // ring row of lo()
     __device__ __forceinline__ int lo(const StreamParams &p) const { return pair_halo(pa, p.H); }
     __device__ __forceinline__ int hi(const StreamParams &p) const { return pair_halo(pe - 1, p.H) + 7; }
@@ -308,8 +312,10 @@ struct SlideWalk {
         bh = gb / p.NP;
         pa = gb - bh * p.NP;
         pe = step_end(p);
-        h = bh % p.heads;
-        b = bh / p.heads;
+        const int map = bh / p.nb;
+        band = bh - map * p.nb;
+        h = map % p.heads;
+        b = map / p.heads;
         ring_lo = 0;
     }
     // byte offset of image (b, h) for the given batch / head strides
@@ -324,9 +330,12 @@ struct SlideWalk {
         const int hi_ring = wrap(ring_lo + old_hi - old_lo, p.NR);
         if (pe == p.NP) {
             ++bh;
-            if (++h == p.heads) {
-                h = 0;
-                ++b;
+            if (++band == p.nb) {
+                band = 0;
+                if (++h == p.heads) {
+                    h = 0;
+                    ++b;
+                }
             }
             pa = 0;
             pe = step_end(p);
@@ -339,6 +348,13 @@ struct SlideWalk {
         return old_hi + 1;
     }
 };
+
+// Column band k: first image column and width (whole 8-column warp spans;
+// the last band ends at the image's right edge).
+__device__ __forceinline__ void band_cols(const StreamParams &p, int k, int &bx0, int &bw) {
+    bx0 = 8 * (k * p.band_oct + min(k, p.band_extra));
+    bw = min(8 * (p.band_oct + (k < p.band_extra ? 1 : 0)), p.W - bx0);
+}
 
 // Number of steps in the pair range [gb, ge): per image, ceil(pairs / SP).
 __device__ __forceinline__ int slide_steps(const StreamParams &p, int gb, int ge) {
@@ -562,7 +578,7 @@ __device__ __forceinline__ void consumers_sync(int nthreads) {
 // up once.  The producer starts copying right after the barriers are set up;
 // the consumers build the bias table and allocate tensor memory meanwhile.
 // ---------------------------------------------------------------------------
-template <typename T, int NWC, int NT>
+template <typename T, int NWC, int NT, bool BANDED>
 __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __grid_constant__ StreamParams p) {
     static_assert(32 * NT * ((NWC + 3) / 4) <= kTmemCols, "bias columns of all consumer warps fit in TMEM");
     extern __shared__ __align__(1024) unsigned char smem[];
@@ -647,8 +663,76 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
     } else if (warp == NWC) {
         // =================== producer ===================
         // one thread issues one bulk copy per image row: the step's new K and
-        // V rows into the ring, its query rows into the stage
-        if (lane == 0) {
+        // V rows into the ring, its query rows into the stage.  Column bands
+        // (BANDED): each copy takes the band's columns and 3 on either side
+        // that lie on the map; in a band at the map's left or right edge the
+        // warp first zeroes the ring rows' columns off the map.
+        if constexpr (BANDED) {
+            grid_dep_wait();   // no global read before the previous kernel completes
+            const bool leader = lane == 0;
+            // a banded row's pixels end one pixel short of its pitch, so the
+            // 16 (r & 3) skew never reaches the next row's first pixel
+            const int row16 = (int)(pitch / 16) - 4;
+            SlideWalk w;
+            w.init(p, s_begin, s_end);
+            int issued = 0;
+            for (int i = 0; i < nst; ++i) {
+                const int stage = i % NS;
+                const int first = i ? w.next(p) : w.lo(p);
+                const bool ok_lane = i >= NS ? sb_wait(bar_empty + 8 * stage, (uint32_t)(((i / NS) - 1) & 1), p.wait_limit)
+                                             : (i == 0 || sb_wait(bar_full + 8 * (i - 1), 0u, p.wait_limit));
+                const bool ok = __all_sync(0xffffffffu, ok_lane);
+                if (!ok) {
+                    if (leader) {
+                        atomicAdd(&g_stream_timeouts, 1u);
+                        *abort_flag = 1;
+                    }
+                    break;
+                }
+                if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+                const int hi = w.hi(p);
+                const int y0 = 2 * w.pa, y1 = min(2 * w.pe, p.H);
+                int bx0, bw;
+                band_cols(p, w.band, bx0, bw);
+                const int cs = max(0, bx0 - kMargin), ce = min(p.W, bx0 + bw + kMargin);
+                const uint32_t rowbytes = (uint32_t)(ce - cs) * kPixB;
+                const uint32_t dcol = kLead + (uint32_t)(cs - bx0) * kPixB;   // shared column of image column cs
+                // 16-byte pieces off the map: [0, zl) and [zr, row16) of each new row
+                // (row16: the row's pixels, without the spare one)
+                const int zl = bx0 == 0 ? 4 * kMargin : 0;
+                const int zr = bx0 + bw == p.W ? 4 * (p.W - bx0 + kMargin) : row16;
+                const int nz = zl + row16 - zr;
+                for (int row = first; row <= hi; ++row) {
+                    const uint32_t o = row_base(w.ring(p, row), pitch);
+                    for (int t = lane; t < nz; t += 32) {
+                        const uint32_t off = o + 16u * (uint32_t)(t < zl ? t : zr + t - zl);
+                        *reinterpret_cast<uint4 *>(smem + p.off_k + off) = make_uint4(0, 0, 0, 0);
+                        *reinterpret_cast<uint4 *>(smem + p.off_v + off) = make_uint4(0, 0, 0, 0);
+                    }
+                }
+                __syncwarp();
+                if (leader) {
+                    const uint32_t bar = bar_full + 8 * stage;
+                    const int64_t img = w.image(p.in_sb, p.in_sh) + (int64_t)cs * p.in_sx;
+                    sb_expect_tx(bar, (uint32_t)(2 * (hi - first + 1) + (y1 - y0)) * rowbytes);
+                    for (int row = first; row <= hi; ++row) {
+                        const uint32_t o = row_base(w.ring(p, row), pitch) + dcol;
+                        const int64_t src = img + (int64_t)row * p.in_sy;
+                        bulk_g2s(sbase + p.off_k + o, p.k + src, rowbytes, bar);
+                        bulk_g2s(sbase + p.off_v + o, p.v + src, rowbytes, bar);
+                    }
+                    for (int y = y0; y < y1; ++y)
+                        bulk_g2s(sbase + row_base(stage * 2 * p.SP + (y - y0), pitch) + dcol,
+                                 p.q + img + (int64_t)y * p.in_sy, rowbytes, bar);
+                    ++issued;
+                }
+            }
+            // copies still in flight must land before the CTA's shared
+            // memory is released (all of them, unless a wait ran out)
+            if (leader)
+                for (int j = max(0, issued - NS); j < issued; ++j)
+                    sb_wait(bar_full + 8 * (j % NS), (uint32_t)((j / NS) & 1));
+        } else if (lane == 0) {
             grid_dep_wait();   // no global read before the previous kernel completes
             const uint32_t rowbytes = (uint32_t)p.W * kPixB;
             SlideWalk w;
@@ -705,9 +789,10 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
             const int ntab = p.heads * kTabHead;
             const float first = (int)threadIdx.x < ntab ? tab_entry(threadIdx.x) : 0.f;
             // zero the margins of every ring row of K and V (the copies write
-            // only the image columns): one warp per row
+            // only the image columns): one warp per row.  Banded rows get
+            // their margins from the producer, band by band.
             const int lead16 = kMargin * 4, tail0 = lead16 + 4 * p.W, per_row = lead16 + (int)(pitch / 16) - tail0;
-            for (int r = warp; r < 2 * p.NR; r += NWC) {
+            for (int r = BANDED ? 2 * p.NR : warp; r < 2 * p.NR; r += NWC) {
                 const uint32_t rowoff = r < p.NR ? p.off_k + row_base(r, pitch) : p.off_v + row_base(r - p.NR, pitch);
                 for (int t = lane; t < per_row; t += 32)
                     *reinterpret_cast<uint4 *>(smem + rowoff + 16u * (uint32_t)(t < lead16 ? t : t - lead16 + tail0)) =
@@ -736,34 +821,43 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
         // the query's window along x
         int cb[NT][2];
         uint32_t xin[NT];
+        bool shared_cols = false;
+        int bx0 = 0, bw = W;   // this warp's column band (the whole map unless BANDED)
+        // column geometry of the warp's tiles in band k (image column x sits
+        // at shared column x - bx0 + kMargin)
+        auto set_band = [&](int k) {
+            if constexpr (BANDED) band_cols(p, k, bx0, bw);
 #pragma unroll
-        for (int u = 0; u < NT; ++u) {
-            xq[u] = x0 + kTileCols * u;
-            // halo columns hx .. hx + 9: x0 - 3 .. x0 + 6, except for a last
-            // tile that starts within 3 columns of the right edge, whose
-            // queries all share the window W - 7 .. W - 1
-            const int hx = min(xq[u] - kMargin, W - KW);
-            qcol[u] = (uint32_t)(min(xq[u] + (lane & 3), W - 1) + kMargin) * kPixB + 16u * (uint32_t)(lane >> 3);
-            kcol[u] = (uint32_t)(hx + kMargin + (mk & 1)) * kPixB + 16u * (uint32_t)(lane >> 4);
-            vcol[u] = (uint32_t)(hx + kMargin + (mv & 1)) * kPixB + 16u * (uint32_t)((lane >> 3) & 1);
-            xin[u] = 0;
+            for (int u = 0; u < NT; ++u) {
+                xq[u] = bx0 + x0 + kTileCols * u;
+                // halo columns hx .. hx + 9: x0 - 3 .. x0 + 6, except for a last
+                // tile that starts within 3 columns of the right edge, whose
+                // queries all share the window W - 7 .. W - 1
+                const int hx = min(xq[u] - kMargin, W - KW);
+                qcol[u] = (uint32_t)(min(xq[u] + (lane & 3), W - 1) - bx0 + kMargin) * kPixB + 16u * (uint32_t)(lane >> 3);
+                kcol[u] = (uint32_t)(hx - bx0 + kMargin + (mk & 1)) * kPixB + 16u * (uint32_t)(lane >> 4);
+                vcol[u] = (uint32_t)(hx - bx0 + kMargin + (mv & 1)) * kPixB + 16u * (uint32_t)((lane >> 3) & 1);
+                xin[u] = 0;
 #pragma unroll
-            for (int jlo = 0; jlo < 2; ++jlo) {
-                const int qx = min(xq[u] + 2 * (c & 1) + jlo, W - 1), sx = win_start(qx, W);
-                // kx - qx + 6 for key column kx = hx + 2t + (g & 1): within
-                // [0, 12]
-                cb[u][jlo] = hx + (g & 1) - qx + 6;
+                for (int jlo = 0; jlo < 2; ++jlo) {
+                    const int qx = min(xq[u] + 2 * (c & 1) + jlo, W - 1), sx = win_start(qx, W);
+                    // kx - qx + 6 for key column kx = hx + 2t + (g & 1): within
+                    // [0, 12]
+                    cb[u][jlo] = hx + (g & 1) - qx + 6;
 #pragma unroll
-                for (int t = 0; t < kKG; ++t) {
-                    const int kx = hx + 2 * t + (g & 1);
-                    xin[u] |= ((unsigned)(kx - sx) < (unsigned)KW ? 1u : 0u) << (2 * t + jlo);
+                    for (int t = 0; t < kKG; ++t) {
+                        const int kx = hx + 2 * t + (g & 1);
+                        xin[u] |= ((unsigned)(kx - sx) < (unsigned)KW ? 1u : 0u) << (2 * t + jlo);
+                    }
                 }
             }
-        }
-        // the two tiles' halos are 4 columns apart (all but a warp that holds
-        // a last tile starting within 3 columns of the right edge): their key
-        // groups can be shared
-        const bool shared_cols = NT == 2 && min(xq[NT - 1] - kMargin, W - KW) == xq[0] - kMargin + kTileCols;
+            // the two tiles' halos are 4 columns apart (all but a warp that
+            // holds a last tile starting within 3 columns of the right edge):
+            // their key groups can be shared
+            shared_cols = NT == 2 && min(xq[NT - 1] - kMargin, W - KW) == xq[0] - kMargin + kTileCols;
+        };
+        int cur_band = 0;
+        set_band(0);
         const int qsel = (lane >> 2) & 1;
         // output pixel of this lane's epilogue query (lane / 4): tile row g / 4, column g % 4
         const int orow = g >> 2, ocol0 = g & 3;
@@ -772,19 +866,25 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
         // after the previous step's tiles, while their last products and
         // stores drain.
         struct Geo {
-            int pair, h, key;
+            int pair, h, key, band;
             bool work;
             uint32_t qrow, krb, vrb;
             unsigned char *orow;   // output row of this lane's epilogue query, or null
         };
         auto geo_of = [&](const SlideWalk &w, int stage, Geo &e) {
             e.pair = w.pa + pw;
+            e.band = w.band;
             e.work = active && e.pair < w.pe;
+            if constexpr (BANDED) {
+                int b0, bwk;
+                band_cols(p, w.band, b0, bwk);
+                e.work = e.work && x0 < bwk;   // a warp past a narrow last band has no tiles
+            }
             e.h = w.h;
             const int qy0 = 2 * e.pair, qy1 = min(qy0 + 1, H - 1);
             const int hy = pair_halo(e.pair, H);
-            e.key = ((w.h * 8 + (qy0 - hy)) * 2 + (qy1 - qy0)) * 4 + (win_start(qy0, H) - hy) * 2 +
-                    (win_start(qy1, H) - hy);
+            e.key = (((w.h * 8 + (qy0 - hy)) * 2 + (qy1 - qy0)) * 4 + (win_start(qy0, H) - hy) * 2 +
+                     (win_start(qy1, H) - hy)) * p.nb + w.band;
             e.qrow = sbase + row_base(stage * 2 * p.SP + (qsel ? qy1 : qy0) - 2 * w.pa, pitch);
             // ring rows of this lane's K and V fragment rows
             const int rb = w.ring_lo - w.lo(p) + hy;
@@ -800,6 +900,12 @@ __global__ void __launch_bounds__((NWC + 1) * 32, 1) fwd_stream_kernel(const __g
         int stage = 0;
         uint32_t parity = 0;
         for (int i = 0; i < nst; ++i) {
+            if constexpr (BANDED) {
+                if (cur.band != cur_band) {
+                    cur_band = cur.band;
+                    set_band(cur_band);
+                }
+            }
             if (cur.work && cur.key != bias_key) {
                 // bias: rewritten when the head or the row geometry changes,
                 // before the wait for the step's rows (it needs none of them),
@@ -941,7 +1047,7 @@ std::atomic<long long> &wait_limit_store() {
 }
 long long stream_wait_limit() { return wait_limit_store().load(); }
 
-template <typename T, int NWC, int NT>
+template <typename T, int NWC, int NT, bool BANDED>
 cudaError_t launch_stream_t(const StreamParams &sp, uint32_t smem, int grid, cudaStream_t st, bool *launched) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
@@ -953,7 +1059,7 @@ cudaError_t launch_stream_t(const StreamParams &sp, uint32_t smem, int grid, cud
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, fwd_stream_kernel<T, NWC, NT>, sp);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, fwd_stream_kernel<T, NWC, NT, BANDED>, sp);
     *launched = true;
     note_kernel("fwd_stream_kernel");
     return e != cudaSuccess ? e : cudaGetLastError();
@@ -961,8 +1067,7 @@ cudaError_t launch_stream_t(const StreamParams &sp, uint32_t smem, int grid, cud
 
 // Plan for SP query-row pairs per step; returns the shared-memory bytes.
 // `aligned`: every CTA's range lies inside one image.
-uint32_t plan_slide(StreamParams &sp, const Problem &pr, int SP, int span, bool aligned) {
-    sp.MX = (pr.W + span - 1) / span;
+uint32_t plan_slide(StreamParams &sp, const Problem &pr, int SP, bool aligned) {
     sp.SP = SP;
     sp.NP = (pr.H + 1) / 2;
     const int spi = (sp.NP + sp.SP - 1) / sp.SP;   // steps per image
@@ -972,8 +1077,10 @@ uint32_t plan_slide(StreamParams &sp, const Problem &pr, int SP, int span, bool 
     sp.NR = (int)align_up((uint32_t)(2 * sp.SP * NS + 6 * images), 4);
     // rows: kMargin zero pixels, the image, kMargin zero pixels.  A tile's
     // halo starts at min(x0 - 3, W - 7) >= -3 and spans 10 columns, so every
-    // halo column lies in [-3, W + 2]; see row_base
-    sp.pitch = (uint32_t)(pr.W + 2 * kMargin) * kPixB;
+    // halo column lies in [-3, W + 2]; see row_base.  Banded rows hold a
+    // band's MX spans of 8 columns and kMargin columns on either side, plus
+    // one spare pixel that keeps the row skew off the next row's pixels.
+    sp.pitch = sp.nb > 1 ? (uint32_t)(8 * sp.MX + 2 * kMargin + 1) * kPixB : (uint32_t)(pr.W + 2 * kMargin) * kPixB;
     const uint32_t qbytes = (uint32_t)(NS * 2 * sp.SP) * sp.pitch + 64;
     const uint32_t ring = (uint32_t)sp.NR * sp.pitch + 64;
     sp.off_k = align_up(qbytes, 128);
@@ -985,14 +1092,24 @@ uint32_t plan_slide(StreamParams &sp, const Problem &pr, int SP, int span, bool 
 
 template <typename T, int NWC, int NT>
 cudaError_t launch_slide(StreamParams &sp, const Problem &pr, cudaStream_t st, bool *launched) {
-    const void *kern = reinterpret_cast<const void *>(&fwd_stream_kernel<T, NWC, NT>);
+    const int span = kTileCols * NT;   // query columns per consumer warp
+    // maps wider than 64 columns: column bands of whole spans, at most 56
+    // columns each (7 warps per query-row pair), as even as whole spans allow
+    const int spans = (pr.W + span - 1) / span;
+    sp.nb = pr.W > 64 ? (pr.W + 55) / 56 : 1;
+    sp.band_oct = spans / sp.nb;
+    sp.band_extra = spans - sp.band_oct * sp.nb;
+    sp.MX = sp.band_oct + (sp.band_extra ? 1 : 0);
+    const bool banded = sp.nb > 1;
+    const void *kern = banded ? reinterpret_cast<const void *>(&fwd_stream_kernel<T, NWC, NT, true>)
+                              : reinterpret_cast<const void *>(&fwd_stream_kernel<T, NWC, NT, false>);
     int sms = 0, cap = 0;
     cudaError_t e = stream_device(&sms, &cap, kern);
     if (e != cudaSuccess) return e;
-    const int span = kTileCols * NT;   // query columns per consumer warp
-    const int MX = (pr.W + span - 1) / span;
     sp.NP = (pr.H + 1) / 2;
-    const int64_t npairs = pr.bh() * sp.NP;
+    // an image of the walk is a column band of one (batch, head) map
+    const int64_t images = pr.bh() * sp.nb;
+    const int64_t npairs = images * sp.NP;
     if (npairs >= INT32_MAX || npairs <= 0) return cudaSuccess;
     sp.nsteps = (int)npairs;
     // CTAs: one per SM with an even split of the pairs, or, when the images
@@ -1000,7 +1117,6 @@ cudaError_t launch_slide(StreamParams &sp, const Problem &pr, cudaStream_t st, b
     // range lies inside one image (no second halo and no second clamped image
     // top, which cost about a step).  The aligned split is taken while it
     // gives a CTA at most one pair more.
-    const int64_t images = pr.bh();
     int grid = (int)std::min<int64_t>(npairs, sms);
     bool aligned = false;
     if (images <= sms) {
@@ -1013,10 +1129,11 @@ cudaError_t launch_slide(StreamParams &sp, const Problem &pr, cudaStream_t st, b
             grid = (int)(images * (aligned ? sp.NP / per : c));
         }
     }
-    for (int SP = std::max(1, NWC / MX); SP >= 1; --SP) {
-        const uint32_t smem = plan_slide(sp, pr, SP, span, aligned);
+    for (int SP = std::max(1, NWC / sp.MX); SP >= 1; --SP) {
+        const uint32_t smem = plan_slide(sp, pr, SP, aligned);
         if ((int)smem > cap) continue;
-        return launch_stream_t<T, NWC, NT>(sp, smem, grid, st, launched);
+        return banded ? launch_stream_t<T, NWC, NT, true>(sp, smem, grid, st, launched)
+                      : launch_stream_t<T, NWC, NT, false>(sp, smem, grid, st, launched);
     }
     return cudaSuccess;
 }
@@ -1034,6 +1151,7 @@ cudaError_t launch_stream_impl(const Problem &pr, const View &q, const View &k, 
     sp.in_sb = q.sb * e; sp.in_sh = q.sh * e; sp.in_sy = q.sy * e; sp.in_sx = q.sx * e;
     sp.out_sb = out.sb * e; sp.out_sh = out.sh * e; sp.out_sy = out.sy * e; sp.out_sx = out.sx * e;
     sp.rows_contiguous = (q.sx == 32 && q.sy == (int64_t)32 * pr.W) ? 1 : 0;
+    if (pr.W > 64 && !sp.rows_contiguous) return cudaSuccess;   // bands copy contiguous row segments
     const long long lim = stream_wait_limit();
     sp.wait_limit = lim > 0 ? lim : kWaitLimit;
     sp.H = pr.H; sp.W = pr.W; sp.heads = pr.heads;
@@ -1056,7 +1174,7 @@ bool stream_views_supported(const Problem &p, const View &q, const View &k, cons
 bool stream_supported(const Problem &p) {
     if (p.dtype != DType::F16 && p.dtype != DType::BF16) return false;
     if (p.k != KW || p.D != 32 || p.heads > 64) return false;
-    return p.d == 1 && p.W >= 14 && p.W <= 64 && p.H >= 8;          // sliding rows
+    return p.d == 1 && p.W >= 14 && p.H >= 8;                      // sliding rows (bands above 64 columns)
 }
 
 cudaError_t launch_forward_stream(const Problem &p, const View &q, const View &k, const View &v, const void *rpb,

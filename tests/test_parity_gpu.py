@@ -122,6 +122,13 @@ def _stream_cases():
     cases.append((Shape(1, 64, 7, 7, 32, 7, 1, "bf16", 7100), True))
     cases.append((Shape(3, 101, 7, 7, 32, 7, 1, "f16", 7101), True))
     cases.append((Shape(75, 2, 14, 14, 32, 7, 1, "f16", 7102), True))
+    # maps wider than 64 columns: column bands (a partial last band, three
+    # and four bands, more band images than SMs)
+    cases.append((Shape(1, 2, 12, 65, 32, 7, 1, "f16", 7103), True))
+    cases.append((Shape(2, 1, 17, 100, 32, 7, 1, "bf16", 7104), True))
+    cases.append((Shape(1, 1, 10, 128, 32, 7, 1, "f16", 7105), False))
+    cases.append((Shape(1, 1, 9, 200, 32, 7, 1, "bf16", 7106), True))
+    cases.append((Shape(60, 1, 8, 72, 32, 7, 1, "f16", 7107), True))
     return cases
 
 
@@ -230,6 +237,7 @@ def test_bench_buffers_sampled(name):
 DISPATCH = [
     (Shape(1, 3, 14, 14, 32, 7, 2, "bf16", 601), "fwd_umma_kernel"),            # every group exactly 7 x 7
     (Shape(1, 2, 16, 16, 32, 7, 1, "f16", 602), "fwd_stream_kernel"),           # k = 7 sliding rows
+    (Shape(1, 2, 12, 100, 32, 7, 1, "bf16", 613), "fwd_stream_kernel"),         # k = 7 sliding rows, column bands
     (Shape(1, 2, 28, 28, 32, 7, 2, "bf16", 603), "fwd_sync_kernel/full_tma"),   # k <= 7, equal groups >= 14 long
     (Shape(1, 2, 12, 12, 32, 3, 1, "f16", 604), "fwd_sync_kernel/full_tma"),
     (Shape(1, 2, 6, 6, 32, 3, 2, "bf16", 605), "fwd_sync_kernel/dense_tma"),    # k <= 5, every group exactly k
