@@ -249,10 +249,12 @@ NA2D_API int na2d_version(void);
 NA2D_API const char *na2d_last_kernel(void);
 
 /* Test hook for the error path of the bounded waits.  The streaming kernel
- * (the k = 7 sliding-window forward) waits for its copies with a limit; when
- * a wait runs out the kernel counts the event (see na2d_device_faults), stops
- * issuing and computing, waits for its copies already in flight (always with
- * the full limit, so nothing lands in released shared memory), and returns;
+ * (the k = 7 sliding-window forward) and the tcgen05 kernel for dilation
+ * groups of up to 16 x 16 pixels with k >= 9 wait for their copies and
+ * products with a limit; when a wait runs out the kernel counts the event
+ * (see na2d_device_faults), stops issuing and computing, waits for its copies
+ * and products already in flight (always with the full limit, so nothing
+ * lands in released memory), and returns;
  * the outputs of that call are then unspecified.  This call shortens the
  * data waits' limit to sm_clocks for the calls that follow on any thread
  * (0 restores the default, about 2^31 clocks).  A limit of a few hundred

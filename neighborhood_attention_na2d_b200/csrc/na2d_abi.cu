@@ -167,6 +167,8 @@ na2d_status na2d_forward(const na2d_problem *p, const void *q, const void *k, co
         bool launched = false;
         cudaError_t e = na2d::launch_forward_umma(pr, q, k, v, rpb, out, st, &launched);
         if (e != cudaSuccess || launched) return from_cuda(e);
+        e = na2d::launch_forward_ugrp(pr, q, k, v, rpb, out, st, &launched);
+        if (e != cudaSuccess || launched) return from_cuda(e);
         e = na2d::launch_forward_stream(pr, View::contiguous(q, pr), View::contiguous(k, pr), View::contiguous(v, pr),
                                         rpb, View::contiguous(out, pr), st, &launched);
         if (e != cudaSuccess || launched) return from_cuda(e);
@@ -396,12 +398,13 @@ na2d_status na2d_backward_noalloc(const na2d_problem *p, const void *q, const vo
 
 na2d_status na2d_device_faults(unsigned int *count, void *stream) {
     if (!count) return NA2D_ERR_NULL;
-    unsigned int a = 0, b = 0, c = 0;
+    unsigned int a = 0, b = 0, c = 0, g = 0;
     cudaError_t e = na2d::read_device_faults(&a, static_cast<cudaStream_t>(stream));
     if (e == cudaSuccess) e = na2d::read_stream_faults(&b, static_cast<cudaStream_t>(stream));
     if (e == cudaSuccess) e = na2d::read_umma_faults(&c, static_cast<cudaStream_t>(stream));
+    if (e == cudaSuccess) e = na2d::read_ugrp_faults(&g, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return from_cuda(e);
-    *count = a + b + c;
+    *count = a + b + c + g;
     return NA2D_OK;
 }
 
@@ -425,6 +428,9 @@ int na2d_version(void) { return 200; }
 
 const char *na2d_last_kernel(void) { return t_last_kernel; }
 
-void na2d_debug_set_wait_limit(long long sm_clocks) { na2d::set_stream_wait_limit(sm_clocks); }
+void na2d_debug_set_wait_limit(long long sm_clocks) {
+    na2d::set_stream_wait_limit(sm_clocks);
+    na2d::set_ugrp_wait_limit(sm_clocks);
+}
 
 }  // extern "C"

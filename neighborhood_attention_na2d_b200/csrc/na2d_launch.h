@@ -101,8 +101,21 @@ cudaError_t launch_forward_umma(const Problem &p, const void *q, const void *k, 
 // As read_device_faults, for the tcgen05 kernel's counter.
 cudaError_t read_umma_faults(unsigned int *count, cudaStream_t stream);
 
+// Forward on the tcgen05 tensor cores for maps whose dilation groups are
+// between k and 16 pixels on each side with k >= 9 (H and W multiples of d,
+// D = 32, f16 / bf16).  Sets *launched when it took the problem.
+bool ugrp_supported(const Problem &p);
+cudaError_t launch_forward_ugrp(const Problem &p, const void *q, const void *k, const void *v,
+                                const void *rpb, void *out, cudaStream_t stream, bool *launched);
+// Test hook: the kernel's data waits give up after `clocks` SM clocks (0: the
+// default, about a second).
+void set_ugrp_wait_limit(long long clocks);
+// As read_device_faults, for this kernel's counter.
+cudaError_t read_ugrp_faults(unsigned int *count, cudaStream_t stream);
+
 // Streaming tensor-core forward for k = 7 (f16 / bf16, D = 32): d = 1 maps with
-// 14 <= W <= 64 and H >= 8, or H = W = 7d (every dilation group 7 x 7).  Sets
+// W >= 14 and H >= 8 (maps wider than 64 columns in column bands), or
+// H = W = 7d (every dilation group 7 x 7).  Sets
 // *launched when it took the problem; otherwise the caller uses
 // launch_forward_tc.
 bool stream_supported(const Problem &p);

@@ -1,0 +1,534 @@
+// na2d_ugrp.cu -- NA2D forward on the 5th-generation tensor cores (tcgen05)
+// for maps whose dilation groups are between k and 16 pixels on each side,
+// with k >= 9 (f16 / bf16, D = 32): for instance the segmentation-scale
+// k = 13, d = 8 layer on a 128 x 128 map, whose groups are 16 x 16.
+//
+// What it computes is the same as the other forward kernels ("Dilated
+// Neighborhood Attention Transformer", gitcode DiNAT article, section
+// "DiNAT 的核心思想": natten2dqkrpb -> softmax -> natten2dav, fused, NATTEN
+// clamp rule).  In a group at most 16 long the windows of 8 consecutive query
+// rows together cover at most k + 1 key rows when k >= 13, and at most 12
+// and 13 rows for k = 9 and 11 (the clamp keeps the window starts of
+// neighbouring rows together), so 8 x 16 queries against a key tile of NKR
+// group rows (NKR <= 14) form a dense contraction whose scores are mostly
+// used (169 of 224 at k = 13): it is one M = 128 tcgen05 tile.
+//
+// Work unit: one dilation group.  Its Q, K and V arrive by TMA as a 16 x 16
+// box of pixels (columns past the group's width zero-filled, rows past its
+// height whatever finite values follow), 64 bytes per pixel, 64-byte
+// swizzled: slot 16 * row + col is tile row 16 * row + col.  Strip e (group
+// rows 8e .. 8e + 7) is the M = 128 tile of Q rows 128e .. 128e + 127; its
+// keys are the group rows kr0[e] .. kr0[e] + NKR - 1 (tile rows from
+// 16 kr0[e]).
+//   1. S_e = Q_e K_e^T: two tcgen05.mma (K = 16 each, both operands K-major
+//      in shared memory), N = 16 NKR, fp32 in tensor memory (TMEM).
+//   2. softmax: one thread per query (its TMEM lane).  Scores are scaled and
+//      biased from a shared-memory table that holds, per query column and
+//      relative key row, the 16 bias values of a key row in log2 units with
+//      the window mask folded in (-1e30 outside the window).  Pass 1 writes
+//      the biased scores back and takes their maximum; pass 2 exponentiates
+//      and writes P as 16-bit pairs over the first 8 NKR columns of S_e.  Key
+//      rows in no window of the warp's queries are skipped (P = 0).
+//   3. O_e = P_e V_e: NKR tcgen05.mma (K = 16 keys = one key row each, A = P
+//      in TMEM, B = V MN-major in shared memory).
+//   4. epilogue: the same thread loads its O row, divides by its row sum and
+//      stores 64 bytes.
+// Warpgroup e (warps 4e .. 4e + 3) runs strip e of every unit, with S_e at
+// TMEM columns e N and O_e at 2N + 32e.  Warp 8, lane 0 issues the TMA copies
+// into a ring of NSTG stages; warps 9 and 10, lane 0, issue the MMAs of strip
+// 0 and strip 1 (each unit's P.V, then the next unit's Q K^T) and signal
+// completion with tcgen05.commit on mbarriers; warp 9 owns the TMEM
+// allocation.  Every wait is bounded: one that runs out counts the event,
+// raises the block's abort flag, and the block winds down (its MMAs and
+// copies in flight are waited for before TMEM and shared memory are
+// released).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <map>
+#include <mutex>
+#include <set>
+#include <type_traits>
+
+#include "na2d_device.cuh"
+#include "na2d_launch.h"
+#include "na2d_tcgen05.cuh"
+
+namespace na2d {
+namespace {
+
+constexpr int NSTG = 3;                    // shared-memory stages (units in flight)
+constexpr uint32_t kGroupBytes = 16384;    // one tensor of a unit: 16 x 16 pixels of 64 bytes
+constexpr uint32_t kStage = 3 * kGroupBytes;
+constexpr int kMaxNKR = 14;                // two S buffers of 16 NKR columns and two O buffers fit in TMEM
+constexpr int kThreads = 352;              // 8 softmax warps, producer warp, two MMA warps
+constexpr int kWarpTma = 8, kWarpMma = 9;  // MMA warps 9 (strip 0) and 10 (strip 1)
+constexpr float kMasked = -1.0e30f;        // bias outside the window: exp2 gives 0
+
+__device__ unsigned int g_ugrp_timeouts;
+
+struct UgrpParams {
+    CUtensorMap tq, tk, tv;   // 5-D group views, 32 x 1 x 16 x 1 x 16 boxes
+    unsigned char *out;
+    const void *rpb;
+    int H, W, heads, d, k;
+    int Lgy, Lgx;             // group height and width
+    int GU;                   // units (groups): B * heads * d * d
+    int NKR;                  // key rows of a strip's tile
+    int kr0[2];               // first group row of strip 0 / 1's key tile
+    float c_log2;             // log2(e) / sqrt(D)
+    long long wait_limit;     // SM clocks a data wait may take
+    uint32_t qstride;         // bytes per query column of a bias table
+    uint32_t tab_bytes;       // bytes per bias table (16 query columns)
+    uint32_t off_tab, off_bar;   // byte offsets from the 1024-aligned base
+};
+
+// Stores 8 consecutive 32-bit columns of this thread's lane.
+__device__ __forceinline__ void tmem_st8(uint32_t ta, const uint32_t *v) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};\n" ::"r"(ta), "r"(v[0]),
+                 "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+                 : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Kernel.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(kThreads, 1) fwd_ugrp_kernel(const __grid_constant__ UgrpParams p) {
+    extern __shared__ unsigned char smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t sbase = (raw + 1023u) & ~1023u;   // swizzled tiles need 1024-byte alignment
+    unsigned char *smem = smem_raw + (sbase - raw);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int u_begin = (int)((int64_t)p.GU * blockIdx.x / gridDim.x);
+    const int u_end = (int)((int64_t)p.GU * (blockIdx.x + 1) / gridDim.x);
+    grid_dep_launch();
+    if (u_begin >= u_end) return;
+    const int nst = u_end - u_begin;
+    const int dd = p.d * p.d;
+    // the block's units lie in at most two (batch, head) planes (the launch
+    // sizes the ranges so), each with its own bias table
+    const int bh_first = u_begin / dd;
+    if ((u_end - 1) / dd - bh_first > 1) {   // never, by the launch; counted rather than overrun the tables
+        if (threadIdx.x == 0) atomicAdd(&g_ugrp_timeouts, 1u);
+        return;
+    }
+    const int NKR = p.NKR, N = 16 * NKR;
+
+    const uint32_t bar_full = sbase + p.off_bar;        // [NSTG] stage landed (TMA bytes)
+    const uint32_t bar_empty = bar_full + 8 * NSTG;     // [NSTG] stage consumed (two commits)
+    const uint32_t bar_s = bar_empty + 8 * NSTG;        // [2] S_e ready (commit)
+    const uint32_t bar_p = bar_s + 16;                  // [2] P_e written (4 warps)
+    const uint32_t bar_o = bar_p + 16;                  // [2] O_e ready (commit)
+    const uint32_t bar_drain = bar_o + 16;              // [2] all MMAs of an MMA warp done (commit)
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + p.off_bar + 16 * NSTG + 64);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + p.off_bar + 16 * NSTG + 68);
+
+    auto issue_unit = [&](int j) {
+        const uint32_t fb = bar_full + 8 * (j % NSTG);
+        const uint32_t st = sbase + (uint32_t)(j % NSTG) * kStage;
+        mb_expect_tx(fb, kStage);
+        const int g = u_begin + j;
+        const int bh = g / dd, rem = g - bh * dd, gy = rem / p.d, gx = rem - gy * p.d;
+        const int row = bh * p.Lgy;   // merged (plane, group row) coordinate of group row 0
+        tma_load_5d(st, &p.tq, fb, gx, 0, gy, row);
+        tma_load_5d(st + kGroupBytes, &p.tk, fb, gx, 0, gy, row);
+        tma_load_5d(st + 2 * kGroupBytes, &p.tv, fb, gx, 0, gy, row);
+    };
+    const int n_first = min(2, nst);
+
+    // ---- prologue.  The producer thread initialises the barriers and starts
+    // the first units' copies; meanwhile the other threads build the bias
+    // tables and allocate TMEM.
+    {
+        if (warp == kWarpTma && lane == 0) {
+            for (int i = 0; i < NSTG; ++i) {
+                mb_init(bar_full + 8 * i, 1);
+                mb_init(bar_empty + 8 * i, 2);
+            }
+            for (int i = 0; i < 2; ++i) {
+                mb_init(bar_s + 8 * i, 1);
+                mb_init(bar_p + 8 * i, 4);
+                mb_init(bar_o + 8 * i, 1);
+                mb_init(bar_drain + 8 * i, 1);
+            }
+            *abort_flag = 0;
+            asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+            grid_dep_wait();   // before the first copy
+            for (int j = 0; j < n_first; ++j) issue_unit(j);
+        }
+        grid_dep_wait();   // before the bias tables' reads
+        // table t (plane bh_first + t), query column qc, row a, key column j:
+        // a < 2k - 1 is the relative key row a - (k - 1); a = 2k - 1 is an
+        // all-masked row.  Entry: rpb[h, a, j - qc + k - 1] * log2(e) when key
+        // column j is in the window of query column qc, else kMasked.  Query
+        // columns past the group's width take the last column's window and
+        // bias (their outputs are not stored).
+        const int k = p.k, nrel = 2 * k - 1;
+        const int nplanes = (u_end - 1) / dd - bh_first + 1;
+        const T *rpb = reinterpret_cast<const T *>(p.rpb);
+        const int per_tab = 16 * 2 * k * 16;
+        for (int i = threadIdx.x; i < nplanes * per_tab; i += kThreads) {
+            const int t = i / per_tab, r = i - t * per_tab;
+            const int qc = r / (2 * k * 16), a = (r / 16) % (2 * k), j = r & 15;
+            const int qcc = min(qc, p.Lgx - 1);
+            const int wx = window_start(qcc, p.Lgx, k);
+            float v = kMasked;
+            if (a < nrel && (unsigned)(j - wx) < (unsigned)k) {
+                const int h = (int)((bh_first + t) % p.heads);
+                v = rpb ? Elem<T>::to_f(rpb[((int64_t)h * nrel + a) * nrel + (j - qcc + k - 1)]) * kLog2e : 0.f;
+            }
+            *reinterpret_cast<float *>(smem + p.off_tab + (uint32_t)t * p.tab_bytes + (uint32_t)qc * p.qstride +
+                                       (uint32_t)(a * 16 + j) * 4u) = v;
+        }
+        if (warp == kWarpMma) tmem_alloc(smem_u32(tmem_slot));
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    }
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == kWarpTma) {
+        // =================== TMA producer ===================
+        if (lane == 0) {
+            int issued = n_first;
+            for (int j = n_first; j < nst; ++j) {
+                const int s = j % NSTG;
+                if (j >= NSTG && !mb_wait(bar_empty + 8 * s, (uint32_t)(((j / NSTG) - 1) & 1), p.wait_limit)) {
+                    atomicAdd(&g_ugrp_timeouts, 1u);
+                    *abort_flag = 1;
+                    break;
+                }
+                if (*abort_flag) break;
+                issue_unit(j);
+                ++issued;
+            }
+            // copies still in flight land before shared memory is released
+            for (int j = max(0, issued - NSTG); j < issued; ++j)
+                mb_wait(bar_full + 8 * (j % NSTG), (uint32_t)((j / NSTG) & 1));
+        }
+    } else if (warp == kWarpMma || warp == kWarpMma + 1) {
+        // =================== MMA issuers ===================
+        // Warp kWarpMma + e issues strip e of every unit: S_0, then per unit
+        // j: O_j = P_j V_j, S_{j+1} = Q K^T.  S_{j+1} reuses the columns of
+        // P_j after the P.V that reads them (tcgen05.mma of one thread
+        // execute in issue order); O_j is free again once the warpgroup's
+        // epilogue of unit j - 1, which precedes its P_j, has read it.
+        const int e = warp - kWarpMma;
+        if (lane == 0) {
+            const uint32_t idesc_qk = idesc_f16<T>(N, 0);
+            constexpr uint32_t idesc_pv = idesc_f16<T>(32, 1);
+            const uint32_t koff = (uint32_t)p.kr0[e] * 1024u;   // 16 pixels of 64 bytes per group row
+            const uint32_t dS = tmem + (uint32_t)(e * N), dO = tmem + (uint32_t)(2 * N + 32 * e);
+            auto issue_qk = [&](int j) -> bool {
+                const int s = j % NSTG;
+                if (!mb_wait(bar_full + 8 * s, (uint32_t)((j / NSTG) & 1), p.wait_limit) || *abort_flag) return false;
+                tc_fence_after();
+                const uint32_t st = sbase + (uint32_t)s * kStage;
+                // K-major, 64-byte rows: 8-row groups 512 bytes apart; the
+                // second K = 16 step starts 32 bytes into the rows
+                const uint64_t da = sw64_desc(st + (uint32_t)e * 8192u, 16, 512);
+                const uint64_t db = sw64_desc(st + kGroupBytes + koff, 16, 512);
+                umma_ss(dS, da, db, idesc_qk, 0);
+                umma_ss(dS, da + 2, db + 2, idesc_qk, 1);
+                umma_commit(bar_s + 8 * e);
+                return true;
+            };
+            bool ok = issue_qk(0);
+            for (int j = 0; ok && j < nst; ++j) {
+                const int s = j % NSTG;
+                if (!mb_wait(bar_p + 8 * e, (uint32_t)(j & 1), p.wait_limit) || *abort_flag) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t vt = sbase + (uint32_t)s * kStage + 2 * kGroupBytes + koff;
+                // V MN-major: 64-byte rows of 32 channels, 8-key groups 512
+                // bytes apart; k-step t takes key row t (16 keys)
+                for (int t = 0; t < NKR; ++t)
+                    umma_ts(dO, dS + 8u * (uint32_t)t, sw64_desc(vt + 1024u * (uint32_t)t, 16, 512), idesc_pv,
+                            t > 0 ? 1u : 0u);
+                umma_commit(bar_o + 8 * e);
+                umma_commit(bar_empty + 8 * s);
+                if (j + 1 < nst && !issue_qk(j + 1)) ok = false;
+            }
+            if (!ok) {
+                atomicAdd(&g_ugrp_timeouts, 1u);
+                *abort_flag = 1;
+            }
+            // every MMA this thread issued has completed before TMEM is released
+            umma_commit(bar_drain + 8 * e);
+            mb_wait(bar_drain + 8 * e, 0);
+        }
+    } else {
+        // =================== softmax warpgroups ===================
+        const int e = warp >> 2;                      // strip of this warpgroup
+        const int q4 = warp & 3;                      // lane quarter of this warp
+        const int m = q4 * 32 + lane;                 // tile row = TMEM lane
+        const int qr = m >> 4, qc = m & 15;           // query slot within the strip
+        const int row = 8 * e + qr;                   // group row
+        const bool qok = row < p.Lgy && qc < p.Lgx;
+        const int rowc = min(row, p.Lgy - 1);
+        const int k = p.k;
+        // key-tile rows wy .. wy + k - 1 are this query's window rows
+        const int wy = window_start(rowc, p.Lgy, k) - p.kr0[e];
+        const uint32_t vrows = ((1u << k) - 1u) << wy;
+        const uint32_t wrows = __reduce_or_sync(0xffffffffu, vrows);   // rows some query of the warp needs
+        // table row of key-tile row i: a0 + i (relative row + k - 1) when valid
+        const int a0 = p.kr0[e] - rowc + k - 1;
+        const uint32_t tl = tmem + ((uint32_t)(32 * q4) << 16);
+        const uint32_t tS = tl + (uint32_t)(e * N), tO = tl + (uint32_t)(2 * N + 32 * e);
+        const float c = p.c_log2;
+        const unsigned char *tab_q = smem + p.off_tab + (uint32_t)qc * p.qstride;
+        const int nrel = 2 * k - 1;
+
+        for (int j = 0; j < nst; ++j) {
+            const int g = u_begin + j;
+            const int bh = g / dd;
+            const float4 *tq = reinterpret_cast<const float4 *>(tab_q + (uint32_t)(bh - bh_first) * p.tab_bytes);
+            const bool ok = mb_wait(bar_s + 8 * e, (uint32_t)(j & 1), p.wait_limit);
+            if (!__all_sync(0xffffffffu, ok) || __any_sync(0xffffffffu, *abort_flag != 0)) {
+                if (lane == 0) {
+                    atomicAdd(&g_ugrp_timeouts, 1u);
+                    *abort_flag = 1;
+                }
+                break;
+            }
+            tc_fence_after();
+            // ---- pass 1: biased scores (log2 units) back into S, and their maximum
+            float mx = -3.0e38f;
+            for (int i = 0; i < NKR; ++i) {
+                if (!((wrows >> i) & 1u)) continue;
+                float s[16];
+                tmem_ld16(tS + 16u * (uint32_t)i, s);
+                const bool inwin = (unsigned)(i - wy) < (unsigned)k;
+                const float4 *br = tq + (inwin ? (a0 + i) : nrel) * 4;
+                const float4 b0 = br[0], b1 = br[1], b2 = br[2], b3 = br[3];
+                tmem_ld_wait();
+                s[0] = fmaf(s[0], c, b0.x);   s[1] = fmaf(s[1], c, b0.y);
+                s[2] = fmaf(s[2], c, b0.z);   s[3] = fmaf(s[3], c, b0.w);
+                s[4] = fmaf(s[4], c, b1.x);   s[5] = fmaf(s[5], c, b1.y);
+                s[6] = fmaf(s[6], c, b1.z);   s[7] = fmaf(s[7], c, b1.w);
+                s[8] = fmaf(s[8], c, b2.x);   s[9] = fmaf(s[9], c, b2.y);
+                s[10] = fmaf(s[10], c, b2.z); s[11] = fmaf(s[11], c, b2.w);
+                s[12] = fmaf(s[12], c, b3.x); s[13] = fmaf(s[13], c, b3.y);
+                s[14] = fmaf(s[14], c, b3.z); s[15] = fmaf(s[15], c, b3.w);
+                mx = max3(mx, max3(s[0], s[1], s[2]), max3(s[3], s[4], s[5]));
+                mx = max3(mx, max3(s[6], s[7], s[8]), max3(s[9], s[10], s[11]));
+                mx = max3(mx, max3(s[12], s[13], s[14]), s[15]);
+                uint32_t sb[16];
+#pragma unroll
+                for (int t = 0; t < 16; ++t) sb[t] = __float_as_uint(s[t]);
+                tmem_st16(tS + 16u * (uint32_t)i, sb);
+            }
+            tmem_st_wait();
+            // ---- pass 2: P = exp2(score - max) as 16-bit pairs over the first
+            // 8 NKR columns (key row i at columns 8i .. 8i + 7, whose scores
+            // were read at row i / 2 <= i); rows outside every window: zeros
+            float l0 = 0.f, l1 = 0.f;
+            for (int i = 0; i < NKR; ++i) {
+                uint32_t pk[8];
+                if ((wrows >> i) & 1u) {
+                    float s[16];
+                    tmem_ld16(tS + 16u * (uint32_t)i, s);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int t = 0; t < 8; ++t) {
+                        const float p0 = ex2(s[2 * t] - mx), p1 = ex2(s[2 * t + 1] - mx);
+                        if (t & 1) l1 += p0 + p1; else l0 += p0 + p1;
+                        pk[t] = Pack2<T>::run(p0, p1);
+                    }
+                } else {
+#pragma unroll
+                    for (int t = 0; t < 8; ++t) pk[t] = 0u;
+                }
+                tmem_st8(tS + 8u * (uint32_t)i, pk);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mb_arrive(bar_p + 8 * e);
+            // ---- epilogue: O / row sum -> 64 bytes
+            const bool oko = mb_wait(bar_o + 8 * e, (uint32_t)(j & 1), p.wait_limit);
+            if (!__all_sync(0xffffffffu, oko)) {
+                if (lane == 0) {
+                    atomicAdd(&g_ugrp_timeouts, 1u);
+                    *abort_flag = 1;
+                }
+                break;
+            }
+            tc_fence_after();
+            float o[32];
+            tmem_ld32(tO, o);
+            tmem_ld_wait();
+            if (qok) {
+                float inv;
+                asm("rcp.approx.ftz.f32 %0, %1;\n" : "=f"(inv) : "f"(l0 + l1));
+                const int rem = g - bh * dd, gy = rem / p.d, gx = rem - gy * p.d;
+                uint4 *dst = reinterpret_cast<uint4 *>(
+                    p.out + ((((size_t)bh * p.H + gy + (size_t)p.d * row) * p.W) + gx + (size_t)p.d * qc) * 64);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    dst[i] = make_uint4(Pack2<T>::run(o[8 * i + 0] * inv, o[8 * i + 1] * inv),
+                                        Pack2<T>::run(o[8 * i + 2] * inv, o[8 * i + 3] * inv),
+                                        Pack2<T>::run(o[8 * i + 4] * inv, o[8 * i + 5] * inv),
+                                        Pack2<T>::run(o[8 * i + 6] * inv, o[8 * i + 7] * inv));
+            }
+        }
+    }
+    // ---- teardown: TMEM released by the warp that took it, after every
+    // thread is done with it
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kWarpMma) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Host side.
+// ---------------------------------------------------------------------------
+struct UgrpCache {
+    std::mutex mu;
+    std::map<int, std::pair<int, int>> dev;   // device -> (SMs, opt-in smem per block)
+    std::set<std::pair<int, const void *>> attr;
+};
+UgrpCache &gcache() {
+    static UgrpCache c;
+    return c;
+}
+
+cudaError_t ugrp_device(int *sms, int *smem_cap, const void *kern) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    UgrpCache &c = gcache();
+    std::lock_guard<std::mutex> lock(c.mu);
+    auto it = c.dev.find(dev);
+    if (it == c.dev.end()) {
+        int n = 0, m = 0;
+        if ((e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+        if ((e = cudaDeviceGetAttribute(&m, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) return e;
+        it = c.dev.emplace(dev, std::make_pair(n, m)).first;
+    }
+    *sms = it->second.first;
+    *smem_cap = it->second.second;
+    if (!c.attr.count({dev, kern})) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, *smem_cap);
+        if (e != cudaSuccess) return e;
+        c.attr.insert({dev, kern});
+    }
+    return cudaSuccess;
+}
+
+std::atomic<long long> &ugrp_limit_store() {
+    static std::atomic<long long> v{0};
+    return v;
+}
+
+// Key tile of each strip: NKR group rows covering the windows of the strip's
+// query rows (8e .. min(8e + 7, Lg - 1)), starting at kr0[e] and inside the
+// group.
+int strip_key_rows(int Lg, int k, int kr0[2]) {
+    int nkr = 0;
+    int first[2];
+    for (int e = 0; e < 2; ++e) {
+        const int r0 = 8 * e, r1 = std::min(8 * e + 7, Lg - 1);
+        first[e] = window_start(r0, Lg, k);
+        nkr = std::max(nkr, window_start(r1, Lg, k) - first[e] + k);
+    }
+    for (int e = 0; e < 2; ++e) kr0[e] = std::min(first[e], Lg - nkr);
+    return nkr;
+}
+
+template <typename T>
+cudaError_t launch_ugrp_t(const Problem &pr, const void *q, const void *k, const void *v, const void *rpb, void *out,
+                          cudaStream_t st, bool *launched) {
+    const void *kern = reinterpret_cast<const void *>(&fwd_ugrp_kernel<T>);
+    int sms = 0, cap = 0;
+    cudaError_t e = ugrp_device(&sms, &cap, kern);
+    if (e != cudaSuccess) return e;
+    UgrpParams up{};
+    const int64_t bh = pr.bh();
+    const int dd = pr.d * pr.d;
+    const int64_t gu = bh * dd;
+    up.Lgy = pr.H / pr.d;
+    up.Lgx = pr.W / pr.d;
+    if (gu <= 0 || gu >= INT32_MAX || bh * up.Lgy >= INT32_MAX) return cudaSuccess;
+    up.NKR = strip_key_rows(up.Lgy, pr.k, up.kr0);
+    if (up.NKR > kMaxNKR) return cudaSuccess;
+    if (!encode_group_map(&up.tq, q, pr.dtype, bh, pr.H, pr.W, pr.d, 16, 16, 1) ||
+        !encode_group_map(&up.tk, k, pr.dtype, bh, pr.H, pr.W, pr.d, 16, 16, 1) ||
+        !encode_group_map(&up.tv, v, pr.dtype, bh, pr.H, pr.W, pr.d, 16, 16, 1))
+        return cudaSuccess;
+    up.out = static_cast<unsigned char *>(out);
+    up.rpb = rpb;
+    up.H = pr.H; up.W = pr.W; up.heads = pr.heads; up.d = pr.d; up.k = pr.k;
+    up.GU = (int)gu;
+    up.c_log2 = kLog2e / std::sqrt((float)pr.D);
+    const long long lim = ugrp_limit_store().load();
+    up.wait_limit = lim > 0 ? lim : (1LL << 31);
+    // bias table: per query column 2k rows of 16 floats, plus 16 bytes so
+    // that the 8 query columns a quarter-warp reads lie in different banks
+    up.qstride = (uint32_t)(2 * pr.k * 64 + 16);
+    up.tab_bytes = 16 * up.qstride;
+    up.off_tab = NSTG * kStage;
+    up.off_bar = up.off_tab + 2 * up.tab_bytes;
+    const uint32_t smem = up.off_bar + 16 * NSTG + 72 + 1024;   // + 1024 bytes for aligning the base
+    if ((int)smem > cap) return cudaSuccess;
+    // units per block at most d^2 + 1, so that a block's units lie in at
+    // most two (batch, head) planes
+    const int64_t grid = std::max<int64_t>(std::min<int64_t>(gu, sms), (gu + dd) / (dd + 1));
+    if (grid >= INT32_MAX) return cudaSuccess;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t el = cudaLaunchKernelEx(&cfg, fwd_ugrp_kernel<T>, up);
+    *launched = true;
+    note_kernel("fwd_ugrp_kernel");
+    return el != cudaSuccess ? el : cudaGetLastError();
+}
+
+}  // namespace
+
+bool ugrp_supported(const Problem &p) {
+    if (p.dtype != DType::F16 && p.dtype != DType::BF16) return false;
+    if (p.D != 32 || p.k < 9 || p.k > 13 || !(p.k & 1) || p.d < 1 || p.heads > 4096) return false;
+    if (p.H % p.d || p.W % p.d) return false;
+    const int Lgy = p.H / p.d, Lgx = p.W / p.d;
+    return Lgy >= p.k && Lgy <= 16 && Lgx >= p.k && Lgx <= 16;
+}
+
+cudaError_t launch_forward_ugrp(const Problem &p, const void *q, const void *k, const void *v, const void *rpb,
+                                void *out, cudaStream_t st, bool *launched) {
+    *launched = false;
+    if (!ugrp_supported(p)) return cudaSuccess;
+    if (p.dtype == DType::F16) return launch_ugrp_t<__half>(p, q, k, v, rpb, out, st, launched);
+    return launch_ugrp_t<__nv_bfloat16>(p, q, k, v, rpb, out, st, launched);
+}
+
+void set_ugrp_wait_limit(long long clocks) { ugrp_limit_store().store(clocks); }
+
+cudaError_t read_ugrp_faults(unsigned int *count, cudaStream_t st) {
+    unsigned int zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbolAsync(count, g_ugrp_timeouts, sizeof(unsigned int), 0,
+                                              cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess)
+        e = cudaMemcpyToSymbolAsync(g_ugrp_timeouts, &zero, sizeof(unsigned int), 0, cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    return e;
+}
+
+}  // namespace na2d

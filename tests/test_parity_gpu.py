@@ -141,6 +141,40 @@ def test_stream_shapes(shape, with_rpb):
     assert err <= TOL[shape.dtype], f"{shape.describe()} rpb={with_rpb}: max abs err {err}"
 
 
+def _ugrp_cases():
+    """Shapes of the tcgen05 kernel for dilation groups of k .. 16 pixels a
+    side with k >= 9: every key-tile height (NKR 9 .. 14), square and
+    non-square groups, widths below 16 (zero-filled columns), heights below 16
+    (a short second strip), ranges of units that span two (batch, head)
+    planes, and blocks with more units than ring stages."""
+    rows = [
+        (1, 1, 9, 9, 9, 1, "f16", True),        # NKR 9, one group
+        (1, 2, 10, 12, 9, 1, "bf16", True),     # NKR 10 / 12 strips
+        (2, 1, 33, 36, 9, 3, "f16", False),     # 11 x 12 groups
+        (1, 3, 16, 16, 9, 1, "bf16", True),     # NKR 12
+        (2, 2, 14, 11, 11, 1, "bf16", True),    # 14 x 11 groups, NKR 13
+        (1, 2, 24, 22, 11, 2, "f16", True),     # 12 x 11 groups
+        (1, 2, 13, 16, 13, 1, "f16", True),     # NKR 13
+        (2, 3, 42, 39, 13, 3, "bf16", True),    # 14 x 13 groups, NKR 14
+        (1, 2, 32, 32, 13, 2, "f16", False),    # 16 x 16 groups
+        (2, 4, 64, 64, 13, 4, "bf16", True),    # 16 x 16 groups, 3 - 4 units per block
+        (8, 8, 64, 64, 9, 4, "f16", True),      # about 7 units per block: the ring wraps twice
+        (30, 10, 16, 16, 13, 1, "bf16", True),  # 300 planes of one group: blocks span two planes
+        (20, 10, 24, 24, 11, 2, "f16", True),   # 800 units, 5 per block across plane boundaries
+    ]
+    return [(Shape(B, h, H, W, 32, k, d, dt, 7300 + i), rpb) for i, (B, h, H, W, k, d, dt, rpb) in enumerate(rows)]
+
+
+@pytest.mark.parametrize("shape,with_rpb", _ugrp_cases(), ids=lambda x: x.describe() if isinstance(x, Shape) else str(x))
+def test_ugrp_shapes(shape, with_rpb):
+    """The tcgen05 kernel for groups of k .. 16 pixels, every output element."""
+    (q, k, v, rpb), got = run_forward(shape, with_rpb)
+    assert na.na2d_last_kernel() == "fwd_ugrp_kernel"
+    want = oracle.forward(f64(q), f64(k), f64(v), f64(rpb), shape.k, shape.d)
+    err = max_err(got, want)
+    assert err <= TOL[shape.dtype], f"{shape.describe()} rpb={with_rpb}: max abs err {err}"
+
+
 @pytest.mark.parametrize("k,d,L", [(3, 1, 3), (7, 1, 7), (13, 1, 13), (7, 2, 14), (13, 2, 26), (5, 8, 40), (13, 9, 117)])
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
 def test_window_covers_group(k, d, L, dtype):
@@ -242,7 +276,8 @@ DISPATCH = [
     (Shape(1, 2, 12, 12, 32, 3, 1, "f16", 604), "fwd_sync_kernel/full_tma"),
     (Shape(1, 2, 6, 6, 32, 3, 2, "bf16", 605), "fwd_sync_kernel/dense_tma"),    # k <= 5, every group exactly k
     (Shape(1, 2, 30, 30, 32, 9, 1, "f16", 606), "fwd_tc_kernel/full"),          # k >= 9, long groups
-    (Shape(1, 2, 13, 13, 32, 13, 1, "bf16", 607), "fwd_tc_kernel/dense"),       # k >= 9, every group exactly k
+    (Shape(1, 2, 13, 13, 32, 13, 1, "bf16", 607), "fwd_ugrp_kernel"),           # k >= 9, groups k .. 16 long
+    (Shape(1, 2, 32, 32, 32, 13, 2, "f16", 614), "fwd_ugrp_kernel"),
     (Shape(1, 2, 20, 18, 32, 7, 2, "bf16", 608), "fwd_tc_kernel/generic"),      # short groups
     (Shape(1, 2, 23, 19, 32, 5, 2, "f16", 609), "fwd_tc_kernel/full"),          # ragged groups (H, W not multiples of d)
     (Shape(1, 2, 15, 17, 32, 5, 2, "bf16", 612), "fwd_tc_kernel/generic"),      # ragged short groups
@@ -329,6 +364,32 @@ def test_bounded_wait_error_path_runs_out_and_recovers():
     assert na.na2d_device_faults() == 0
     want = oracle.forward(f64(q), f64(k), f64(v), f64(rpb), 7, 1)
     assert max_err(out.double().cpu().numpy(), want) <= TOL["f16"]
+
+
+def test_bounded_wait_error_path_tcgen05_groups():
+    """The same error path in the tcgen05 kernel for groups of up to 16 x 16
+    pixels: with the wait limit cut to 200 SM clocks the MMA warps' wait for
+    the first 48 KB copy and the softmax warps' wait for the first scores run
+    out; the kernel counts the event, waits for its copies and products in
+    flight, releases its tensor memory and returns.  With the default limit
+    restored the next call is correct and counts nothing."""
+    from neighborhood_attention_na2d_b200 import _native
+    shape = Shape(2, 4, 128, 128, 32, 13, 8, "bf16", 1702)
+    q, k, v, rpb = make_inputs(shape)
+    qd, kd, vd, rd = (t.cuda() for t in (q, k, v, rpb))
+    assert na.na2d_device_faults() == 0
+    try:
+        _native.lib().na2d_debug_set_wait_limit(200)
+        na.na2d_forward(qd, kd, vd, rd, 13, 8)
+        assert na.na2d_last_kernel() == "fwd_ugrp_kernel"
+        assert na.na2d_device_faults() > 0
+    finally:
+        _native.lib().na2d_debug_set_wait_limit(0)
+    out = na.na2d_forward(qd, kd, vd, rd, 13, 8)
+    torch.cuda.synchronize()
+    assert na.na2d_device_faults() == 0
+    want = oracle.forward(f64(q), f64(k), f64(v), f64(rpb), 13, 8)
+    assert max_err(out.double().cpu().numpy(), want) <= TOL["bf16"]
 
 
 def test_no_device_wait_timed_out():
