@@ -83,7 +83,7 @@ struct UgrpParams {
     long long wait_limit;     // SM clocks a data wait may take
     uint32_t qstride;         // bytes per query column of a bias table
     uint32_t tab_bytes;       // bytes per bias table (16 query columns)
-    uint32_t off_tab, off_bar;   // byte offsets from the 1024-aligned base
+    uint32_t off_tab, off_bar, off_rpb;   // byte offsets from the 1024-aligned base
 };
 
 // Stores 8 consecutive 32-bit columns of this thread's lane.
@@ -93,11 +93,36 @@ __device__ __forceinline__ void tmem_st8(uint32_t ta, const uint32_t *v) {
                  : "memory");
 }
 
+// P as 16-bit pairs and its contribution to the row sum.  bf16: the upper
+// halves of the fp32 values (rounding toward zero, relative error below
+// 2^-8), packed by one byte permute on the integer pipe instead of a
+// conversion on the pipe the exponentials use; the row sum adds exactly the
+// values packed, so the normalisation matches the P of the products.  f16:
+// round-to-nearest conversion, row sum of the fp32 values.
+template <typename T> struct PackP;
+template <> struct PackP<__nv_bfloat16> {
+    __device__ __forceinline__ static uint32_t run(float p0, float p1, float &l) {
+        const uint32_t a = __float_as_uint(p0), b = __float_as_uint(p1);
+        uint32_t r;
+        asm("prmt.b32 %0, %1, %2, 0x7632;\n" : "=r"(r) : "r"(a), "r"(b));
+        l += __uint_as_float(a & 0xffff0000u) + __uint_as_float(b & 0xffff0000u);
+        return r;
+    }
+};
+template <> struct PackP<__half> {
+    __device__ __forceinline__ static uint32_t run(float p0, float p1, float &l) {
+        l += p0 + p1;
+        return Pack2<__half>::run(p0, p1);
+    }
+};
+
 // ---------------------------------------------------------------------------
 // Kernel.
 // ---------------------------------------------------------------------------
-template <typename T>
+template <typename T, int NKR>
 __global__ void __launch_bounds__(kThreads, 1) fwd_ugrp_kernel(const __grid_constant__ UgrpParams p) {
+    static_assert(NKR >= 1 && NKR <= kMaxNKR, "key tile of 1 .. 14 group rows");
+    constexpr int N = 16 * NKR;
     extern __shared__ unsigned char smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t sbase = (raw + 1023u) & ~1023u;   // swizzled tiles need 1024-byte alignment
@@ -116,7 +141,6 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_ugrp_kernel(const __grid_cons
         if (threadIdx.x == 0) atomicAdd(&g_ugrp_timeouts, 1u);
         return;
     }
-    const int NKR = p.NKR, N = 16 * NKR;
 
     const uint32_t bar_full = sbase + p.off_bar;        // [NSTG] stage landed (TMA bytes)
     const uint32_t bar_empty = bar_full + 8 * NSTG;     // [NSTG] stage consumed (two commits)
@@ -167,9 +191,17 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_ugrp_kernel(const __grid_cons
         // column j is in the window of query column qc, else kMasked.  Query
         // columns past the group's width take the last column's window and
         // bias (their outputs are not stored).
-        const int k = p.k, nrel = 2 * k - 1;
+        const int k = p.k, nrel = 2 * k - 1, nr2 = nrel * nrel;
         const int nplanes = (u_end - 1) / dd - bh_first + 1;
+        // the planes' bias rows first, in log2 units (all loads in flight at once)
+        float *rpbs = reinterpret_cast<float *>(smem + p.off_rpb);
         const T *rpb = reinterpret_cast<const T *>(p.rpb);
+        for (int i = threadIdx.x; i < nplanes * nr2; i += kThreads) {
+            const int t = i / nr2, r = i - t * nr2;
+            const int h = (int)((bh_first + t) % p.heads);
+            rpbs[i] = rpb ? Elem<T>::to_f(rpb[(int64_t)h * nr2 + r]) * kLog2e : 0.f;
+        }
+        __syncthreads();
         const int per_tab = 16 * 2 * k * 16;
         for (int i = threadIdx.x; i < nplanes * per_tab; i += kThreads) {
             const int t = i / per_tab, r = i - t * per_tab;
@@ -177,10 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_ugrp_kernel(const __grid_cons
             const int qcc = min(qc, p.Lgx - 1);
             const int wx = window_start(qcc, p.Lgx, k);
             float v = kMasked;
-            if (a < nrel && (unsigned)(j - wx) < (unsigned)k) {
-                const int h = (int)((bh_first + t) % p.heads);
-                v = rpb ? Elem<T>::to_f(rpb[((int64_t)h * nrel + a) * nrel + (j - qcc + k - 1)]) * kLog2e : 0.f;
-            }
+            if (a < nrel && (unsigned)(j - wx) < (unsigned)k) v = rpbs[t * nr2 + a * nrel + (j - qcc + k - 1)];
             *reinterpret_cast<float *>(smem + p.off_tab + (uint32_t)t * p.tab_bytes + (uint32_t)qc * p.qstride +
                                        (uint32_t)(a * 16 + j) * 4u) = v;
         }
@@ -275,8 +304,6 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_ugrp_kernel(const __grid_cons
         const int k = p.k;
         // key-tile rows wy .. wy + k - 1 are this query's window rows
         const int wy = window_start(rowc, p.Lgy, k) - p.kr0[e];
-        const uint32_t vrows = ((1u << k) - 1u) << wy;
-        const uint32_t wrows = __reduce_or_sync(0xffffffffu, vrows);   // rows some query of the warp needs
         // table row of key-tile row i: a0 + i (relative row + k - 1) when valid
         const int a0 = p.kr0[e] - rowc + k - 1;
         const uint32_t tl = tmem + ((uint32_t)(32 * q4) << 16);
@@ -298,55 +325,69 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_ugrp_kernel(const __grid_cons
                 break;
             }
             tc_fence_after();
-            // ---- pass 1: biased scores (log2 units) back into S, and their maximum
-            float mx = -3.0e38f;
-            for (int i = 0; i < NKR; ++i) {
-                if (!((wrows >> i) & 1u)) continue;
-                float s[16];
-                tmem_ld16(tS + 16u * (uint32_t)i, s);
-                const bool inwin = (unsigned)(i - wy) < (unsigned)k;
-                const float4 *br = tq + (inwin ? (a0 + i) : nrel) * 4;
-                const float4 b0 = br[0], b1 = br[1], b2 = br[2], b3 = br[3];
-                tmem_ld_wait();
-                s[0] = fmaf(s[0], c, b0.x);   s[1] = fmaf(s[1], c, b0.y);
-                s[2] = fmaf(s[2], c, b0.z);   s[3] = fmaf(s[3], c, b0.w);
-                s[4] = fmaf(s[4], c, b1.x);   s[5] = fmaf(s[5], c, b1.y);
-                s[6] = fmaf(s[6], c, b1.z);   s[7] = fmaf(s[7], c, b1.w);
-                s[8] = fmaf(s[8], c, b2.x);   s[9] = fmaf(s[9], c, b2.y);
-                s[10] = fmaf(s[10], c, b2.z); s[11] = fmaf(s[11], c, b2.w);
-                s[12] = fmaf(s[12], c, b3.x); s[13] = fmaf(s[13], c, b3.y);
-                s[14] = fmaf(s[14], c, b3.z); s[15] = fmaf(s[15], c, b3.w);
-                mx = max3(mx, max3(s[0], s[1], s[2]), max3(s[3], s[4], s[5]));
-                mx = max3(mx, max3(s[6], s[7], s[8]), max3(s[9], s[10], s[11]));
-                mx = max3(mx, max3(s[12], s[13], s[14]), s[15]);
-                uint32_t sb[16];
+            // ---- pass 1: biased scores (log2 units) back into S, and their
+            // maximum.  Every key row, without branches (a row outside this
+            // query's window reads the table's all-masked row), two rows
+            // per wait for the loads, one running maximum per row slot.
+            constexpr int kB = 2;
+            float mxr[kB] = {-3.0e38f, -3.0e38f};
+#pragma unroll 2
+            for (int i0 = 0; i0 < NKR; i0 += kB) {
+                float s[kB][16];
 #pragma unroll
-                for (int t = 0; t < 16; ++t) sb[t] = __float_as_uint(s[t]);
-                tmem_st16(tS + 16u * (uint32_t)i, sb);
+                for (int r = 0; r < kB; ++r)
+                    if (i0 + r < NKR) tmem_ld16(tS + 16u * (uint32_t)(i0 + r), s[r]);
+                tmem_ld_wait();
+#pragma unroll
+                for (int r = 0; r < kB; ++r) {
+                    const int i = i0 + r;
+                    if (i >= NKR) continue;
+                    float *x = s[r];
+                    const float4 *br = tq + ((unsigned)(i - wy) < (unsigned)k ? (a0 + i) : nrel) * 4;
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        const float4 bb = br[t];
+                        x[4 * t + 0] = fmaf(x[4 * t + 0], c, bb.x);
+                        x[4 * t + 1] = fmaf(x[4 * t + 1], c, bb.y);
+                        x[4 * t + 2] = fmaf(x[4 * t + 2], c, bb.z);
+                        x[4 * t + 3] = fmaf(x[4 * t + 3], c, bb.w);
+                    }
+                    const float m0 = max3(max3(x[0], x[1], x[2]), max3(x[3], x[4], x[5]), max3(x[6], x[7], x[8]));
+                    const float m1 = max3(max3(x[9], x[10], x[11]), max3(x[12], x[13], x[14]), x[15]);
+                    mxr[r] = max3(mxr[r], m0, m1);
+                    uint32_t sb[16];
+#pragma unroll
+                    for (int t = 0; t < 16; ++t) sb[t] = __float_as_uint(x[t]);
+                    tmem_st16(tS + 16u * (uint32_t)i, sb);
+                }
             }
+            const float mx = fmaxf(mxr[0], mxr[1]);
             tmem_st_wait();
             // ---- pass 2: P = exp2(score - max) as 16-bit pairs over the first
             // 8 NKR columns (key row i at columns 8i .. 8i + 7, whose scores
-            // were read at row i / 2 <= i); rows outside every window: zeros
-            float l0 = 0.f, l1 = 0.f;
-            for (int i = 0; i < NKR; ++i) {
-                uint32_t pk[8];
-                if ((wrows >> i) & 1u) {
-                    float s[16];
-                    tmem_ld16(tS + 16u * (uint32_t)i, s);
-                    tmem_ld_wait();
+            // were read at row i / 2 <= i); one row-sum accumulator per row slot
+            float lr[kB] = {0.f, 0.f};
+#pragma unroll 2
+            for (int i0 = 0; i0 < NKR; i0 += kB) {
+                float s[kB][16];
+#pragma unroll
+                for (int r = 0; r < kB; ++r)
+                    if (i0 + r < NKR) tmem_ld16(tS + 16u * (uint32_t)(i0 + r), s[r]);
+                tmem_ld_wait();
+#pragma unroll
+                for (int r = 0; r < kB; ++r) {
+                    const int i = i0 + r;
+                    if (i >= NKR) continue;
+                    uint32_t pk[8];
 #pragma unroll
                     for (int t = 0; t < 8; ++t) {
-                        const float p0 = ex2(s[2 * t] - mx), p1 = ex2(s[2 * t + 1] - mx);
-                        if (t & 1) l1 += p0 + p1; else l0 += p0 + p1;
-                        pk[t] = Pack2<T>::run(p0, p1);
+                        const float p0 = ex2(s[r][2 * t] - mx), p1 = ex2(s[r][2 * t + 1] - mx);
+                        pk[t] = PackP<T>::run(p0, p1, lr[r]);
                     }
-                } else {
-#pragma unroll
-                    for (int t = 0; t < 8; ++t) pk[t] = 0u;
+                    tmem_st8(tS + 8u * (uint32_t)i, pk);
                 }
-                tmem_st8(tS + 8u * (uint32_t)i, pk);
             }
+            const float l0 = lr[0], l1 = lr[1];
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
@@ -446,13 +487,21 @@ int strip_key_rows(int Lg, int k, int kr0[2]) {
     return nkr;
 }
 
+template <typename T> void (*ugrp_kernel(int nkr))(UgrpParams) {
+    switch (nkr) {
+    case 9: return fwd_ugrp_kernel<T, 9>;
+    case 10: return fwd_ugrp_kernel<T, 10>;
+    case 11: return fwd_ugrp_kernel<T, 11>;
+    case 12: return fwd_ugrp_kernel<T, 12>;
+    case 13: return fwd_ugrp_kernel<T, 13>;
+    case 14: return fwd_ugrp_kernel<T, 14>;
+    default: return nullptr;
+    }
+}
+
 template <typename T>
 cudaError_t launch_ugrp_t(const Problem &pr, const void *q, const void *k, const void *v, const void *rpb, void *out,
                           cudaStream_t st, bool *launched) {
-    const void *kern = reinterpret_cast<const void *>(&fwd_ugrp_kernel<T>);
-    int sms = 0, cap = 0;
-    cudaError_t e = ugrp_device(&sms, &cap, kern);
-    if (e != cudaSuccess) return e;
     UgrpParams up{};
     const int64_t bh = pr.bh();
     const int dd = pr.d * pr.d;
@@ -461,7 +510,12 @@ cudaError_t launch_ugrp_t(const Problem &pr, const void *q, const void *k, const
     up.Lgx = pr.W / pr.d;
     if (gu <= 0 || gu >= INT32_MAX || bh * up.Lgy >= INT32_MAX) return cudaSuccess;
     up.NKR = strip_key_rows(up.Lgy, pr.k, up.kr0);
-    if (up.NKR > kMaxNKR) return cudaSuccess;
+    void (*kfn)(UgrpParams) = ugrp_kernel<T>(up.NKR);   // NKR is 9 .. 14 for k = 9 .. 13 and groups <= 16
+    if (!kfn) return cudaSuccess;
+    const void *kern = reinterpret_cast<const void *>(kfn);
+    int sms = 0, cap = 0;
+    cudaError_t e = ugrp_device(&sms, &cap, kern);
+    if (e != cudaSuccess) return e;
     if (!encode_group_map(&up.tq, q, pr.dtype, bh, pr.H, pr.W, pr.d, 16, 16, 1) ||
         !encode_group_map(&up.tk, k, pr.dtype, bh, pr.H, pr.W, pr.d, 16, 16, 1) ||
         !encode_group_map(&up.tv, v, pr.dtype, bh, pr.H, pr.W, pr.d, 16, 16, 1))
@@ -479,7 +533,9 @@ cudaError_t launch_ugrp_t(const Problem &pr, const void *q, const void *k, const
     up.tab_bytes = 16 * up.qstride;
     up.off_tab = NSTG * kStage;
     up.off_bar = up.off_tab + 2 * up.tab_bytes;
-    const uint32_t smem = up.off_bar + 16 * NSTG + 72 + 1024;   // + 1024 bytes for aligning the base
+    up.off_rpb = up.off_bar + 16 * NSTG + 80;   // two planes' (2k - 1)^2 bias values
+    const int nrel = 2 * pr.k - 1;
+    const uint32_t smem = up.off_rpb + 2u * nrel * nrel * 4u + 1024;   // + 1024 bytes for aligning the base
     if ((int)smem > cap) return cudaSuccess;
     // units per block at most d^2 + 1, so that a block's units lie in at
     // most two (batch, head) planes
@@ -495,7 +551,7 @@ cudaError_t launch_ugrp_t(const Problem &pr, const void *q, const void *k, const
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const cudaError_t el = cudaLaunchKernelEx(&cfg, fwd_ugrp_kernel<T>, up);
+    const cudaError_t el = cudaLaunchKernelEx(&cfg, kfn, up);
     *launched = true;
     note_kernel("fwd_ugrp_kernel");
     return el != cudaSuccess ? el : cudaGetLastError();
