@@ -93,28 +93,21 @@ __device__ __forceinline__ void tmem_st8(uint32_t ta, const uint32_t *v) {
                  : "memory");
 }
 
-// P as 16-bit pairs and its contribution to the row sum.  bf16: the upper
-// halves of the fp32 values (rounding toward zero, relative error below
-// 2^-8), packed by one byte permute on the integer pipe instead of a
-// conversion on the pipe the exponentials use; the row sum adds exactly the
-// values packed, so the normalisation matches the P of the products.  f16:
-// round-to-nearest conversion, row sum of the fp32 values.
-template <typename T> struct PackP;
-template <> struct PackP<__nv_bfloat16> {
-    __device__ __forceinline__ static uint32_t run(float p0, float p1, float &l) {
-        const uint32_t a = __float_as_uint(p0), b = __float_as_uint(p1);
-        uint32_t r;
-        asm("prmt.b32 %0, %1, %2, 0x7632;\n" : "=r"(r) : "r"(a), "r"(b));
-        l += __uint_as_float(a & 0xffff0000u) + __uint_as_float(b & 0xffff0000u);
-        return r;
-    }
-};
-template <> struct PackP<__half> {
-    __device__ __forceinline__ static uint32_t run(float p0, float p1, float &l) {
-        l += p0 + p1;
-        return Pack2<__half>::run(p0, p1);
-    }
-};
+// 2^x for x <= 0 on the FMA and integer pipes, for a share of the
+// exponentials that the MUFU pipe (4 results per clock and sub-partition)
+// would otherwise serialise: x = r + f with r = round(x) and |f| <= 1/2; 2^f
+// from a cubic fitted to it on [-1/2, 1/2] (least squares on the relative
+// error, with p(0) = 1; largest relative error 1.0e-4, below the 16-bit
+// rounding of P), then r added to the exponent field.  Arguments below -125
+// (masked keys) give 2^-125, which rounds to zero in f16 and contributes
+// nothing measurable in bf16.
+__device__ __forceinline__ float ex2_fma(float x) {
+    x = fmaxf(x, -125.f);
+    const float xr = x + 12582912.f;   // 1.5 * 2^23: round(x) in the low mantissa bits
+    const float f = x - (xr - 12582912.f);
+    const float p = fmaf(fmaf(fmaf(0.05500755f, f, 0.24220777f), f, 0.69328272f), f, 1.f);
+    return __int_as_float(__float_as_int(p) + (__float_as_int(xr) << 23));
+}
 
 // ---------------------------------------------------------------------------
 // Kernel.
@@ -202,16 +195,22 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_ugrp_kernel(const __grid_cons
             rpbs[i] = rpb ? Elem<T>::to_f(rpb[(int64_t)h * nr2 + r]) * kLog2e : 0.f;
         }
         __syncthreads();
-        const int per_tab = 16 * 2 * k * 16;
-        for (int i = threadIdx.x; i < nplanes * per_tab; i += kThreads) {
-            const int t = i / per_tab, r = i - t * per_tab;
-            const int qc = r / (2 * k * 16), a = (r / 16) % (2 * k), j = r & 15;
+        // one 16-entry table row (plane t, query column qc, row a) per step
+        const int rows_per_tab = 16 * 2 * k;
+        for (int ri = threadIdx.x; ri < nplanes * rows_per_tab; ri += kThreads) {
+            const int t = ri / rows_per_tab, rr = ri - t * rows_per_tab;
+            const int qc = rr / (2 * k), a = rr - qc * (2 * k);
             const int qcc = min(qc, p.Lgx - 1);
             const int wx = window_start(qcc, p.Lgx, k);
-            float v = kMasked;
-            if (a < nrel && (unsigned)(j - wx) < (unsigned)k) v = rpbs[t * nr2 + a * nrel + (j - qcc + k - 1)];
-            *reinterpret_cast<float *>(smem + p.off_tab + (uint32_t)t * p.tab_bytes + (uint32_t)qc * p.qstride +
-                                       (uint32_t)(a * 16 + j) * 4u) = v;
+            // key column j of query column qcc is bias column j - qcc + k - 1
+            const float *src = rpbs + t * nr2 + a * nrel + (k - 1 - qcc);
+            float v[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] = (a < nrel && (unsigned)(j - wx) < (unsigned)k) ? src[j] : kMasked;
+            float4 *dst = reinterpret_cast<float4 *>(smem + p.off_tab + (uint32_t)t * p.tab_bytes +
+                                                     (uint32_t)qc * p.qstride + (uint32_t)a * 64u);
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) dst[q4] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
         }
         if (warp == kWarpMma) tmem_alloc(smem_u32(tmem_slot));
         tc_fence_before();
@@ -312,6 +311,37 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_ugrp_kernel(const __grid_cons
         const unsigned char *tab_q = smem + p.off_tab + (uint32_t)qc * p.qstride;
         const int nrel = 2 * k - 1;
 
+        float l_prev = 1.f;   // row sum of the unit whose output is pending
+        // O of unit jj (ready once its P.V completed) / row sum -> 64 bytes
+        auto epilogue = [&](int jj) -> bool {
+            const bool oko = mb_wait(bar_o + 8 * e, (uint32_t)(jj & 1), p.wait_limit);
+            if (!__all_sync(0xffffffffu, oko)) {
+                if (lane == 0) {
+                    atomicAdd(&g_ugrp_timeouts, 1u);
+                    *abort_flag = 1;
+                }
+                return false;
+            }
+            tc_fence_after();
+            float o[32];
+            tmem_ld32(tO, o);
+            tmem_ld_wait();
+            if (qok) {
+                float inv;
+                asm("rcp.approx.ftz.f32 %0, %1;\n" : "=f"(inv) : "f"(l_prev));
+                const int g = u_begin + jj;
+                const int bh = g / dd, rem = g - bh * dd, gy = rem / p.d, gx = rem - gy * p.d;
+                uint4 *dst = reinterpret_cast<uint4 *>(
+                    p.out + ((((size_t)bh * p.H + gy + (size_t)p.d * row) * p.W) + gx + (size_t)p.d * qc) * 64);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    dst[i] = make_uint4(Pack2<T>::run(o[8 * i + 0] * inv, o[8 * i + 1] * inv),
+                                        Pack2<T>::run(o[8 * i + 2] * inv, o[8 * i + 3] * inv),
+                                        Pack2<T>::run(o[8 * i + 4] * inv, o[8 * i + 5] * inv),
+                                        Pack2<T>::run(o[8 * i + 6] * inv, o[8 * i + 7] * inv));
+            }
+            return true;
+        };
         for (int j = 0; j < nst; ++j) {
             const int g = u_begin + j;
             const int bh = g / dd;
@@ -379,45 +409,27 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_ugrp_kernel(const __grid_cons
                     const int i = i0 + r;
                     if (i >= NKR) continue;
                     uint32_t pk[8];
+                    // columns 3, 7, 11 and 15 on the FMA pipe, the rest on MUFU
 #pragma unroll
                     for (int t = 0; t < 8; ++t) {
-                        const float p0 = ex2(s[r][2 * t] - mx), p1 = ex2(s[r][2 * t + 1] - mx);
-                        pk[t] = PackP<T>::run(p0, p1, lr[r]);
+                        const float x0 = s[r][2 * t] - mx, x1 = s[r][2 * t + 1] - mx;
+                        const float p0 = ex2(x0), p1 = (t & 1) ? ex2_fma(x1) : ex2(x1);
+                        lr[r] += p0 + p1;
+                        pk[t] = Pack2<T>::run(p0, p1);
                     }
                     tmem_st8(tS + 8u * (uint32_t)i, pk);
                 }
             }
-            const float l0 = lr[0], l1 = lr[1];
+            // ---- the previous unit's epilogue (its P.V completed while this
+            // unit's scores were computed), before P_j is handed over: P.V_j
+            // overwrites O_e only after the arrive below
+            if (j > 0 && !epilogue(j - 1)) break;
+            l_prev = lr[0] + lr[1];
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mb_arrive(bar_p + 8 * e);
-            // ---- epilogue: O / row sum -> 64 bytes
-            const bool oko = mb_wait(bar_o + 8 * e, (uint32_t)(j & 1), p.wait_limit);
-            if (!__all_sync(0xffffffffu, oko)) {
-                if (lane == 0) {
-                    atomicAdd(&g_ugrp_timeouts, 1u);
-                    *abort_flag = 1;
-                }
-                break;
-            }
-            tc_fence_after();
-            float o[32];
-            tmem_ld32(tO, o);
-            tmem_ld_wait();
-            if (qok) {
-                float inv;
-                asm("rcp.approx.ftz.f32 %0, %1;\n" : "=f"(inv) : "f"(l0 + l1));
-                const int rem = g - bh * dd, gy = rem / p.d, gx = rem - gy * p.d;
-                uint4 *dst = reinterpret_cast<uint4 *>(
-                    p.out + ((((size_t)bh * p.H + gy + (size_t)p.d * row) * p.W) + gx + (size_t)p.d * qc) * 64);
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    dst[i] = make_uint4(Pack2<T>::run(o[8 * i + 0] * inv, o[8 * i + 1] * inv),
-                                        Pack2<T>::run(o[8 * i + 2] * inv, o[8 * i + 3] * inv),
-                                        Pack2<T>::run(o[8 * i + 4] * inv, o[8 * i + 5] * inv),
-                                        Pack2<T>::run(o[8 * i + 6] * inv, o[8 * i + 7] * inv));
-            }
+            if (j == nst - 1) epilogue(j);
         }
     }
     // ---- teardown: TMEM released by the warp that took it, after every
