@@ -48,7 +48,11 @@ CSRC = "neighborhood_attention_na2d_b200/csrc/"
 # code that plans and launches it).
 KERNEL_SOURCES = {
     "fwd_stream_kernel": [CSRC + "na2d_stream.cu", CSRC + "na2d_device.cuh", CSRC + "na2d_launch.h"],
-    "fwd_umma_kernel": [CSRC + "na2d_umma.cu", CSRC + "na2d_tc.cu", CSRC + "na2d_device.cuh", CSRC + "na2d_launch.h"],
+    "fwd_umma_kernel": [CSRC + "na2d_umma.cu", CSRC + "na2d_tc.cu", CSRC + "na2d_tcgen05.cuh", CSRC + "na2d_device.cuh",
+                        CSRC + "na2d_launch.h"],
+    "fwd_ugrp_kernel": [CSRC + "na2d_ugrp.cu", CSRC + "na2d_tc.cu", CSRC + "na2d_tcgen05.cuh", CSRC + "na2d_device.cuh",
+                        CSRC + "na2d_launch.h"],
+    "fwd_tc_kernel": [CSRC + "na2d_tc.cu", CSRC + "na2d_device.cuh", CSRC + "na2d_launch.h"],
 }
 
 
@@ -82,9 +86,12 @@ def hbm_peak() -> tuple[float, str]:
 
 def recorded_traffic(kernel: str, workload: str) -> int | None:
     """DRAM bytes per launch from the committed ncu summary of this kernel on
-    this workload, only if it was taken on the current kernel source."""
+    this workload, only if it was taken on the current kernel source.  A
+    kernel name with a mode suffix ("fwd_tc_kernel/full") is looked up by the
+    kernel's name."""
+    kernel = kernel.split("/")[0]
     f = PROFILES / f"{kernel}_{workload}.md"
-    if not f.exists():
+    if not f.exists() or kernel not in KERNEL_SOURCES:
         return None
     text = f.read_text()
     m = re.search(r"traffic_per_launch_bytes\s*=\s*(\d+)\s*;\s*kernel_sha\s*=\s*([0-9a-f]+)", text)
@@ -359,6 +366,20 @@ def tensor_peak() -> tuple[float, str]:
         return 1590.0, "fallback"
 
 
+def step_traffic(kerns, workload: str) -> int | None:
+    """Recorded DRAM bytes of one step: the one kernel's per-launch figure, or
+    the sum over the shapes' kernels when each shape runs a different kernel
+    (each has its own summary for this workload); None if any is missing."""
+    if not kerns:
+        return None
+    if isinstance(kerns, str):
+        kerns = [kerns]
+    if len(set(kerns)) != len(kerns):
+        return None
+    got = [recorded_traffic(k, workload) for k in kerns]
+    return None if any(g is None for g in got) else sum(got)
+
+
 def roofline(wl, ms_per_step, kern):
     """Roofline of one step: the slower of the algorithmic bytes at the HBM
     peak and the useful FLOPs at the tensor peak; achieved is measured against
@@ -378,7 +399,7 @@ def roofline(wl, ms_per_step, kern):
         achieved = flops / sec / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": tc, "unit": "TFLOP/s", "frac": achieved / tc,
                 "peak_source": f"{tc_kind} bf16_tflops (burst)"}
-    roof.update({"traffic": recorded_traffic(kern, wl.name) if kern else None,
+    roof.update({"traffic": step_traffic(kern, wl.name),
                  "algorithmic_bytes_per_step": alg_bytes, "useful_flops_per_step": flops,
                  "t_hbm_us": t_hbm * 1e6, "t_tensor_us": t_tc * 1e6, "kernel": kern})
     return roof
@@ -412,7 +433,7 @@ def run_ours(args, world, rank, local):
     units_rank = sum(s.B * s.heads * s.H * s.W for s in wl.shapes)
     value = world * units_rank / (ms_per_step / 1e3)
     kern = kernels_of(wl)
-    roof = roofline(wl, ms_per_step, kern[0] if len(set(kern)) == 1 else None)
+    roof = roofline(wl, ms_per_step, kern[0] if len(set(kern)) == 1 else kern)
     del sets
 
     # ---- the other workloads of the same problem, each timed the same way (1 GPU)
@@ -425,7 +446,7 @@ def run_ours(args, world, rank, local):
             s2, _ = make_sets(w2, dev, rank, l2)
             t2 = time_steps(w2, s2, K, args.warmup, dev, None)
             k2 = kernels_of(w2)
-            r2 = roofline(w2, t2["ms_per_step"], k2[0] if len(set(k2)) == 1 else None)
+            r2 = roofline(w2, t2["ms_per_step"], k2[0] if len(set(k2)) == 1 else k2)
             per_wl[name] = {"ms_per_step": t2["ms_per_step"],
                             "value": sum(s.B * s.heads * s.H * s.W for s in w2.shapes) / (t2["ms_per_step"] / 1e3),
                             "frac": r2["frac"], "bound": r2["bound"], "achieved": r2["achieved"],

@@ -25,12 +25,12 @@
 //    fragment gives the softmax row sums from the same rounded P.  The
 //    softmax runs in registers; masking and the relative-position bias come
 //    from one bank-conflict-free shared table lookup per score.
-//  * Three compile-time modes share that tile routine.  FULL: every dilation
+//  * Compile-time modes share that tile routine.  FULL: every dilation
 //    group has at least NKR rows, so all NKR halo rows exist and the staged
 //    halo has a fixed row stride (loads use immediate offsets, the tile body
-//    has no branches).  DENSE: H = W = k*d, every window is its whole k x k
-//    group (DiNAT's layers whose dilated window spans the map).  GENERIC:
-//    everything else, with run-time halo geometry.
+//    has no branches).  DENSE (TMA path only, k <= 5 in practice): H = W =
+//    k*d, every window is its whole k x k group.  GENERIC: everything else,
+//    with run-time halo geometry.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -52,7 +52,7 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kPix = 64;   // bytes per D = 32 row of a 16-bit type
 
-enum Mode : int { kGeneric = 0, kFull = 1, kDense = 2, kFullTma = 3, kDenseTma = 4 };
+enum Mode : int { kGeneric = 0, kFull = 1, kFullTma = 3, kDenseTma = 4 };
 
 // Per-k warp tile: TQY x TQX queries (16), halo NKR = TQY + K - 1 rows by NKC
 // columns (padded to a multiple of 8), processed in chunks of CH 8-key tiles;
@@ -71,7 +71,7 @@ constexpr int cround(int x, int m) { return (x + m - 1) / m * m; }
 template <int K, int MODE> struct Geo {
     using C = Cfg<K>;
     static constexpr int TQY = C::TQY, TQX = C::TQX, NKC = C::NKC, TILES = C::TILES, TILES_TMA = C::TILES_TMA;
-    static constexpr bool DENSE = MODE == kDense || MODE == kDenseTma;
+    static constexpr bool DENSE = MODE == kDenseTma;
     static constexpr bool FULL = MODE == kFull || MODE == kFullTma;
     static constexpr bool GENERIC = MODE == kGeneric;
     static constexpr bool TMA = MODE == kFullTma || MODE == kDenseTma;
@@ -783,15 +783,16 @@ cudaError_t launch_geometry(const void *kern, int smem, int *sms, int *occ, int 
     return cudaSuccess;
 }
 
+// (Maps whose groups are all exactly k long take the TMA block kernel for
+// k <= 7 and the tcgen05 group kernel for k >= 9; should either decline, the
+// GENERIC geometry covers them.)
 template <int K> int pick_mode(const Problem &p) {
-    if (p.H == K * p.d && p.W == K * p.d) return kDense;
     if (p.H / p.d >= Geo<K, kFull>::NKR) return kFull;
     return kGeneric;
 }
 
 // Block shapes.  FULL: one column group per block, the group's warp-tile
-// columns split into n_jc equal chunks of at most TILES tiles.  DENSE: whole
-// k x k groups, BG of them per block (about 8 warp tiles).  GENERIC: BJ group
+// columns split into n_jc equal chunks of at most TILES tiles.  GENERIC: BJ group
 // columns by BG column groups, the first candidate (widest BJ first, then the
 // most column groups) whose two stages plus bias tables fit in shared memory.
 // Returns the shared-memory bytes, or -1 if nothing fits.
@@ -815,18 +816,6 @@ int plan_blocks(const Problem &p, Args &a, int mode, int smem_cap) {
         a.q_bytes = a.BJQ * G::TQY * kPix;
         a.kv_bytes = G::NKR * G::CCM * kPix;
         ok = a.tab_bytes + 2 * (a.q_bytes + 2 * a.kv_bytes) <= smem_cap;
-    } else if (mode == kDense) {
-        using G = Geo<K, kDense>;
-        a.BJ = a.BJQ = G::TPG * G::TQX;
-        a.n_jc = 1;
-        a.RMAX = K;
-        a.CCMAX = G::CCM;
-        for (a.BG = std::max(1, std::min(p.d, kWarps / G::TPG)); a.BG >= 1 && !ok; --a.BG) {
-            a.q_bytes = a.BG * a.BJQ * G::TQY * kPix;
-            a.kv_bytes = a.BG * K * G::CCM * kPix;
-            ok = a.tab_bytes + 2 * (a.q_bytes + 2 * a.kv_bytes) <= smem_cap;
-            if (ok) break;
-        }
     } else {
         a.RMAX = std::min(GG::NKR, Lgy_max);
         for (int bj = std::min(round_up(Lgx_max, GG::TQX), 8 * GG::TQX); bj >= GG::TQX && !ok; bj -= GG::TQX) {
@@ -857,7 +846,7 @@ cudaError_t launch_mode(const Args &a, int smem, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     const int64_t grid = std::min<int64_t>(a.nblocks, (int64_t)sms * occ);
     kern<<<(unsigned)grid, kThreads, smem, st>>>(a);
-    note_kernel(MODE == kFull ? "fwd_tc_kernel/full" : MODE == kDense ? "fwd_tc_kernel/dense" : "fwd_tc_kernel/generic");
+    note_kernel(MODE == kFull ? "fwd_tc_kernel/full" : "fwd_tc_kernel/generic");
     return cudaGetLastError();
 }
 
@@ -981,7 +970,6 @@ cudaError_t launch_impl(const Problem &p, const void *q, const void *k, const vo
     if (smem < 0 && mode != kGeneric) smem = plan_blocks<K>(p, a, mode = kGeneric, f.second);
     if (smem < 0) return cudaErrorInvalidConfiguration;
     if (mode == kFull) return launch_mode<T, K, kFull>(a, smem, st);
-    if (mode == kDense) return launch_mode<T, K, kDense>(a, smem, st);
     return launch_mode<T, K, kGeneric>(a, smem, st);
 }
 

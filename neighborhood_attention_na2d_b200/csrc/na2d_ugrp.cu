@@ -573,7 +573,7 @@ cudaError_t launch_ugrp_t(const Problem &pr, const void *q, const void *k, const
 
 bool ugrp_supported(const Problem &p) {
     if (p.dtype != DType::F16 && p.dtype != DType::BF16) return false;
-    if (p.D != 32 || p.k < 9 || p.k > 13 || !(p.k & 1) || p.d < 1 || p.heads > 4096) return false;
+    if (p.D != 32 || p.k < 9 || p.k > 13 || !(p.k & 1) || p.d < 1) return false;
     if (p.H % p.d || p.W % p.d) return false;
     const int Lgy = p.H / p.d, Lgx = p.W / p.d;
     return Lgy >= p.k && Lgy <= 16 && Lgx >= p.k && Lgx <= 16;
