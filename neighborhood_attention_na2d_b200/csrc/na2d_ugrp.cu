@@ -114,8 +114,17 @@ __device__ __forceinline__ float ex2_fma(float x) {
 // ---------------------------------------------------------------------------
 template <typename T, int NKR>
 __global__ void __launch_bounds__(kThreads, 1) fwd_ugrp_kernel(const __grid_constant__ UgrpParams p) {
-    static_assert(NKR >= 1 && NKR <= kMaxNKR, "key tile of 1 .. 14 group rows");
-    constexpr int N = 16 * NKR;
+    static_assert(NKR >= 2 && NKR <= kMaxNKR, "key tile of 2 .. 14 group rows");
+    // The key tile's rows in two halves: lower rows 0 .. NL - 1 and upper rows
+    // NL .. NKR - 1, whose scores are computed by separate MMAs into two
+    // TMEM regions of HS columns each.  For unit j with h = j & 1 the upper
+    // scores go to region h and the lower ones to region 1 - h; P is written
+    // into region h (over the upper scores: order index o = upper rows first,
+    // then lower rows, at column 8o).  Unit j + 1's upper scores then go to
+    // region 1 - h, free once unit j's softmax has read its lower scores, and
+    // can be computed before unit j's P.V; its lower scores follow the P.V.
+    constexpr int NL = NKR / 2, NH = NKR - NL;
+    constexpr int HS = 16 * NH;
     extern __shared__ unsigned char smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t sbase = (raw + 1023u) & ~1023u;   // swizzled tiles need 1024-byte alignment
@@ -137,12 +146,13 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_ugrp_kernel(const __grid_cons
 
     const uint32_t bar_full = sbase + p.off_bar;        // [NSTG] stage landed (TMA bytes)
     const uint32_t bar_empty = bar_full + 8 * NSTG;     // [NSTG] stage consumed (two commits)
-    const uint32_t bar_s = bar_empty + 8 * NSTG;        // [2] S_e ready (commit)
-    const uint32_t bar_p = bar_s + 16;                  // [2] P_e written (4 warps)
+    const uint32_t bar_sh = bar_empty + 8 * NSTG;       // [2] upper scores of strip e ready (commit)
+    const uint32_t bar_sl = bar_sh + 16;                // [2] lower scores ready (commit)
+    const uint32_t bar_p = bar_sl + 16;                 // [2] P_e written (4 warps)
     const uint32_t bar_o = bar_p + 16;                  // [2] O_e ready (commit)
     const uint32_t bar_drain = bar_o + 16;              // [2] all MMAs of an MMA warp done (commit)
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + p.off_bar + 16 * NSTG + 64);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + p.off_bar + 16 * NSTG + 68);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + p.off_bar + 16 * NSTG + 80);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + p.off_bar + 16 * NSTG + 84);
 
     auto issue_unit = [&](int j) {
         const uint32_t fb = bar_full + 8 * (j % NSTG);
@@ -167,7 +177,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_ugrp_kernel(const __grid_cons
                 mb_init(bar_empty + 8 * i, 2);
             }
             for (int i = 0; i < 2; ++i) {
-                mb_init(bar_s + 8 * i, 1);
+                mb_init(bar_sh + 8 * i, 1);
+                mb_init(bar_sl + 8 * i, 1);
                 mb_init(bar_p + 8 * i, 4);
                 mb_init(bar_o + 8 * i, 1);
                 mb_init(bar_drain + 8 * i, 1);
@@ -240,32 +251,41 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_ugrp_kernel(const __grid_cons
         }
     } else if (warp == kWarpMma || warp == kWarpMma + 1) {
         // =================== MMA issuers ===================
-        // Warp kWarpMma + e issues strip e of every unit: S_0, then per unit
-        // j: O_j = P_j V_j, S_{j+1} = Q K^T.  S_{j+1} reuses the columns of
-        // P_j after the P.V that reads them (tcgen05.mma of one thread
-        // execute in issue order); O_j is free again once the warpgroup's
-        // epilogue of unit j - 1, which precedes its P_j, has read it.
+        // Warp kWarpMma + e issues strip e of every unit: unit 0's upper and
+        // lower Q K^T, then per unit j: unit j + 1's upper Q K^T (into the
+        // region unit j's softmax has finished reading), O_j = P_j V_j, unit
+        // j + 1's lower Q K^T (into the region of P_j, after the P.V that
+        // reads it: tcgen05.mma of one thread execute in issue order).  O_j
+        // is free again once the warpgroup's epilogue of unit j - 1, which
+        // precedes its P_j, has read it.
         const int e = warp - kWarpMma;
         if (lane == 0) {
-            const uint32_t idesc_qk = idesc_f16<T>(N, 0);
+            constexpr uint32_t idesc_hi = idesc_f16<T>(16 * NH, 0);
+            constexpr uint32_t idesc_lo = idesc_f16<T>(16 * NL, 0);
             constexpr uint32_t idesc_pv = idesc_f16<T>(32, 1);
             const uint32_t koff = (uint32_t)p.kr0[e] * 1024u;   // 16 pixels of 64 bytes per group row
-            const uint32_t dS = tmem + (uint32_t)(e * N), dO = tmem + (uint32_t)(2 * N + 32 * e);
-            auto issue_qk = [&](int j) -> bool {
+            const uint32_t dR = tmem + (uint32_t)(e * 2 * HS), dO = tmem + (uint32_t)(4 * HS + 32 * e);
+            // one half of unit j's Q K^T; the upper half first waits for the unit's copies
+            auto issue_qk = [&](int j, bool upper) -> bool {
                 const int s = j % NSTG;
-                if (!mb_wait(bar_full + 8 * s, (uint32_t)((j / NSTG) & 1), p.wait_limit) || *abort_flag) return false;
-                tc_fence_after();
+                if (upper) {
+                    if (!mb_wait(bar_full + 8 * s, (uint32_t)((j / NSTG) & 1), p.wait_limit) || *abort_flag)
+                        return false;
+                    tc_fence_after();
+                }
                 const uint32_t st = sbase + (uint32_t)s * kStage;
+                const int h = j & 1;
                 // K-major, 64-byte rows: 8-row groups 512 bytes apart; the
                 // second K = 16 step starts 32 bytes into the rows
                 const uint64_t da = sw64_desc(st + (uint32_t)e * 8192u, 16, 512);
-                const uint64_t db = sw64_desc(st + kGroupBytes + koff, 16, 512);
-                umma_ss(dS, da, db, idesc_qk, 0);
-                umma_ss(dS, da + 2, db + 2, idesc_qk, 1);
-                umma_commit(bar_s + 8 * e);
+                const uint64_t db = sw64_desc(st + kGroupBytes + koff + (upper ? (uint32_t)NL * 1024u : 0u), 16, 512);
+                const uint32_t dS = dR + (uint32_t)((upper ? h : 1 - h) * HS);
+                umma_ss(dS, da, db, upper ? idesc_hi : idesc_lo, 0);
+                umma_ss(dS, da + 2, db + 2, upper ? idesc_hi : idesc_lo, 1);
+                umma_commit((upper ? bar_sh : bar_sl) + 8 * e);
                 return true;
             };
-            bool ok = issue_qk(0);
+            bool ok = issue_qk(0, true) && issue_qk(0, false);
             for (int j = 0; ok && j < nst; ++j) {
                 const int s = j % NSTG;
                 if (!mb_wait(bar_p + 8 * e, (uint32_t)(j & 1), p.wait_limit) || *abort_flag) {
@@ -273,15 +293,24 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_ugrp_kernel(const __grid_cons
                     break;
                 }
                 tc_fence_after();
+                if (j + 1 < nst && !issue_qk(j + 1, true)) {
+                    ok = false;
+                    break;
+                }
                 const uint32_t vt = sbase + (uint32_t)s * kStage + 2 * kGroupBytes + koff;
+                const uint32_t aP = dR + (uint32_t)((j & 1) * HS);
                 // V MN-major: 64-byte rows of 32 channels, 8-key groups 512
-                // bytes apart; k-step t takes key row t (16 keys)
-                for (int t = 0; t < NKR; ++t)
-                    umma_ts(dO, dS + 8u * (uint32_t)t, sw64_desc(vt + 1024u * (uint32_t)t, 16, 512), idesc_pv,
-                            t > 0 ? 1u : 0u);
+                // bytes apart; k-step o takes P columns 8o .. 8o + 7, i.e. key
+                // row NL + o for o < NH and o - NH after
+#pragma unroll
+                for (int o = 0; o < NKR; ++o) {
+                    const int t = o < NH ? NL + o : o - NH;
+                    umma_ts(dO, aP + 8u * (uint32_t)o, sw64_desc(vt + 1024u * (uint32_t)t, 16, 512), idesc_pv,
+                            o > 0 ? 1u : 0u);
+                }
                 umma_commit(bar_o + 8 * e);
                 umma_commit(bar_empty + 8 * s);
-                if (j + 1 < nst && !issue_qk(j + 1)) ok = false;
+                if (j + 1 < nst) issue_qk(j + 1, false);
             }
             if (!ok) {
                 atomicAdd(&g_ugrp_timeouts, 1u);
@@ -306,7 +335,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_ugrp_kernel(const __grid_cons
         // table row of key-tile row i: a0 + i (relative row + k - 1) when valid
         const int a0 = p.kr0[e] - rowc + k - 1;
         const uint32_t tl = tmem + ((uint32_t)(32 * q4) << 16);
-        const uint32_t tS = tl + (uint32_t)(e * N), tO = tl + (uint32_t)(2 * N + 32 * e);
+        const uint32_t tR = tl + (uint32_t)(e * 2 * HS), tO = tl + (uint32_t)(4 * HS + 32 * e);
         const float c = p.c_log2;
         const unsigned char *tab_q = smem + p.off_tab + (uint32_t)qc * p.qstride;
         const int nrel = 2 * k - 1;
@@ -342,84 +371,110 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_ugrp_kernel(const __grid_cons
             }
             return true;
         };
-        for (int j = 0; j < nst; ++j) {
-            const int g = u_begin + j;
-            const int bh = g / dd;
-            const float4 *tq = reinterpret_cast<const float4 *>(tab_q + (uint32_t)(bh - bh_first) * p.tab_bytes);
-            const bool ok = mb_wait(bar_s + 8 * e, (uint32_t)(j & 1), p.wait_limit);
+        constexpr int kB = 2;   // key rows per wait for the TMEM loads
+        // batches unrolled two deep (one deep at NKR = 12, where two spill registers)
+        constexpr int kU = NKR == 12 ? 1 : 2;
+        const float4 *tq = nullptr;
+        float mxr[kB], lr[kB];
+        // pass 1 over CNT key rows from i_first, scores at TMEM column col0 +
+        // 16o: biased scores (log2 units) written back, running maxima.  No
+        // branches: a row outside this query's window reads the table's
+        // all-masked row.
+        auto pass1 = [&](uint32_t col0, int i_first, auto CNT) {
+            constexpr int cnt = decltype(CNT)::value;
+#pragma unroll kU
+            for (int o0 = 0; o0 < cnt; o0 += kB) {
+                float x[kB][16];
+#pragma unroll
+                for (int r = 0; r < kB; ++r)
+                    if (o0 + r < cnt) tmem_ld16(col0 + 16u * (uint32_t)(o0 + r), x[r]);
+                tmem_ld_wait();
+#pragma unroll
+                for (int r = 0; r < kB; ++r) {
+                    if (o0 + r >= cnt) continue;
+                    const int i = i_first + o0 + r;
+                    float *y = x[r];
+                    const float4 *br = tq + ((unsigned)(i - wy) < (unsigned)k ? (a0 + i) : nrel) * 4;
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        const float4 bb = br[t];
+                        y[4 * t + 0] = fmaf(y[4 * t + 0], c, bb.x);
+                        y[4 * t + 1] = fmaf(y[4 * t + 1], c, bb.y);
+                        y[4 * t + 2] = fmaf(y[4 * t + 2], c, bb.z);
+                        y[4 * t + 3] = fmaf(y[4 * t + 3], c, bb.w);
+                    }
+                    const float m0 = max3(max3(y[0], y[1], y[2]), max3(y[3], y[4], y[5]), max3(y[6], y[7], y[8]));
+                    const float m1 = max3(max3(y[9], y[10], y[11]), max3(y[12], y[13], y[14]), y[15]);
+                    mxr[r] = max3(mxr[r], m0, m1);
+                    uint32_t sb[16];
+#pragma unroll
+                    for (int t = 0; t < 16; ++t) sb[t] = __float_as_uint(y[t]);
+                    tmem_st16(col0 + 16u * (uint32_t)(o0 + r), sb);
+                }
+            }
+        };
+        // pass 2 over CNT key rows, scores at scol0 + 16o, P (16-bit pairs)
+        // to pcol0 + 8o: exp2(score - max), columns 3, 7, 11 and 15 of a row
+        // on the FMA pipe, the rest on MUFU; one row-sum accumulator per row
+        // slot
+        auto pass2 = [&](uint32_t scol0, uint32_t pcol0, float mx, auto CNT) {
+            constexpr int cnt = decltype(CNT)::value;
+#pragma unroll kU
+            for (int o0 = 0; o0 < cnt; o0 += kB) {
+                float x[kB][16];
+#pragma unroll
+                for (int r = 0; r < kB; ++r)
+                    if (o0 + r < cnt) tmem_ld16(scol0 + 16u * (uint32_t)(o0 + r), x[r]);
+                tmem_ld_wait();
+#pragma unroll
+                for (int r = 0; r < kB; ++r) {
+                    if (o0 + r >= cnt) continue;
+                    uint32_t pk[8];
+#pragma unroll
+                    for (int t = 0; t < 8; ++t) {
+                        const float x0 = x[r][2 * t] - mx, x1 = x[r][2 * t + 1] - mx;
+                        const float p0 = ex2(x0), p1 = (t & 1) ? ex2_fma(x1) : ex2(x1);
+                        lr[r] += p0 + p1;
+                        pk[t] = Pack2<T>::run(p0, p1);
+                    }
+                    tmem_st8(pcol0 + 8u * (uint32_t)(o0 + r), pk);
+                }
+            }
+        };
+        // a bounded wait for one of this strip's score commits; false ends the warpgroup
+        auto wait_scores = [&](uint32_t bar, int j) -> bool {
+            const bool ok = mb_wait(bar + 8 * e, (uint32_t)(j & 1), p.wait_limit);
             if (!__all_sync(0xffffffffu, ok) || __any_sync(0xffffffffu, *abort_flag != 0)) {
                 if (lane == 0) {
                     atomicAdd(&g_ugrp_timeouts, 1u);
                     *abort_flag = 1;
                 }
-                break;
+                return false;
             }
             tc_fence_after();
-            // ---- pass 1: biased scores (log2 units) back into S, and their
-            // maximum.  Every key row, without branches (a row outside this
-            // query's window reads the table's all-masked row), two rows
-            // per wait for the loads, one running maximum per row slot.
-            constexpr int kB = 2;
-            float mxr[kB] = {-3.0e38f, -3.0e38f};
-#pragma unroll 2
-            for (int i0 = 0; i0 < NKR; i0 += kB) {
-                float s[kB][16];
-#pragma unroll
-                for (int r = 0; r < kB; ++r)
-                    if (i0 + r < NKR) tmem_ld16(tS + 16u * (uint32_t)(i0 + r), s[r]);
-                tmem_ld_wait();
-#pragma unroll
-                for (int r = 0; r < kB; ++r) {
-                    const int i = i0 + r;
-                    if (i >= NKR) continue;
-                    float *x = s[r];
-                    const float4 *br = tq + ((unsigned)(i - wy) < (unsigned)k ? (a0 + i) : nrel) * 4;
-#pragma unroll
-                    for (int t = 0; t < 4; ++t) {
-                        const float4 bb = br[t];
-                        x[4 * t + 0] = fmaf(x[4 * t + 0], c, bb.x);
-                        x[4 * t + 1] = fmaf(x[4 * t + 1], c, bb.y);
-                        x[4 * t + 2] = fmaf(x[4 * t + 2], c, bb.z);
-                        x[4 * t + 3] = fmaf(x[4 * t + 3], c, bb.w);
-                    }
-                    const float m0 = max3(max3(x[0], x[1], x[2]), max3(x[3], x[4], x[5]), max3(x[6], x[7], x[8]));
-                    const float m1 = max3(max3(x[9], x[10], x[11]), max3(x[12], x[13], x[14]), x[15]);
-                    mxr[r] = max3(mxr[r], m0, m1);
-                    uint32_t sb[16];
-#pragma unroll
-                    for (int t = 0; t < 16; ++t) sb[t] = __float_as_uint(x[t]);
-                    tmem_st16(tS + 16u * (uint32_t)i, sb);
-                }
-            }
+            return true;
+        };
+        for (int j = 0; j < nst; ++j) {
+            const int g = u_begin + j;
+            const int bh = g / dd;
+            tq = reinterpret_cast<const float4 *>(tab_q + (uint32_t)(bh - bh_first) * p.tab_bytes);
+            // region of the upper scores (and of P), region of the lower scores
+            const uint32_t up = tR + (uint32_t)((j & 1) * HS), lo = tR + (uint32_t)((1 - (j & 1)) * HS);
+            // ---- pass 1: the upper rows as soon as their scores land (the
+            // previous unit's P.V may still run), then the lower rows
+            mxr[0] = mxr[1] = -3.0e38f;
+            if (!wait_scores(bar_sh, j)) break;
+            pass1(up, NL, std::integral_constant<int, NH>{});
+            if (!wait_scores(bar_sl, j)) break;
+            pass1(lo, 0, std::integral_constant<int, NL>{});
             const float mx = fmaxf(mxr[0], mxr[1]);
             tmem_st_wait();
-            // ---- pass 2: P = exp2(score - max) as 16-bit pairs over the first
-            // 8 NKR columns (key row i at columns 8i .. 8i + 7, whose scores
-            // were read at row i / 2 <= i); one row-sum accumulator per row slot
-            float lr[kB] = {0.f, 0.f};
-#pragma unroll 2
-            for (int i0 = 0; i0 < NKR; i0 += kB) {
-                float s[kB][16];
-#pragma unroll
-                for (int r = 0; r < kB; ++r)
-                    if (i0 + r < NKR) tmem_ld16(tS + 16u * (uint32_t)(i0 + r), s[r]);
-                tmem_ld_wait();
-#pragma unroll
-                for (int r = 0; r < kB; ++r) {
-                    const int i = i0 + r;
-                    if (i >= NKR) continue;
-                    uint32_t pk[8];
-                    // columns 3, 7, 11 and 15 on the FMA pipe, the rest on MUFU
-#pragma unroll
-                    for (int t = 0; t < 8; ++t) {
-                        const float x0 = s[r][2 * t] - mx, x1 = s[r][2 * t + 1] - mx;
-                        const float p0 = ex2(x0), p1 = (t & 1) ? ex2_fma(x1) : ex2(x1);
-                        lr[r] += p0 + p1;
-                        pk[t] = Pack2<T>::run(p0, p1);
-                    }
-                    tmem_st8(tS + 8u * (uint32_t)i, pk);
-                }
-            }
+            // ---- pass 2: P of the upper rows over their own scores (P row o
+            // at 8o overwrites scores of row o / 2 <= o, already read), then
+            // P of the lower rows after them (over upper scores, all read)
+            lr[0] = lr[1] = 0.f;
+            pass2(up, up, mx, std::integral_constant<int, NH>{});
+            pass2(lo, up + 8u * NH, mx, std::integral_constant<int, NL>{});
             // ---- the previous unit's epilogue (its P.V completed while this
             // unit's scores were computed), before P_j is handed over: P.V_j
             // overwrites O_e only after the arrive below
@@ -545,7 +600,7 @@ cudaError_t launch_ugrp_t(const Problem &pr, const void *q, const void *k, const
     up.tab_bytes = 16 * up.qstride;
     up.off_tab = NSTG * kStage;
     up.off_bar = up.off_tab + 2 * up.tab_bytes;
-    up.off_rpb = up.off_bar + 16 * NSTG + 80;   // two planes' (2k - 1)^2 bias values
+    up.off_rpb = up.off_bar + 16 * NSTG + 96;   // after the barriers, abort flag and TMEM slot: two planes' (2k - 1)^2 bias values
     const int nrel = 2 * pr.k - 1;
     const uint32_t smem = up.off_rpb + 2u * nrel * nrel * 4u + 1024;   // + 1024 bytes for aligning the base
     if ((int)smem > cap) return cudaSuccess;
