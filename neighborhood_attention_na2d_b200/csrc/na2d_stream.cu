@@ -261,20 +261,6 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
     return r;
 }
 
-// d = a * b + c on two fp32 lanes at once (packed f32x2 FMA).
-__device__ __forceinline__ void fma2(float &d0, float &d1, float a0, float a1, float b, float c0, float c1) {
-    asm("{\n .reg .b64 ra, rb, rc, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %4};\n mov.b64 rc, {%5, %6};\n"
-        " fma.rn.f32x2 rd, ra, rb, rc;\n mov.b64 {%0, %1}, rd;\n}\n"
-        : "=f"(d0), "=f"(d1)
-        : "f"(a0), "f"(a1), "f"(b), "f"(c0), "f"(c1));
-}
-// (a0 * b0, a1 * b1) on two fp32 lanes at once.
-__device__ __forceinline__ void mul2(float &d0, float &d1, float a0, float a1, float b0, float b1) {
-    asm("{\n .reg .b64 ra, rb, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n"
-        " mul.rn.f32x2 rd, ra, rb;\n mov.b64 {%0, %1}, rd;\n}\n"
-        : "=f"(d0), "=f"(d1)
-        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
-}
 
 __device__ __forceinline__ int clampi(int x, int lo, int hi) { return x < lo ? lo : (x > hi ? hi : x); }
 

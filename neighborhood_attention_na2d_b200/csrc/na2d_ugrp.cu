@@ -101,12 +101,19 @@ __device__ __forceinline__ void tmem_st8(uint32_t ta, const uint32_t *v) {
 // rounding of P), then r added to the exponent field.  Arguments below -125
 // (masked keys) give 2^-125, which rounds to zero in f16 and contributes
 // nothing measurable in bf16.
-__device__ __forceinline__ float ex2_fma(float x) {
-    x = fmaxf(x, -125.f);
-    const float xr = x + 12582912.f;   // 1.5 * 2^23: round(x) in the low mantissa bits
-    const float f = x - (xr - 12582912.f);
-    const float p = fmaf(fmaf(fmaf(0.05500755f, f, 0.24220777f), f, 0.69328272f), f, 1.f);
-    return __int_as_float(__float_as_int(p) + (__float_as_int(xr) << 23));
+// Two at a time with packed fp32x2 arithmetic.
+__device__ __forceinline__ void ex2_fma2(float &y0, float &y1, float x0, float x1) {
+    x0 = fmaxf(x0, -125.f);
+    x1 = fmaxf(x1, -125.f);
+    float xr0, xr1, r0, r1, f0, f1, p0, p1;
+    add2(xr0, xr1, x0, x1, 12582912.f, 12582912.f);   // 1.5 * 2^23: round(x) in the low mantissa bits
+    add2(r0, r1, xr0, xr1, -12582912.f, -12582912.f);
+    fma2(f0, f1, r0, r1, -1.f, x0, x1);                 // f = x - round(x)
+    fma2(p0, p1, f0, f1, 0.05500755f, 0.24220777f, 0.24220777f);
+    fma2v(p0, p1, p0, p1, f0, f1, 0.69328272f, 0.69328272f);
+    fma2v(p0, p1, p0, p1, f0, f1, 1.f, 1.f);
+    y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(xr0) << 23));
+    y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(xr1) << 23));
 }
 
 // ---------------------------------------------------------------------------
@@ -375,7 +382,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_ugrp_kernel(const __grid_cons
         // batches unrolled two deep (one deep at NKR = 12, where two spill registers)
         constexpr int kU = NKR == 12 ? 1 : 2;
         const float4 *tq = nullptr;
-        float mxr[kB], lr[kB];
+        float mxr[kB], lr[kB][2];
         // pass 1 over CNT key rows from i_first, scores at TMEM column col0 +
         // 16o: biased scores (log2 units) written back, running maxima.  No
         // branches: a row outside this query's window reads the table's
@@ -398,10 +405,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_ugrp_kernel(const __grid_cons
 #pragma unroll
                     for (int t = 0; t < 4; ++t) {
                         const float4 bb = br[t];
-                        y[4 * t + 0] = fmaf(y[4 * t + 0], c, bb.x);
-                        y[4 * t + 1] = fmaf(y[4 * t + 1], c, bb.y);
-                        y[4 * t + 2] = fmaf(y[4 * t + 2], c, bb.z);
-                        y[4 * t + 3] = fmaf(y[4 * t + 3], c, bb.w);
+                        fma2(y[4 * t + 0], y[4 * t + 1], y[4 * t + 0], y[4 * t + 1], c, bb.x, bb.y);
+                        fma2(y[4 * t + 2], y[4 * t + 3], y[4 * t + 2], y[4 * t + 3], c, bb.z, bb.w);
                     }
                     const float m0 = max3(max3(y[0], y[1], y[2]), max3(y[3], y[4], y[5]), max3(y[6], y[7], y[8]));
                     const float m1 = max3(max3(y[9], y[10], y[11]), max3(y[12], y[13], y[14]), y[15]);
@@ -414,9 +419,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_ugrp_kernel(const __grid_cons
             }
         };
         // pass 2 over CNT key rows, scores at scol0 + 16o, P (16-bit pairs)
-        // to pcol0 + 8o: exp2(score - max), columns 3, 7, 11 and 15 of a row
-        // on the FMA pipe, the rest on MUFU; one row-sum accumulator per row
-        // slot
+        // to pcol0 + 8o: exp2(score - max), columns 6, 7, 14 and 15 of a row
+        // on the FMA pipe, the rest on MUFU; row sums in two fp32 lanes per
+        // row slot
         auto pass2 = [&](uint32_t scol0, uint32_t pcol0, float mx, auto CNT) {
             constexpr int cnt = decltype(CNT)::value;
 #pragma unroll kU
@@ -432,9 +437,15 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_ugrp_kernel(const __grid_cons
                     uint32_t pk[8];
 #pragma unroll
                     for (int t = 0; t < 8; ++t) {
-                        const float x0 = x[r][2 * t] - mx, x1 = x[r][2 * t + 1] - mx;
-                        const float p0 = ex2(x0), p1 = (t & 1) ? ex2_fma(x1) : ex2(x1);
-                        lr[r] += p0 + p1;
+                        float x0, x1, p0, p1;
+                        fma2(x0, x1, x[r][2 * t], x[r][2 * t + 1], 1.f, -mx, -mx);
+                        if ((t & 3) == 3) {
+                            ex2_fma2(p0, p1, x0, x1);
+                        } else {
+                            p0 = ex2(x0);
+                            p1 = ex2(x1);
+                        }
+                        add2(lr[r][0], lr[r][1], lr[r][0], lr[r][1], p0, p1);
                         pk[t] = Pack2<T>::run(p0, p1);
                     }
                     tmem_st8(pcol0 + 8u * (uint32_t)(o0 + r), pk);
@@ -472,14 +483,14 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_ugrp_kernel(const __grid_cons
             // ---- pass 2: P of the upper rows over their own scores (P row o
             // at 8o overwrites scores of row o / 2 <= o, already read), then
             // P of the lower rows after them (over upper scores, all read)
-            lr[0] = lr[1] = 0.f;
+            lr[0][0] = lr[0][1] = lr[1][0] = lr[1][1] = 0.f;
             pass2(up, up, mx, std::integral_constant<int, NH>{});
             pass2(lo, up + 8u * NH, mx, std::integral_constant<int, NL>{});
             // ---- the previous unit's epilogue (its P.V completed while this
             // unit's scores were computed), before P_j is handed over: P.V_j
             // overwrites O_e only after the arrive below
             if (j > 0 && !epilogue(j - 1)) break;
-            l_prev = lr[0] + lr[1];
+            l_prev = (lr[0][0] + lr[0][1]) + (lr[1][0] + lr[1][1]);
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
