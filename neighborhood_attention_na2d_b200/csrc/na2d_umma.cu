@@ -333,19 +333,31 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_umma_kernel(const __grid_cons
                 float mx = -3.0e38f;
 #pragma unroll
                 for (int ky = 0; ky < KW; ++ky) {
-#pragma unroll
-                    for (int kx = 0; kx < KW; ++kx) s[ky * 8 + kx] += bias[ky * KW + kx];
-                    mx = max3(mx, max3(s[ky * 8 + 0], s[ky * 8 + 1], s[ky * 8 + 2]),
-                              max3(s[ky * 8 + 3], s[ky * 8 + 4], fmaxf(s[ky * 8 + 5], s[ky * 8 + 6])));
+                    // bias of columns 0-5 as three packed adds, column 6 alone
+                    float *r = s + ky * 8;
+                    const float *b = bias + ky * KW;
+                    add2(r[0], r[1], r[0], r[1], b[0], b[1]);
+                    add2(r[2], r[3], r[2], r[3], b[2], b[3]);
+                    add2(r[4], r[5], r[4], r[5], b[4], b[5]);
+                    r[6] += b[6];
+                    mx = max3(mx, max3(r[0], r[1], r[2]), max3(r[3], r[4], fmaxf(r[5], r[6])));
                 }
                 const float nm = -mx * c;
-                float l0 = 0.f, l1 = 0.f;
+                float l0 = 0.f, l1 = 0.f;   // two lanes of the row sum
                 uint32_t pk[32];
 #pragma unroll
                 for (int i = 0; i < 28; ++i) {
-                    const float p0 = ex2(fmaf(s[2 * i], c, nm));
-                    const float p1 = ((2 * i + 1) & 7) < KW ? ex2(fmaf(s[2 * i + 1], c, nm)) : 0.f;
-                    if (i & 1) l1 += p0 + p1; else l0 += p0 + p1;
+                    float p0, p1;
+                    if (((2 * i + 1) & 7) < KW) {
+                        float x0, x1;
+                        fma2(x0, x1, s[2 * i], s[2 * i + 1], c, nm, nm);
+                        p0 = ex2(x0);
+                        p1 = ex2(x1);
+                    } else {   // column 7 is a pad
+                        p0 = ex2(fmaf(s[2 * i], c, nm));
+                        p1 = 0.f;
+                    }
+                    add2(l0, l1, l0, l1, p0, p1);
                     pk[i] = Pack2<T>::run(p0, p1);
                 }
 #pragma unroll
