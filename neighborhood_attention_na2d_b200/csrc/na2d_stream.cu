@@ -84,7 +84,7 @@ struct StreamParams {
     const unsigned char *q, *k, *v;
     unsigned char *out;
     const void *rpb;
-    int H, W, heads;
+    int H, W, heads, B;
     // byte strides (batch, head, row, pixel) of q, k, v (one set: the three
     // views of one tensor or three contiguous tensors) and of out
     int64_t in_sb, in_sh, in_sy, in_sx;
@@ -280,8 +280,12 @@ __device__ __forceinline__ int pair_halo(int pair, int H) { return min(win_start
 // continues after the last ring row of the previous one.  Producer and
 // consumers run the same walk.  Only the image, the step's pairs and the ring
 // row of the step's first key row are kept; the rest is recomputed.
+// Images are walked head-major (image index h * B + b, then the column band),
+// so that a CTA's consecutive images share their head and its bias rows: with
+// maps of a few pair-steps each (14 x 14), a batch-major walk would change
+// the head, and rewrite the bias, at every step.
 struct SlideWalk {
-    int bh;           // image (a column band of one (batch, head) map when nb > 1)
+    int bh;           // image (a column band of one (head, batch) map when nb > 1)
     int pa, pe;       // the step's first pair and one past its last
     int ge;           // end of the CTA's range (global pair index)
     int h;            // head of image bh
@@ -300,8 +304,8 @@ struct SlideWalk {
         pe = step_end(p);
         const int map = bh / p.nb;
         band = bh - map * p.nb;
-        h = map % p.heads;
-        b = map / p.heads;
+        b = map % p.B;
+        h = map / p.B;
         ring_lo = 0;
     }
     // byte offset of image (b, h) for the given batch / head strides
@@ -318,9 +322,9 @@ struct SlideWalk {
             ++bh;
             if (++band == p.nb) {
                 band = 0;
-                if (++h == p.heads) {
-                    h = 0;
-                    ++b;
+                if (++b == p.B) {
+                    b = 0;
+                    ++h;
                 }
             }
             pa = 0;
@@ -1140,7 +1144,7 @@ cudaError_t launch_stream_impl(const Problem &pr, const View &q, const View &k, 
     if (pr.W > 64 && !sp.rows_contiguous) return cudaSuccess;   // bands copy contiguous row segments
     const long long lim = stream_wait_limit();
     sp.wait_limit = lim > 0 ? lim : kWaitLimit;
-    sp.H = pr.H; sp.W = pr.W; sp.heads = pr.heads;
+    sp.H = pr.H; sp.W = pr.W; sp.heads = pr.heads; sp.B = pr.B;
     sp.c_log2 = kLog2e / std::sqrt((float)pr.D);
     sp.sqrt_d = std::sqrt((float)pr.D);
     // NAT_NWC consumer warps (SP query-row pairs of MX column spans each)
