@@ -19,25 +19,29 @@
 // swizzled: slot 16 * row + col is tile row 16 * row + col.  Strip e (group
 // rows 8e .. 8e + 7) is the M = 128 tile of Q rows 128e .. 128e + 127; its
 // keys are the group rows kr0[e] .. kr0[e] + NKR - 1 (tile rows from
-// 16 kr0[e]).
-//   1. S_e = Q_e K_e^T: two tcgen05.mma (K = 16 each, both operands K-major
-//      in shared memory), N = 16 NKR, fp32 in tensor memory (TMEM).
-//   2. softmax: one thread per query (its TMEM lane).  Scores are scaled and
-//      biased from a shared-memory table that holds, per query column and
-//      relative key row, the 16 bias values of a key row in log2 units with
-//      the window mask folded in (-1e30 outside the window).  Pass 1 writes
-//      the biased scores back and takes their maximum; pass 2 exponentiates
-//      and writes P as 16-bit pairs over the first 8 NKR columns of S_e.  Key
-//      rows in no window of the warp's queries are skipped (P = 0).
-//   3. O_e = P_e V_e: NKR tcgen05.mma (K = 16 keys = one key row each, A = P
-//      in TMEM, B = V MN-major in shared memory).
+// 16 kr0[e]), split into a lower and an upper half of key rows.
+//   1. S = Q K^T per half: two tcgen05.mma (K = 16 each, both operands
+//      K-major in shared memory), N = 16 rows of the half, fp32 in tensor
+//      memory (TMEM).
+//   2. softmax: one thread per query (its TMEM lane), packed fp32x2
+//      arithmetic.  Scores are scaled and biased from a shared-memory table
+//      that holds, per query column and relative key row, the 16 bias values
+//      of a key row in log2 units with the window mask folded in (-1e30
+//      outside the window; a key row outside the query's window reads an
+//      all-masked row, so every row is processed without branches).  Pass 1
+//      writes the biased scores back and takes their maximum; pass 2
+//      exponentiates (a quarter of the columns on the FMA pipe) and writes P
+//      as 16-bit pairs over the upper half's scores.
+//   3. O = P V: NKR tcgen05.mma (K = 16 keys = one key row each, A = P in
+//      TMEM, B = V MN-major in shared memory).
 //   4. epilogue: the same thread loads its O row, divides by its row sum and
-//      stores 64 bytes.
-// Warpgroup e (warps 4e .. 4e + 3) runs strip e of every unit, with S_e at
-// TMEM columns e N and O_e at 2N + 32e.  Warp 8, lane 0 issues the TMA copies
-// into a ring of NSTG stages; warps 9 and 10, lane 0, issue the MMAs of strip
-// 0 and strip 1 (each unit's P.V, then the next unit's Q K^T) and signal
-// completion with tcgen05.commit on mbarriers; warp 9 owns the TMEM
+//      stores 64 bytes; it runs after the next unit's softmax.
+// Warpgroup e (warps 4e .. 4e + 3) runs strip e of every unit, with two TMEM
+// score regions of 16 ceil(NKR / 2) columns and an O buffer of 32 columns.
+// Warp 8, lane 0 issues the TMA copies into a ring of NSTG stages; warps 9
+// and 10, lane 0, issue the MMAs of strip 0 and strip 1 (the next unit's
+// upper-half Q K^T, this unit's P.V, the next unit's lower-half Q K^T) and
+// signal completion with tcgen05.commit on mbarriers; warp 9 owns the TMEM
 // allocation.  Every wait is bounded: one that runs out counts the event,
 // raises the block's abort flag, and the block winds down (its MMAs and
 // copies in flight are waited for before TMEM and shared memory are
