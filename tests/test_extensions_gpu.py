@@ -205,18 +205,24 @@ def test_forward_ex_contiguous_takes_the_fast_kernels():
 
 
 # ---------------------------------------------------------------------------
-STRIDED = ["fused_qkv", "channels_last", "padded_rows"]
+# (layout, W, the kernel that must run): at W <= 64 the streaming kernel takes
+# all three layouts (rows copied as 16-byte pieces when they are strided);
+# above 64 columns its column bands copy rows of densely packed images only,
+# so these views take the generic kernel
+STRIDED = [("fused_qkv", 20, "fwd_stream_kernel"), ("channels_last", 20, "fwd_stream_kernel"),
+           ("padded_rows", 20, "fwd_stream_kernel"), ("padded_rows", 72, "fwd_simt_kernel"),
+           ("fused_qkv", 72, "fwd_simt_kernel"), ("channels_last", 72, "fwd_simt_kernel")]
 
 
-@pytest.mark.parametrize("layout", STRIDED)
-def test_stream_kernel_strided_rows(layout):
-    """The k = 7 sliding-window kernel on q, k, v views whose rows are not
+@pytest.mark.parametrize("layout,W,kernel", STRIDED)
+def test_stream_kernel_strided_rows(layout, W, kernel):
+    """The k = 7 sliding-window forward on q, k, v views whose rows are not
     contiguous: the three views of a fused (B, H, W, 3 heads D) buffer,
     channels-last (B, H, W, heads D) tensors, and [B, heads, H, W, D] slices
-    of tensors with two spare pixels per row.  The producer warp copies such
-    rows as 16-byte pieces; the output equals the oracle."""
-    B, heads, H, W, D, k, d = 2, 2, 14, 20, 32, 7, 1
-    shape = Shape(B, heads, H, W, D, k, d, "f16", 1500)
+    of tensors with two spare pixels per row; the kernel that runs is the
+    one the dispatch promises, and the output equals the oracle."""
+    B, heads, H, D, k, d = 2, 2, 14, 32, 7, 1
+    shape = Shape(B, heads, H, W, D, k, d, "f16", 1500 + W)
     q, kk, v, rpb = make_inputs(shape)
     if layout == "fused_qkv":
         qkv = torch.cat([t.permute(0, 2, 3, 1, 4).reshape(B, H, W, heads * D) for t in (q, kk, v)], dim=-1).cuda()
@@ -232,6 +238,6 @@ def test_stream_kernel_strided_rows(layout):
     out = torch.full((B, heads, H, W, D), float("nan"), dtype=q.dtype, device="cuda")
     na.na2d_forward_ex(qd, kd, vd, rpb.cuda(), k, d, out=out)
     torch.cuda.synchronize()
-    assert na.na2d_last_kernel() == "fwd_stream_kernel"
+    assert na.na2d_last_kernel() == kernel
     want = oracle.forward(f64(q), f64(kk), f64(v), f64(rpb), k, d)
     assert max_err(f64(out), want) <= TOL["f16"]
