@@ -56,15 +56,17 @@ enum Mode : int { kGeneric = 0, kFull = 1, kFullTma = 3, kDenseTma = 4 };
 
 // Per-k warp tile: TQY x TQX queries (16), halo NKR = TQY + K - 1 rows by NKC
 // columns (padded to a multiple of 8), processed in chunks of CH 8-key tiles;
-// at most TILES warp tiles per block in FULL mode.
+// at most TILES warp tiles per block in FULL mode: 8, one per warp of the
+// block (with 4 at k >= 9, half the warps idled through every block's tiles;
+// the two stages of 8 tiles still fit, 219 KB at k = 13).
 template <int K> struct Cfg;
 // TILES_TMA: warp tiles per block on the TMA path (k <= 7 only).
 template <> struct Cfg<3> { static constexpr int TQY = 4, TQX = 4, NKC = 8, CH = 6, TILES = 8, TILES_TMA = 7; };
 template <> struct Cfg<5> { static constexpr int TQY = 4, TQX = 4, NKC = 8, CH = 8, TILES = 8, TILES_TMA = 7; };
 template <> struct Cfg<7> { static constexpr int TQY = 8, TQX = 2, NKC = 8, CH = 14, TILES = 8, TILES_TMA = 7; };
-template <> struct Cfg<9> { static constexpr int TQY = 2, TQX = 8, NKC = 16, CH = 10, TILES = 4, TILES_TMA = 0; };
-template <> struct Cfg<11> { static constexpr int TQY = 4, TQX = 4, NKC = 16, CH = 14, TILES = 4, TILES_TMA = 0; };
-template <> struct Cfg<13> { static constexpr int TQY = 4, TQX = 4, NKC = 16, CH = 16, TILES = 4, TILES_TMA = 0; };
+template <> struct Cfg<9> { static constexpr int TQY = 2, TQX = 8, NKC = 16, CH = 10, TILES = 8, TILES_TMA = 0; };
+template <> struct Cfg<11> { static constexpr int TQY = 4, TQX = 4, NKC = 16, CH = 14, TILES = 8, TILES_TMA = 0; };
+template <> struct Cfg<13> { static constexpr int TQY = 4, TQX = 4, NKC = 16, CH = 16, TILES = 8, TILES_TMA = 0; };
 
 constexpr int cround(int x, int m) { return (x + m - 1) / m * m; }
 
