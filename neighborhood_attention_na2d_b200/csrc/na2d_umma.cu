@@ -273,6 +273,33 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_umma_kernel(const __grid_cons
         int cur_h = -1;
         float l_prev = 1.f;
         // O of unit jj (ready once its P.V completed) / row sum -> 64 bytes
+        // Position of this thread's group in unit j (g = 2 (u_begin + j) + e):
+        // plane bh, head h, group row gy and column gx.  A warpgroup's units are
+        // two apart, four groups, so the position advances by carries instead
+        // of divisions (prev: the position two units back, whose output is
+        // written after this unit's softmax).
+        struct GPos {
+            int g, bh, h, gy, gx;
+        };
+        GPos pos;
+        pos.g = 2 * (u_begin + w) + e;
+        pos.bh = pos.g / dd;
+        pos.h = pos.bh % p.heads;
+        pos.gy = (pos.g - pos.bh * dd) / p.d;
+        pos.gx = pos.g - pos.bh * dd - pos.gy * p.d;
+        GPos prev = pos;
+        auto advance = [&](GPos &x) {
+            x.g += 4;
+            x.gx += 4;
+            while (x.gx >= p.d) {
+                x.gx -= p.d;
+                if (++x.gy == p.d) {
+                    x.gy = 0;
+                    ++x.bh;
+                    if (++x.h == p.heads) x.h = 0;
+                }
+            }
+        };
         auto epilogue_store = [&](int jj) -> bool {
             const bool ok = mb_wait(bar_o + 8 * (jj & 3), (uint32_t)((jj >> 2) & 1));
             if (!__all_sync(0xffffffffu, ok)) {
@@ -286,13 +313,12 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_umma_kernel(const __grid_cons
             float o[32];
             tmem_ld32(tl + 256u + (uint32_t)(jj & 3) * 32, o);
             tmem_ld_wait();
-            const int g = 2 * (u_begin + jj) + e;
-            if (g < p.GU && qok) {
+            if (prev.g < p.GU && qok) {   // prev: unit jj's position
                 float inv;
                 asm("rcp.approx.ftz.f32 %0, %1;\n" : "=f"(inv) : "f"(l_prev));
-                const int bh = g / dd, rem = g - bh * dd, gy = rem / p.d, gx = rem - gy * p.d;
                 uint4 *dst = reinterpret_cast<uint4 *>(
-                    p.out + ((((size_t)bh * p.H + gy + (size_t)p.d * qy) * p.W) + gx + (size_t)p.d * qx) * 64);
+                    p.out + ((((size_t)prev.bh * p.H + prev.gy + (size_t)p.d * qy) * p.W) + prev.gx + (size_t)p.d * qx) *
+                                64);
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
                     dst[i] = make_uint4(Pack2<T>::run(o[8 * i + 0] * inv, o[8 * i + 1] * inv),
@@ -302,10 +328,11 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_umma_kernel(const __grid_cons
             }
             return true;
         };
-        for (int j = w;; j += 2) {
+        for (int j = w;; j += 2, prev = pos, advance(pos)) {
             if (j < nst) {
-                const int g = 2 * (u_begin + j) + e;
-                const int h = (min(g, p.GU - 1) / dd) % p.heads;
+                // (a group past the last one, of an odd count, takes the head
+                // that follows; its outputs are not stored)
+                const int h = pos.h;
                 if (h != cur_h) {
                     cur_h = h;
                     // bias of key (ky, kx): table row ky - qy + 6, column kx - qx + 6
