@@ -352,8 +352,28 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_ugrp_kernel(const __grid_cons
         const int nrel = 2 * k - 1;
 
         float l_prev = 1.f;   // row sum of the unit whose output is pending
-        // O of unit jj (ready once its P.V completed) / row sum -> 64 bytes
-        auto epilogue = [&](int jj) -> bool {
+        // Position of unit j's group (plane bh, group row gy and column gx),
+        // advanced by one group per unit by carries instead of divisions.
+        struct GPos {
+            int bh, gy, gx;
+        };
+        GPos pos;
+        pos.bh = u_begin / dd;
+        pos.gy = (u_begin - pos.bh * dd) / p.d;
+        pos.gx = u_begin - pos.bh * dd - pos.gy * p.d;
+        GPos prev = pos;
+        auto advance = [&](GPos &x) {
+            if (++x.gx == p.d) {
+                x.gx = 0;
+                if (++x.gy == p.d) {
+                    x.gy = 0;
+                    ++x.bh;
+                }
+            }
+        };
+        // O of unit jj (ready once its P.V completed) / row sum -> 64 bytes;
+        // at is unit jj's position
+        auto epilogue = [&](int jj, const GPos &at) -> bool {
             const bool oko = mb_wait(bar_o + 8 * e, (uint32_t)(jj & 1), p.wait_limit);
             if (!__all_sync(0xffffffffu, oko)) {
                 if (lane == 0) {
@@ -369,10 +389,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_ugrp_kernel(const __grid_cons
             if (qok) {
                 float inv;
                 asm("rcp.approx.ftz.f32 %0, %1;\n" : "=f"(inv) : "f"(l_prev));
-                const int g = u_begin + jj;
-                const int bh = g / dd, rem = g - bh * dd, gy = rem / p.d, gx = rem - gy * p.d;
                 uint4 *dst = reinterpret_cast<uint4 *>(
-                    p.out + ((((size_t)bh * p.H + gy + (size_t)p.d * row) * p.W) + gx + (size_t)p.d * qc) * 64);
+                    p.out + ((((size_t)at.bh * p.H + at.gy + (size_t)p.d * row) * p.W) + at.gx + (size_t)p.d * qc) * 64);
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
                     dst[i] = make_uint4(Pack2<T>::run(o[8 * i + 0] * inv, o[8 * i + 1] * inv),
@@ -383,8 +401,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_ugrp_kernel(const __grid_cons
             return true;
         };
         constexpr int kB = 2;   // key rows per wait for the TMEM loads
-        // batches unrolled two deep (one deep at NKR = 12, where two spill registers)
-        constexpr int kU = NKR == 12 ? 1 : 2;
+        // batches unrolled two deep (one deep at NKR = 11 and 12, where two spill registers)
+        constexpr int kU = (NKR == 11 || NKR == 12) ? 1 : 2;
         const float4 *tq = nullptr;
         float mxr[kB], lr[kB][2];
         // pass 1 over CNT key rows from i_first, scores at TMEM column col0 +
@@ -469,10 +487,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_ugrp_kernel(const __grid_cons
             tc_fence_after();
             return true;
         };
-        for (int j = 0; j < nst; ++j) {
-            const int g = u_begin + j;
-            const int bh = g / dd;
-            tq = reinterpret_cast<const float4 *>(tab_q + (uint32_t)(bh - bh_first) * p.tab_bytes);
+        for (int j = 0; j < nst; ++j, prev = pos, advance(pos)) {
+            tq = reinterpret_cast<const float4 *>(tab_q + (uint32_t)(pos.bh - bh_first) * p.tab_bytes);
             // region of the upper scores (and of P), region of the lower scores
             const uint32_t up = tR + (uint32_t)((j & 1) * HS), lo = tR + (uint32_t)((1 - (j & 1)) * HS);
             // ---- pass 1: the upper rows as soon as their scores land (the
@@ -493,13 +509,13 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_ugrp_kernel(const __grid_cons
             // ---- the previous unit's epilogue (its P.V completed while this
             // unit's scores were computed), before P_j is handed over: P.V_j
             // overwrites O_e only after the arrive below
-            if (j > 0 && !epilogue(j - 1)) break;
+            if (j > 0 && !epilogue(j - 1, prev)) break;
             l_prev = (lr[0][0] + lr[0][1]) + (lr[1][0] + lr[1][1]);
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mb_arrive(bar_p + 8 * e);
-            if (j == nst - 1) epilogue(j);
+            if (j == nst - 1) epilogue(j, pos);
         }
     }
     // ---- teardown: TMEM released by the warp that took it, after every
