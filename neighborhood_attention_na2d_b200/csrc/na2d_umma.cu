@@ -19,23 +19,26 @@
 //      diagonal 64 x 64 blocks (a query and a key of the same group) are used.
 //   2. softmax: one thread per tile row (its TMEM lane) loads its 56 scores,
 //      adds the bias (pre-multiplied by sqrt(D), kept in registers per head),
-//      exponentiates in fp32 and writes P as 16-bit pairs over its own S
-//      columns: 32 columns for its group's 64 keys and 32 columns of zeros for
-//      the other group's keys.
+//      exponentiates in fp32 and writes P as 16-bit pairs into its
+//      warpgroup's P columns: 32 columns for its group's 64 keys; the other
+//      group's 32 columns hold zeros, written once before the first unit.
 //   3. O = P V: eight tcgen05.mma with A = P in TMEM and B = V (MN-major in
 //      shared memory), O = [128 x 32] fp32 in TMEM.
 //   4. epilogue: the same thread loads its O row, divides by its row sum and
 //      stores 64 bytes.
 // Warps 0-3 and 4-7 are two softmax warpgroups taking alternate units, each
-// with its own S / P columns (TMEM columns 0-127 / 128-255); O rotates over
-// four 32-column buffers (256-383).  A warpgroup runs the softmax of its
-// unit j and then the epilogue of its unit j - 2, so it never waits for a
-// P.V that was just issued, and one warpgroup's softmax overlaps the other's
-// MMAs and epilogue.  Warp 8, lane 0 issues the TMA copies into a ring of
-// NSTG stages; warps 9 and 10, lane 0, issue the MMAs of the even and the
-// odd units (each unit's P.V before the Q K^T two units ahead, so a P.V
-// never waits for a copy) and signal completion with tcgen05.commit on
-// mbarriers; warp 9 owns the TMEM allocation.  Every wait is bounded: one that runs out counts the event,
+// with its own S columns (TMEM columns 0-127 / 128-255) and P columns
+// (256-319 / 320-383); O rotates over four 32-column buffers (384-511).  A
+// warpgroup runs the softmax of its unit j and then the epilogue of its unit
+// j - 2, so it never waits for a P.V that was just issued, and one
+// warpgroup's softmax overlaps the other's MMAs and epilogue.  Warp 8, lane 0
+// issues the TMA copies into a ring of NSTG stages; warps 9 and 10, lane 0,
+// issue the MMAs of the even and the odd units and signal completion with
+// tcgen05.commit on mbarriers: once unit j's P is handed over, the Q K^T two
+// units ahead goes first (its S columns are free, so the warpgroup's next
+// scores are not queued behind this P.V), then unit j's P.V.  Before a
+// warpgroup rewrites P it waits for the P.V two units back, which read it.
+// Warp 9 owns the TMEM allocation.  Every wait is bounded: one that runs out counts the event,
 // raises the block's abort flag, and the block winds down (its MMAs and
 // copies in flight are waited for before TMEM and shared memory are
 // released).
@@ -233,9 +236,15 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_umma_kernel(const __grid_cons
                     break;
                 }
                 tc_fence_after();
+                // the next unit's scores first (its S buffer was read before
+                // P_j was handed over), then P_j V_j
+                if (j + 2 < nst && !issue_qk(j + 2)) {
+                    ok = false;
+                    break;
+                }
                 const uint32_t vt = sbase + (uint32_t)s * kStage + 2 * kTile;
-                const uint32_t dO = tmem + 256u + (uint32_t)(j & 3) * 32;
-                const uint32_t aP = tmem + (uint32_t)b * 128;
+                const uint32_t dO = tmem + 384u + (uint32_t)(j & 3) * 32;
+                const uint32_t aP = tmem + 256u + (uint32_t)b * 64;
                 // V MN-major: 64-byte rows of 32 channels, 8-key groups 512
                 // bytes apart; k-step t takes keys 16t .. 16t + 15
 #pragma unroll
@@ -243,7 +252,6 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_umma_kernel(const __grid_cons
                     umma_ts(dO, aP + 8u * t, sw64_desc(vt + 1024u * t, 16, 512), idesc_pv, t > 0 ? 1u : 0u);
                 umma_commit(bar_o + 8 * (j & 3));
                 umma_commit(bar_empty + 8 * s);
-                if (j + 2 < nst && !issue_qk(j + 2)) ok = false;
             }
             if (!ok) {
                 atomicAdd(&g_umma_timeouts, 1u);
@@ -267,7 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_umma_kernel(const __grid_cons
         const int qyc = min(qy, KW - 1), qxc = min(qx, KW - 1);
         const uint32_t tl = tmem + ((uint32_t)(32 * q4) << 16);
         const uint32_t tS = tl + (uint32_t)w * 128 + (uint32_t)e * 64;
-        const uint32_t tP = tl + (uint32_t)w * 128;
+        const uint32_t tP = tl + 256u + (uint32_t)w * 64;   // P of this warpgroup's units
         const float c = p.c_log2;
         float bias[KW * KW];
         int cur_h = -1;
@@ -311,7 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_umma_kernel(const __grid_cons
             }
             tc_fence_after();
             float o[32];
-            tmem_ld32(tl + 256u + (uint32_t)(jj & 3) * 32, o);
+            tmem_ld32(tl + 384u + (uint32_t)(jj & 3) * 32, o);
             tmem_ld_wait();
             if (prev.g < p.GU && qok) {   // prev: unit jj's position
                 float inv;
@@ -328,6 +336,14 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_umma_kernel(const __grid_cons
             }
             return true;
         };
+        {   // the other group's P columns of this thread's lane: zeros, once
+            uint32_t zero[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) zero[i] = 0u;
+            tmem_st16(tP + (uint32_t)(e ^ 1) * 32, zero);
+            tmem_st16(tP + (uint32_t)(e ^ 1) * 32 + 16, zero);
+            tmem_st_wait();
+        }
         for (int j = w;; j += 2, prev = pos, advance(pos)) {
             if (j < nst) {
                 // (a group past the last one, of an odd count, takes the head
@@ -389,14 +405,23 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_umma_kernel(const __grid_cons
                 }
 #pragma unroll
                 for (int i = 28; i < 32; ++i) pk[i] = 0u;
-                uint32_t zero[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) zero[i] = 0u;
-                // own group's keys: P columns 32e .. 32e + 31; the other group's: zeros
+                // P of unit j - 2 has been read by its P.V before it is
+                // overwritten (that P.V completed long ago; bounded wait)
+                if (j >= 2) {
+                    const bool okp = mb_wait(bar_o + 8 * ((j - 2) & 3), (uint32_t)(((j - 2) >> 2) & 1));
+                    if (!__all_sync(0xffffffffu, okp)) {
+                        if (lane == 0) {
+                            atomicAdd(&g_umma_timeouts, 1u);
+                            *abort_flag = 1;
+                        }
+                        break;
+                    }
+                    tc_fence_after();
+                }
+                // own group's keys: P columns 32e .. 32e + 31 (the other
+                // group's columns hold the zeros written before the loop)
                 tmem_st16(tP + (uint32_t)e * 32, pk);
                 tmem_st16(tP + (uint32_t)e * 32 + 16, pk + 16);
-                tmem_st16(tP + (uint32_t)(e ^ 1) * 32, zero);
-                tmem_st16(tP + (uint32_t)(e ^ 1) * 32 + 16, zero);
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
