@@ -165,6 +165,29 @@ template <> struct Pack2<__nv_bfloat16> {
     }
 };
 
+// One output pixel of D = 32 channels (64 bytes): o scaled by inv, packed to
+// 16-bit pairs.  With st32 (the pixel is 32-byte aligned) as two 32-byte
+// stores, else four 16-byte ones; a warp's pixels lie in different lines
+// (they are d pixels apart), so the wider stores halve the store wavefronts.
+template <typename T>
+__device__ __forceinline__ void store_pixel64(unsigned char *dst, const float (&o)[32], float inv, bool st32) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) pk[i] = Pack2<T>::run(o[2 * i] * inv, o[2 * i + 1] * inv);
+    if (st32) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+            asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};\n" ::"l"(dst + 32 * h),
+                         "r"(pk[8 * h]), "r"(pk[8 * h + 1]), "r"(pk[8 * h + 2]), "r"(pk[8 * h + 3]), "r"(pk[8 * h + 4]),
+                         "r"(pk[8 * h + 5]), "r"(pk[8 * h + 6]), "r"(pk[8 * h + 7])
+                         : "memory");
+    } else {
+        uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+    }
+}
+
 __device__ __forceinline__ float max3(float a, float b, float c) {
     float r;
     asm("max.f32 %0, %1, %2, %3;\n" : "=f"(r) : "f"(a), "f"(b), "f"(c));

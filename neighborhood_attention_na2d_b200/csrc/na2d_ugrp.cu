@@ -348,6 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_ugrp_kernel(const __grid_cons
         const uint32_t tl = tmem + ((uint32_t)(32 * q4) << 16);
         const uint32_t tR = tl + (uint32_t)(e * 2 * HS), tO = tl + (uint32_t)(4 * HS + 32 * e);
         const float c = p.c_log2;
+        const bool st32 = (reinterpret_cast<uintptr_t>(p.out) & 31u) == 0;
         const unsigned char *tab_q = smem + p.off_tab + (uint32_t)qc * p.qstride;
         const int nrel = 2 * k - 1;
 
@@ -389,14 +390,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_ugrp_kernel(const __grid_cons
             if (qok) {
                 float inv;
                 asm("rcp.approx.ftz.f32 %0, %1;\n" : "=f"(inv) : "f"(l_prev));
-                uint4 *dst = reinterpret_cast<uint4 *>(
-                    p.out + ((((size_t)at.bh * p.H + at.gy + (size_t)p.d * row) * p.W) + at.gx + (size_t)p.d * qc) * 64);
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    dst[i] = make_uint4(Pack2<T>::run(o[8 * i + 0] * inv, o[8 * i + 1] * inv),
-                                        Pack2<T>::run(o[8 * i + 2] * inv, o[8 * i + 3] * inv),
-                                        Pack2<T>::run(o[8 * i + 4] * inv, o[8 * i + 5] * inv),
-                                        Pack2<T>::run(o[8 * i + 6] * inv, o[8 * i + 7] * inv));
+                store_pixel64<T>(
+                    p.out + ((((size_t)at.bh * p.H + at.gy + (size_t)p.d * row) * p.W) + at.gx + (size_t)p.d * qc) * 64,
+                    o, inv, st32);
             }
             return true;
         };

@@ -277,6 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_umma_kernel(const __grid_cons
         const uint32_t tS = tl + (uint32_t)w * 128 + (uint32_t)e * 64;
         const uint32_t tP = tl + 256u + (uint32_t)w * 64;   // P of this warpgroup's units
         const float c = p.c_log2;
+        const bool st32 = (reinterpret_cast<uintptr_t>(p.out) & 31u) == 0;
         float bias[KW * KW];
         int cur_h = -1;
         float l_prev = 1.f;
@@ -324,15 +325,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_umma_kernel(const __grid_cons
             if (prev.g < p.GU && qok) {   // prev: unit jj's position
                 float inv;
                 asm("rcp.approx.ftz.f32 %0, %1;\n" : "=f"(inv) : "f"(l_prev));
-                uint4 *dst = reinterpret_cast<uint4 *>(
-                    p.out + ((((size_t)prev.bh * p.H + prev.gy + (size_t)p.d * qy) * p.W) + prev.gx + (size_t)p.d * qx) *
-                                64);
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    dst[i] = make_uint4(Pack2<T>::run(o[8 * i + 0] * inv, o[8 * i + 1] * inv),
-                                        Pack2<T>::run(o[8 * i + 2] * inv, o[8 * i + 3] * inv),
-                                        Pack2<T>::run(o[8 * i + 4] * inv, o[8 * i + 5] * inv),
-                                        Pack2<T>::run(o[8 * i + 6] * inv, o[8 * i + 7] * inv));
+                store_pixel64<T>(
+                    p.out + ((((size_t)prev.bh * p.H + prev.gy + (size_t)p.d * qy) * p.W) + prev.gx + (size_t)p.d * qx) * 64,
+                    o, inv, st32);
             }
             return true;
         };
