@@ -239,6 +239,30 @@ def test_side_stream_and_determinism():
     assert torch.equal(a, b)
 
 
+@pytest.mark.parametrize("shape,kernel", [
+    (Shape(2, 2, 56, 56, 32, 7, 8, "bf16", 7401), "fwd_umma_kernel"),
+    (Shape(1, 2, 32, 32, 32, 13, 2, "f16", 7402), "fwd_ugrp_kernel"),
+    (Shape(2, 2, 28, 28, 32, 7, 1, "bf16", 7403), "fwd_stream_kernel"),
+], ids=lambda x: x.describe() if isinstance(x, Shape) else x)
+def test_output_only_16_byte_aligned(shape, kernel):
+    """An output that starts 16 bytes past a 32-byte boundary takes the kernels'
+    16-byte store path; every element still matches the oracle and nothing is
+    written outside the output."""
+    q, k, v, rpb = make_inputs(shape)
+    n, pad = q.numel(), 8   # 8 16-bit elements: 16 bytes
+    buf = torch.full((n + 2 * PAD,), SENTINEL, dtype=q.dtype, device="cuda")
+    out = buf[PAD + pad:PAD + pad + n].view(q.shape)
+    assert out.data_ptr() % 32 == 16
+    na.na2d_forward(q.cuda(), k.cuda(), v.cuda(), rpb.cuda(), shape.k, shape.d, out=out)
+    torch.cuda.synchronize()
+    assert na.na2d_last_kernel() == kernel
+    edge = torch.cat([buf[:PAD + pad], buf[PAD + pad + n:]]).float()
+    assert bool((edge == float(torch.tensor(SENTINEL, dtype=buf.dtype).float())).all()), "write outside the output"
+    want = oracle.forward(f64(q), f64(k), f64(v), f64(rpb), shape.k, shape.d)
+    err = max_err(out.double().cpu().numpy(), want)
+    assert err <= TOL[shape.dtype], f"{shape.describe()}: max abs err {err}"
+
+
 def test_misaligned_tensor_is_rejected():
     q = torch.zeros(2 * 14 * 14 * 32 + 4, dtype=torch.float16, device="cuda")[4:].view(1, 2, 14, 14, 32)
     with pytest.raises(na.Na2dError) as e:
