@@ -30,3 +30,24 @@ def test_roofline_picks_the_slower_limit():
     r = bench.roofline(wl, 0.010, None)
     assert r["bound"] == "hbm" and r["t_hbm_us"] > r["t_tensor_us"]
     assert abs(r["achieved"] - wl.shapes[0].algorithmic_bytes() / 1e-5 / 1e9) < 1e-6 * r["achieved"]
+
+
+def _profile_summaries():
+    out = []
+    for f in sorted(bench.PROFILES.glob("*.md")):
+        kernel = next((k for k in bench.KERNEL_SOURCES if f.stem.startswith(k + "_")), None)
+        if kernel is not None:
+            out.append((kernel, f.stem[len(kernel) + 1:]))
+    return out
+
+
+@pytest.mark.parametrize("kernel,workload", _profile_summaries(), ids=lambda x: x)
+def test_committed_profile_matches_the_kernel_source(kernel, workload):
+    """Every committed ncu summary that records a traffic figure was taken on
+    the current source of its kernel, so the bench line reports it (a kernel
+    change without a new capture would turn the line's traffic to null)."""
+    text = (bench.PROFILES / f"{kernel}_{workload}.md").read_text()
+    if "traffic_per_launch_bytes" not in text:
+        pytest.skip("summary without a traffic figure")
+    assert bench.recorded_traffic(kernel, workload) is not None, \
+        f"{kernel}_{workload}.md was captured on another source (sha now {bench.kernel_sha(kernel)})"
