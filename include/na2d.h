@@ -32,7 +32,8 @@
  *     attn         : [B, heads, H, W, k*k] fp32 (split path only)
  *
  * Ownership and threading: every buffer is a DEVICE pointer owned by the
- * caller.  The library allocates no memory and keeps no per-call state; calls
+ * caller (na2d_forward_host alone takes host buffers and a device
+ * workspace).  The library allocates no memory and keeps no per-call state; calls
  * are asynchronous on `stream` (a cudaStream_t; NULL means the legacy default
  * stream) and never synchronise the host.  Calls from several host threads
  * are safe.  Outputs must not overlap inputs.
@@ -125,6 +126,38 @@ NA2D_API na2d_status na2d_av(const na2d_problem *p, const float *attn, const voi
  * (dilated) window, in one kernel; no k*k tensor is written to memory. */
 NA2D_API na2d_status na2d_forward(const na2d_problem *p, const void *q, const void *k, const void *v,
                          const void *rpb, void *out, void *stream);
+
+/* Bytes of device workspace na2d_forward_host needs for problem p (two chunk
+ * slots of q, k, v and out, plus the bias table; see na2d_forward_host).
+ * Writes 0 for an empty problem.  Host-only; launches nothing. */
+NA2D_API na2d_status na2d_forward_host_workspace_size(const na2d_problem *p, size_t *bytes);
+
+/* na2d_forward on HOST buffers: the call a program makes when its tensors
+ * live in host memory.  q, k, v, out: [B,heads,H,W,D] and rpb
+ * [heads,2k-1,2k-1] (or NULL) in host memory, in the problem's dtype; they
+ * should be page-locked (cudaHostAlloc / pinned), or the copies run
+ * synchronously.  The batch is cut into at most 8 chunks of equal size (the
+ * last one shorter); chunk i is copied host -> device into workspace slot
+ * i % 2, computed by na2d_forward on the caller's stream, and copied back,
+ * so that the copy in of one chunk, the forward of the next and the copy
+ * out of a third overlap (two copy directions and the kernels run at once).
+ * workspace: a caller-owned device buffer of at least
+ * na2d_forward_host_workspace_size() bytes, 16-byte aligned (256-byte
+ * aligned lets the kernels use their widest stores), scratch afterwards.
+ * Ordering: the call's work starts after the work already queued on
+ * `stream`, and everything it does, the last copy into out included, is
+ * complete when `stream` reaches the point after the call; out must not be
+ * read (nor q, k, v, rpb written) by the host before then.  The call creates
+ * two CUDA streams and a few events for its copies and releases them before
+ * it returns (the release finishes when their work does); it allocates no
+ * memory and does not synchronise the host.  Errors: the argument checks of
+ * na2d_forward, with out not overlapping an input (NA2D_ERR_ALIAS), a NULL or
+ * too small workspace (NA2D_ERR_NULL / NA2D_ERR_SHAPE) and a misaligned one
+ * (NA2D_ERR_ALIGN), all before any copy; NA2D_ERR_CUDA if a CUDA call fails,
+ * after which out is unspecified. */
+NA2D_API na2d_status na2d_forward_host(const na2d_problem *p, const void *q, const void *k, const void *v,
+                                       const void *rpb, void *out, void *workspace, size_t workspace_bytes,
+                                       void *stream);
 
 /* Bytes of device workspace na2d_backward needs for problem p: fp32
  * log-sum-exp and delta per query and head (8 bytes each pair) plus an fp32

@@ -25,12 +25,14 @@ the current torch stream.  A non-OK status from the library raises
 """
 from __future__ import annotations
 
+import ctypes
+
 from ._native import (Dropout, Na2dError, Problem, Tensor, backward_workspace_size, check, device_faults, lib,  # noqa: F401
                       status_str)
 
 __all__ = ["na2d_qk_rpb", "na2d_softmax", "na2d_av", "na2d_forward", "na2d_status_str", "na2d_device_faults",
            "na2d_last_kernel", "na2d_backward", "na2d", "na2d_forward_ex", "na2d_backward_ex", "na2d_qkv_packed",
-           "Na2dError", "make_problem"]
+           "na2d_forward_host", "na2d_forward_host_workspace_size", "Na2dError", "make_problem"]
 
 # status codes used for argument errors raised before the library is called
 _ERR_NULL, _ERR_DTYPE, _ERR_SHAPE = 1, 2, 3
@@ -134,6 +136,49 @@ def na2d_forward(q, k, v, rpb, kernel_size: int, dilation: int = 1, out=None):
     ptrs = (_ptr(q), _ptr(k), _ptr(v), _ptr(rpb), _ptr(out))
     with _torch().cuda.device(q.device):
         check(lib().na2d_forward(p, *ptrs, _stream(q)), "na2d_forward")
+    return out
+
+
+def na2d_forward_host_workspace_size(shape, kernel_size: int, dilation: int = 1, dtype=None) -> int:
+    """Bytes of device workspace na2d_forward_host needs for a [B, heads, H, W, D]
+    problem of the given dtype."""
+    p = make_problem(tuple(shape), kernel_size, dilation, dtype or _torch().float16)
+    n = ctypes.c_size_t(0)
+    check(lib().na2d_forward_host_workspace_size(p, ctypes.byref(n)), "na2d_forward_host_workspace_size")
+    return n.value
+
+
+def na2d_forward_host(q, k, v, rpb, kernel_size: int, dilation: int = 1, out=None, workspace=None, device=None):
+    """na2d_forward on host (CPU) tensors: the library copies the batch to the
+    GPU in chunks, runs the forward and copies the output back, overlapping
+    the copies with the kernels.  q, k, v, rpb and out should be pinned
+    (``pin_memory()``); out is allocated pinned when not given.  workspace: a
+    CUDA uint8 tensor of at least na2d_forward_host_workspace_size() bytes,
+    allocated here when not given.  Asynchronous: out holds the result once
+    the device's current stream has passed this call."""
+    torch = _torch()
+    _check_qkv(q, kernel_size)
+    p = make_problem(q.shape, kernel_size, dilation, q.dtype)
+    for name, t in (("q", q), ("k", k), ("v", v), ("rpb", rpb), ("out", out)):
+        if t is not None and (t.device.type != "cpu" or not t.is_contiguous()):
+            raise Na2dError(_ERR_NULL, name, f"{name} must be a contiguous host (CPU) tensor")
+    _like("k", k, q)
+    _like("v", v, q)
+    _check_rpb(rpb, q, kernel_size)
+    if out is None:
+        out = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    _like("out", out, q)
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    need = na2d_forward_host_workspace_size(q.shape, kernel_size, dilation, q.dtype)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    if not workspace.is_cuda or workspace.device != dev or not workspace.is_contiguous():
+        raise Na2dError(_ERR_NULL, "workspace", f"workspace must be a contiguous CUDA tensor on {dev}")
+    nbytes = workspace.numel() * workspace.element_size()
+    host = [None if t is None else t.data_ptr() for t in (q, k, v, rpb, out)]
+    with torch.cuda.device(dev):
+        st = torch.cuda.current_stream(dev).cuda_stream
+        check(lib().na2d_forward_host(p, *host, workspace.data_ptr(), nbytes, st), "na2d_forward_host")
     return out
 
 

@@ -20,7 +20,8 @@ STATUS_NAMES = {
 # every symbol the header declares
 EXPORTS = ("na2d_qk_rpb", "na2d_softmax", "na2d_av", "na2d_forward", "na2d_device_faults", "na2d_status_str",
            "na2d_version", "na2d_last_kernel", "na2d_backward_workspace_size", "na2d_backward",
-           "na2d_backward_noalloc", "na2d_forward_ex", "na2d_backward_ex", "na2d_debug_set_wait_limit")
+           "na2d_backward_noalloc", "na2d_forward_ex", "na2d_backward_ex", "na2d_debug_set_wait_limit",
+           "na2d_forward_host_workspace_size", "na2d_forward_host")
 
 
 class Problem(ctypes.Structure):
@@ -84,6 +85,10 @@ def lib() -> ctypes.CDLL:
         L.na2d_forward_ex.restype = ctypes.c_int
         L.na2d_backward_ex.argtypes = [P, TP, TP, TP, vp, TP, TP, TP, TP, vp, DP, vp, ctypes.c_size_t, vp]
         L.na2d_backward_ex.restype = ctypes.c_int
+        L.na2d_forward_host_workspace_size.argtypes = [P, ctypes.POINTER(ctypes.c_size_t)]
+        L.na2d_forward_host_workspace_size.restype = ctypes.c_int
+        L.na2d_forward_host.argtypes = [P, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
+        L.na2d_forward_host.restype = ctypes.c_int
         L.na2d_debug_set_wait_limit.argtypes = [ctypes.c_longlong]
         L.na2d_debug_set_wait_limit.restype = None
         L.na2d_last_kernel.argtypes = []

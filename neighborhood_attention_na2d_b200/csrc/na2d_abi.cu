@@ -55,6 +55,19 @@ size_t tensor_bytes(const na2d_problem *p) {
     return (size_t)p->B * p->heads * p->H * p->W * p->D * elem_size(p->dtype);
 }
 size_t attn_bytes(const na2d_problem *p) { return (size_t)p->B * p->heads * p->H * p->W * p->k * p->k * 4; }
+// Chunks of the batch for na2d_forward_host: at most kHostChunks of cb
+// batch elements each (the last one shorter), and two workspace slots of q,
+// k, v and out (one when there is a single chunk), each tensor 256-byte
+// aligned within the workspace, then the bias table.
+constexpr int kHostChunks = 8;
+struct HostPlan {
+    int cb = 0, nchunk = 0, slots = 0;
+    size_t batch_bytes = 0;   // one batch element of one tensor
+    size_t per = 0;           // one tensor of one slot, rounded up to 256 bytes
+    size_t rpb_off = 0, ws = 0;
+};
+size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
+HostPlan host_plan(const na2d_problem *p);
 size_t rpb_bytes(const na2d_problem *p) {
     return (size_t)p->heads * (2 * p->k - 1) * (2 * p->k - 1) * elem_size(p->dtype);
 }
@@ -146,6 +159,24 @@ namespace na2d {
 void note_kernel(const char *name) { t_last_kernel = name; }
 }  // namespace na2d
 
+namespace {
+
+HostPlan host_plan(const na2d_problem *p) {
+    HostPlan h;
+    if (p->B <= 0 || p->heads <= 0) return h;
+    const int n = p->B < kHostChunks ? p->B : kHostChunks;
+    h.cb = (p->B + n - 1) / n;
+    h.nchunk = (p->B + h.cb - 1) / h.cb;
+    h.slots = h.nchunk > 1 ? 2 : 1;
+    h.batch_bytes = (size_t)p->heads * p->H * p->W * p->D * elem_size(p->dtype);
+    h.per = round256(h.batch_bytes * (size_t)h.cb);
+    h.rpb_off = 4 * (size_t)h.slots * h.per;
+    h.ws = h.rpb_off + round256(rpb_bytes(p));
+    return h;
+}
+
+}  // namespace
+
 extern "C" {
 
 na2d_status na2d_forward(const na2d_problem *p, const void *q, const void *k, const void *v, const void *rpb,
@@ -177,6 +208,84 @@ na2d_status na2d_forward(const na2d_problem *p, const void *q, const void *k, co
     return from_cuda(na2d::launch_forward_simt(pr, View::contiguous(q, pr), View::contiguous(k, pr),
                                                View::contiguous(v, pr), rpb, View::contiguous(out, pr), nullptr,
                                                Dropout{0.f, 0, 0}, st));
+}
+
+na2d_status na2d_forward_host_workspace_size(const na2d_problem *p, size_t *bytes) {
+    Problem pr;
+    bool empty = false;
+    if (!bytes) return NA2D_ERR_NULL;
+    na2d_status s = check_problem(p, &pr, &empty);
+    if (s != NA2D_OK) return s;
+    *bytes = empty ? 0 : host_plan(p).ws;
+    return NA2D_OK;
+}
+
+na2d_status na2d_forward_host(const na2d_problem *p, const void *q, const void *k, const void *v, const void *rpb,
+                              void *out, void *workspace, size_t workspace_bytes, void *stream) {
+    Problem pr;
+    bool empty = false;
+    na2d_status s = check_problem(p, &pr, &empty);
+    if (s != NA2D_OK) return s;
+    if (empty) return NA2D_OK;
+    if (!q || !k || !v || !out || !workspace) return NA2D_ERR_NULL;
+    if (!aligned16(workspace) || !rpb_aligned(p, rpb)) return NA2D_ERR_ALIGN;
+    const HostPlan h = host_plan(p);
+    if (workspace_bytes < h.ws) return NA2D_ERR_SHAPE;
+    const size_t n = tensor_bytes(p), nr = rpb ? rpb_bytes(p) : 0;
+    if (overlap(out, n, q, n) || overlap(out, n, k, n) || overlap(out, n, v, n) || overlap(out, n, rpb, nr))
+        return NA2D_ERR_ALIAS;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    unsigned char *ws = static_cast<unsigned char *>(workspace);
+    auto slot = [&](int b, int t) { return ws + (4 * (size_t)b + (size_t)t) * h.per; };   // t: q, k, v, out
+    const unsigned char *src[3] = {static_cast<const unsigned char *>(q), static_cast<const unsigned char *>(k),
+                                   static_cast<const unsigned char *>(v)};
+    unsigned char *dst = static_cast<unsigned char *>(out);
+
+    // two copy streams and the events that order them with the caller's
+    // stream; released at the end (the release completes with their work)
+    cudaStream_t s_in = nullptr, s_out = nullptr;
+    cudaEvent_t ev[8] = {};   // start, in[2], comp[2], out[2], done
+    cudaError_t e = cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking);
+    for (int i = 0; i < 8 && e == cudaSuccess; ++i) e = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming);
+    cudaEvent_t &e_start = ev[0], *e_in = ev + 1, *e_comp = ev + 3, *e_out = ev + 5, &e_done = ev[7];
+    if (e == cudaSuccess) e = cudaEventRecord(e_start, st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s_in, e_start, 0);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s_out, e_start, 0);
+    if (e == cudaSuccess && rpb)
+        e = cudaMemcpyAsync(ws + h.rpb_off, rpb, nr, cudaMemcpyHostToDevice, s_in);
+    s = NA2D_OK;
+    for (int i = 0; i < h.nchunk && e == cudaSuccess && s == NA2D_OK; ++i) {
+        const int b = i % h.slots;
+        const int bi = (i + 1) * h.cb <= p->B ? h.cb : p->B - i * h.cb;
+        const size_t off = (size_t)i * h.cb * h.batch_bytes, bytes = (size_t)bi * h.batch_bytes;
+        // the slot's inputs were read by the forward two chunks back
+        if (i >= h.slots) e = cudaStreamWaitEvent(s_in, e_comp[b], 0);
+        for (int t = 0; t < 3 && e == cudaSuccess; ++t)
+            e = cudaMemcpyAsync(slot(b, t), src[t] + off, bytes, cudaMemcpyHostToDevice, s_in);
+        if (e == cudaSuccess) e = cudaEventRecord(e_in[b], s_in);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(st, e_in[b], 0);
+        // the slot's output was copied out two chunks back
+        if (e == cudaSuccess && i >= h.slots) e = cudaStreamWaitEvent(st, e_out[b], 0);
+        if (e != cudaSuccess) break;
+        na2d_problem pc = *p;
+        pc.B = bi;
+        s = na2d_forward(&pc, slot(b, 0), slot(b, 1), slot(b, 2), rpb ? ws + h.rpb_off : nullptr, slot(b, 3), st);
+        if (s != NA2D_OK) break;
+        e = cudaEventRecord(e_comp[b], st);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(s_out, e_comp[b], 0);
+        if (e == cudaSuccess) e = cudaMemcpyAsync(dst + off, slot(b, 3), bytes, cudaMemcpyDeviceToHost, s_out);
+        if (e == cudaSuccess) e = cudaEventRecord(e_out[b], s_out);
+    }
+    // the caller's stream passes the call's end only after the last copy out
+    if (e == cudaSuccess && s == NA2D_OK) e = cudaEventRecord(e_done, s_out);
+    if (e == cudaSuccess && s == NA2D_OK) e = cudaStreamWaitEvent(st, e_done, 0);
+    for (int i = 0; i < 8; ++i)
+        if (ev[i]) cudaEventDestroy(ev[i]);
+    if (s_in) cudaStreamDestroy(s_in);
+    if (s_out) cudaStreamDestroy(s_out);
+    if (s != NA2D_OK) return s;
+    return from_cuda(e);
 }
 
 na2d_status na2d_forward_ex(const na2d_problem *p, const na2d_tensor *q, const na2d_tensor *k,

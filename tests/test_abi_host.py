@@ -106,6 +106,19 @@ def _host_checks() -> dict:
     r["fx_fused_clash"] = L.na2d_forward_ex(ctypes.byref(p), ctypes.byref(T(base, **P3)),
                                             ctypes.byref(T(base + 128, **P3)), ctypes.byref(T(base + 256, **P3)),
                                             None, ctypes.byref(T(base + 192, **P3)), None, None, None)
+    # the host-buffer forward: workspace and alias checks before any copy
+    ws = ctypes.c_size_t(0)
+    L.na2d_forward_host_workspace_size(ctypes.byref(p), ctypes.byref(ws))
+    r["fh_ws_size"] = ws.value
+    big = 1 << 24
+    r["fh_null_ws"] = L.na2d_forward_host(ctypes.byref(p), FAKE, FAKE, FAKE, None, FAKE2, None, big, None)
+    r["fh_align_ws"] = L.na2d_forward_host(ctypes.byref(p), FAKE, FAKE, FAKE, None, FAKE2, FAKE + 8, big, None)
+    r["fh_small_ws"] = L.na2d_forward_host(ctypes.byref(p), FAKE, FAKE, FAKE, None, FAKE2, FAKE, ws.value - 16,
+                                           None)
+    r["fh_alias"] = L.na2d_forward_host(ctypes.byref(p), FAKE, FAKE2, FAKE2, None, FAKE + 64, FAKE, big, None)
+    r["fh_null_q"] = L.na2d_forward_host(ctypes.byref(p), None, FAKE, FAKE, None, FAKE2, FAKE, big, None)
+    r["fh_bad_k"] = L.na2d_forward_host(ctypes.byref(prob(k=6)), FAKE, FAKE, FAKE, None, FAKE2, FAKE, big, None)
+    r["fh_empty"] = L.na2d_forward_host(ctypes.byref(prob(B=0)), FAKE, FAKE, FAKE, None, FAKE2, None, 0, None)
     return r
 
 
@@ -125,6 +138,13 @@ def test_fused_views_pass_the_host_checks(host_results):
     check; with no device the call then fails only at the launch
     (NA2D_ERR_CUDA), never with an argument error."""
     assert host_results["fx_fused_ok"] == 8
+
+
+def test_forward_host_workspace_size(host_results):
+    """B=2 heads=2 14x14 D=32 f16: two chunks of one batch element, two slots of
+    q, k, v and out (25,088 bytes each, already a multiple of 256) and the
+    676-byte bias table rounded up to 768."""
+    assert host_results["fh_ws_size"] == 8 * 2 * 14 * 14 * 32 * 2 + 768
 
 
 def test_backward_workspace_size(host_results):
@@ -173,6 +193,8 @@ def test_forward_rejects_bad_problems(host_results, i):
     ("bwd_alias_out", 7), ("bwd_alias_ws", 7), ("bwd_bad_k", 4), ("bwd_empty", 0),
     ("fx_null", 1), ("fx_stride_align", 6), ("fx_neg_stride", 6), ("fx_out_self_overlap", 7), ("fx_out_on_input", 7),
     ("fx_attn_on_input", 7), ("fx_drop_p", 3), ("fx_drop_neg", 3), ("fx_empty", 0), ("fx_fused_clash", 7),
+    ("fh_null_ws", 1), ("fh_align_ws", 6), ("fh_small_ws", 3), ("fh_alias", 7), ("fh_null_q", 1), ("fh_bad_k", 4),
+    ("fh_empty", 0),
 ])
 def test_host_checks(host_results, case, status):
     assert host_results[case] == status

@@ -263,6 +263,49 @@ def test_output_only_16_byte_aligned(shape, kernel):
     assert err <= TOL[shape.dtype], f"{shape.describe()}: max abs err {err}"
 
 
+@pytest.mark.parametrize("shape,pinned,with_rpb", [
+    (Shape(5, 2, 28, 28, 32, 7, 1, "f16", 7501), True, True),     # 5 chunks of one batch element
+    (Shape(9, 2, 56, 56, 32, 7, 8, "bf16", 7502), True, True),    # chunks of 2, the last one of 1
+    (Shape(3, 2, 14, 14, 32, 5, 2, "f32", 7503), False, False),   # pageable buffers, no bias
+    (Shape(1, 4, 32, 32, 32, 13, 2, "bf16", 7504), True, True),   # a single chunk
+], ids=lambda x: x.describe() if isinstance(x, Shape) else str(x))
+def test_forward_on_host_buffers(shape, pinned, with_rpb):
+    """na2d_forward_host: host tensors in, host tensor out, the batch pipelined
+    through the device in chunks; every element matches the oracle and the
+    device-buffer forward of the same inputs."""
+    q, k, v, rpb = make_inputs(shape)
+    if not with_rpb:
+        rpb = None
+    host = [None if t is None else (t.pin_memory() if pinned else t.clone()) for t in (q, k, v, rpb)]
+    out = torch.full(q.shape, SENTINEL, dtype=q.dtype)
+    out = out.pin_memory() if pinned else out
+    na.na2d_forward_host(*host, shape.k, shape.d, out=out)
+    torch.cuda.current_stream().synchronize()
+    want = oracle.forward(f64(q), f64(k), f64(v), f64(rpb), shape.k, shape.d)
+    err = max_err(out.double().numpy(), want)
+    assert err <= TOL[shape.dtype], f"{shape.describe()}: max abs err {err}"
+    dev = na.na2d_forward(q.cuda(), k.cuda(), v.cuda(), None if rpb is None else rpb.cuda(), shape.k, shape.d)
+    torch.cuda.synchronize()
+    assert float((out.double() - dev.double().cpu()).abs().max()) <= TOL[shape.dtype]
+
+
+def test_forward_on_host_buffers_back_to_back():
+    """Calls queued back to back on one stream (the host does not wait in
+    between) each see their own inputs and write their own outputs."""
+    shape = Shape(6, 2, 28, 28, 32, 7, 1, "f16", 7510)
+    sets = [make_inputs(shape, shape.seed + i) for i in range(3)]
+    pinned = [[t.pin_memory() for t in s] for s in sets]
+    outs = [torch.empty(sets[0][0].shape, dtype=torch.float16).pin_memory() for _ in sets]
+    ws = torch.empty(na.na2d_forward_host_workspace_size(sets[0][0].shape, 7, 1, torch.float16),
+                     dtype=torch.uint8, device="cuda")
+    for (q, k, v, rpb), o in zip(pinned, outs):
+        na.na2d_forward_host(q, k, v, rpb, 7, 1, out=o, workspace=ws)
+    torch.cuda.current_stream().synchronize()
+    for (q, k, v, rpb), o in zip(sets, outs):
+        want = oracle.forward(f64(q), f64(k), f64(v), f64(rpb), 7, 1)
+        assert max_err(o.double().numpy(), want) <= TOL["f16"]
+
+
 def test_misaligned_tensor_is_rejected():
     q = torch.zeros(2 * 14 * 14 * 32 + 4, dtype=torch.float16, device="cuda")[4:].view(1, 2, 14, 14, 32)
     with pytest.raises(na.Na2dError) as e:
