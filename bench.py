@@ -173,6 +173,17 @@ def dist_setup(args):
     return world, rank, local
 
 
+def max_over_ranks(x: float, pg, dev) -> float:
+    """The largest of every rank's x (every rank calls this at the same point,
+    so all of them take the same collective steps); x itself on one rank."""
+    if not pg:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
 def run_reference(args, world, rank):
     """The oracle on host cores, per step a bounded sample of the workload."""
     if rank != 0:
@@ -332,11 +343,7 @@ def time_steps(wl, sets, K, warmup, dev, pg=None, min_seconds=0.25, min_runs=5, 
                     graphs[1].replay()
                 end.record(stream)
                 end.synchronize()
-                ms = start.elapsed_time(end)
-                if pg:
-                    t = torch.tensor([ms], device=dev)
-                    pg.all_reduce(t, op=pg.ReduceOp.MAX)
-                    ms = float(t.item())
+                ms = max_over_ranks(start.elapsed_time(end), pg, dev)
                 runs.append(ms)
                 t_total += ms
                 if len(runs) >= 10000:
@@ -672,11 +679,7 @@ def run_e2e(args, wl, dev, rank, world, pg):
         step()
     b.record(stream)
     b.synchronize()
-    ms = a.elapsed_time(b)
-    if pg:
-        t = torch.tensor([ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(a.elapsed_time(b), pg, dev)
     units = world * sum(s.B * s.heads * s.H * s.W for s in wl.shapes)
     return {"value": units / (ms / n / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "steps": n, "api": "neighborhood_attention_na2d_b200.na2d_forward_host (C ABI na2d_forward_host: "
