@@ -147,6 +147,27 @@ def test_forward_host_workspace_size(host_results):
     assert host_results["fh_ws_size"] == 8 * 2 * 14 * 14 * 32 * 2 + 768
 
 
+@pytest.mark.parametrize("B", [1, 2, 7, 8, 9, 16, 33, 100])
+def test_forward_host_workspace_size_chunks(B):
+    """The host-buffer forward's workspace for a range of batches: at most 8
+    chunks of ceil(B / min(B, 8)) batch elements, two slots of q, k, v and
+    out (one slot for a single chunk), each rounded up to 256 bytes, then the
+    bias table rounded up to 256 bytes.  Host-only: no CUDA call."""
+    import ctypes
+    build()
+    heads, H, W, D, k = 3, 10, 9, 32, 5
+    p = prob(B=B, heads=heads, H=H, W=W, D=D, k=k)
+    n = ctypes.c_size_t(0)
+    assert _native.lib().na2d_forward_host_workspace_size(ctypes.byref(p), ctypes.byref(n)) == 0
+    cb = -(-B // min(B, 8))
+    nchunk = -(-B // cb)
+    slots = 2 if nchunk > 1 else 1
+    r256 = lambda x: -(-x // 256) * 256
+    per = r256(cb * heads * H * W * D * 2)
+    assert nchunk <= 8
+    assert n.value == 4 * slots * per + r256(heads * (2 * k - 1) ** 2 * 2)
+
+
 def test_backward_workspace_size(host_results):
     """[lse, delta] fp32 per query and head plus the fp32 bias table."""
     assert host_results["ws_bytes"] == (2 * 2 * 2 * 14 * 14 + 2 * 13 * 13) * 4
